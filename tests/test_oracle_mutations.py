@@ -1,0 +1,112 @@
+"""Planted mistakes: each plausible slip in the oracle must fail a pin.
+
+Every case rewrites one oracle function (on the CPU, in this process only),
+runs the pins that should notice, and checks that at least one of them fails.
+"""
+import contextlib
+import inspect
+import textwrap
+
+import numpy as np
+import pytest
+
+import oracle
+import oracle.bifocal_ref as ref
+import test_oracle_pins as pins
+
+
+@contextlib.contextmanager
+def mutated(func_name, old, new):
+    src = textwrap.dedent(inspect.getsource(getattr(ref, func_name)))
+    assert old in src, (func_name, old)
+    ns = dict(ref.__dict__)
+    exec(compile(src.replace(old, new, 1), f"<mutant {func_name}>", "exec"), ns)
+    saved_ref = getattr(ref, func_name)
+    saved_pkg = getattr(oracle, func_name, None)
+    setattr(ref, func_name, ns[func_name])
+    setattr(oracle, func_name, ns[func_name])
+    try:
+        yield
+    finally:
+        setattr(ref, func_name, saved_ref)
+        if saved_pkg is not None:
+            setattr(oracle, func_name, saved_pkg)
+
+
+def some_pin_fails(tests):
+    for t in tests:
+        try:
+            t()
+        except AssertionError:
+            return True
+    return False
+
+
+PREFILL_PINS = [
+    pins.test_native_window_reduces_to_plain_rope_attention,
+    pins.test_wide_window_equals_true_position_attention,
+    pins.test_zero_window_equals_remote_position_attention,
+    pins.test_rows_inside_local_window_see_true_positions,
+    pins.test_band_and_remote_parts_via_masked_library_attention,
+    pins.test_literal_per_pair_brute_force,
+    pins.test_grouped_query_heads_share_kv_heads_in_blocks,
+]
+
+
+def decode_pins():
+    return [lambda L=L: pins.test_decode_equals_last_prefill_row(L) for L in (129, 300, 512)] + [
+        pins.test_decode_group_transition_page_boundary]
+
+
+MUTANTS = [
+    # schedule
+    ("group_size", "max(1, -((-L) // w))", "max(1, L // w)",
+     [pins.test_group_size_matches_page_values, pins.test_group_size_is_minimal_integer_compression]),
+    ("group_size", "max(1, -((-L) // w))", "max(1, -((-L) // w) + (L % w == 0))",
+     [pins.test_group_size_matches_page_values]),
+    ("remap", "np.floor_divide(np.asarray(x, dtype=np.int64), int(G))",
+     "-np.floor_divide(-np.asarray(x, dtype=np.int64), int(G))",
+     [pins.test_remap_identity_iff_native_and_monotone] + PREFILL_PINS),
+    # RoPE
+    ("rope", "a * c - b * s, a * s + b * c", "a * c + b * s, -a * s + b * c",
+     [pins.test_rope_matches_complex_rotation]),
+    ("rope", "a * c - b * s, a * s + b * c", "a * c - b * s, b * s + a * c",
+     [pins.test_rope_matches_complex_rotation, pins.test_rope_norm_identity_and_composition]),
+    ("inv_freq", "-2.0 * i / np.float64(D)", "-2.0 * (i + 1) / np.float64(D)",
+     [pins.test_rope_matches_complex_rotation]),
+    ("inv_freq", "-2.0 * i / np.float64(D)", "-1.0 * i / np.float64(D)",
+     [pins.test_rope_matches_complex_rotation]),
+    # score rule
+    ("prefill_rows", "dist <= w0", "dist < w0", PREFILL_PINS),
+    ("prefill_rows", "np.where(dist <= w0, s_local, s_remote)", "np.where(dist <= w0, s_remote, s_local)",
+     PREFILL_PINS),
+    ("prefill_rows", "n = i + 1", "n = i if i > 0 else 1", PREFILL_PINS),
+    ("prefill_rows", "scale = 1.0 / math.sqrt(D)", "scale = 1.0 / D", PREFILL_PINS),
+    ("prefill_rows", "q_remote = rope(xq, remap(np.int64(i), G), theta)",
+     "q_remote = rope(xq, np.int64(i), theta)", PREFILL_PINS),
+    ("prefill_rows", "heads = np.arange(g * grp, (g + 1) * grp)",
+     "heads = np.arange(g, Hq, Hkv)", PREFILL_PINS),
+    ("prefill_rows", "lse[b, heads, r] = m + np.log(tot)", "lse[b, heads, r] = np.log(tot)",
+     PREFILL_PINS),
+    # decode / correction
+    ("correction_rotate", "delta = remap(kpos, G) - kpos", "delta = kpos - remap(kpos, G)",
+     [pins.test_correction_rotation_recovers_remote_phase] + decode_pins()),
+    ("decode", "    p = L - 1\n", "    p = L\n", decode_pins()),
+    ("decode", "local = (p - jpos) <= w0", "local = (p - jpos) < w0", decode_pins()),
+    ("decode", "q_remote = rope(q[b, heads], remap(np.int64(p), G), theta)",
+     "q_remote = rope(q[b, heads], np.int64(p), theta)", decode_pins()),
+    ("rope_cache", "+ int(pos0)", "+ int(pos0) + 1", [pins.test_rope_cache_offset] + decode_pins()),
+]
+
+
+@pytest.mark.parametrize("case", range(len(MUTANTS)))
+def test_planted_mistake_is_caught(case):
+    name, old, new, tests = MUTANTS[case]
+    with mutated(name, old, new):
+        assert some_pin_fails(tests), f"mutant of {name} ({new!r}) passed every pin"
+
+
+def test_unmutated_oracle_passes_the_same_pins():
+    for _, _, _, tests in MUTANTS:
+        for t in tests:
+            t()
