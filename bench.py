@@ -1,0 +1,438 @@
+#!/usr/bin/env python3
+"""Benchmark of the bifocal-RoPE attention hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl native|reference]
+
+One step = one prefill of a Qwen3-8B-shaped attention layer at L = 131072
+(B=1, Hq=32, Hkv=8, D=128, w_pretrained=32768, w0=4096, theta=1e6, G=4):
+the RoPE operand pass (jetlong_prefill_rotate) followed by the attention
+kernel (jetlong_prefill_attend), with inputs resident in HBM.  The headline
+``value`` is algorithmic prefill TFLOP/s = 4 * B * Hq * D * L(L+1)/2 / time.
+After the prefill steps, 256 decode steps on a 131072-token true-position
+cache (Qwen3-8B shapes) are timed the same way and reported as microseconds
+per token and achieved HBM bandwidth over the K+V bytes a step must read.
+
+Every input is synthetic and seeded (zero_shot_rope_bifocal_b200.synth);
+each is larger than the 126 MB L2 (q alone is 1 GiB), so no flush is needed
+between steps.  Under torchrun each rank runs its own independent layer
+(different seed): weak scaling, no collective in the data path; rank 0 prints
+the JSON line with the max-over-ranks time and the summed work.
+
+``--impl reference`` times the fp64 CPU oracle on the host's cores instead,
+on a bounded sample of query rows of the same workload, in the same unit.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+PREFILL_WORKLOAD = "qwen3_8b_128k"
+DECODE_WORKLOAD = "decode_8b_128k"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+NOMINAL = {"hbm_gbs": 8000.0, "bf16_tflops": 2250.0}
+
+
+# ---------------------------------------------------------------- accounting
+def prefill_flops(B: int, Hq: int, L: int, D: int) -> int:
+    """Algorithmic FLOPs: every causal pair gets one Q.K dot (2D) and one P.V axpy (2D)."""
+    return 4 * B * Hq * D * (L * (L + 1) // 2)
+
+
+def row_flops(Hq: int, D: int, rows) -> int:
+    return sum(4 * Hq * D * (int(i) + 1) for i in rows)
+
+
+def decode_bytes(B: int, Hkv: int, L: int, D: int) -> int:
+    """K and V BF16 bytes one decode step must stream."""
+    return 2 * B * L * Hkv * D * 2
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as fh:
+            d = json.load(fh)
+        return {k: float(d[k]) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")}, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ---------------------------------------------------------------- ranks
+def dist_env():
+    return int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")), \
+        int(os.environ.get("LOCAL_RANK", "0"))
+
+
+def reduce_max(x: float, world: int, device=None) -> float:
+    """Max over ranks (host plumbing for the timing report)."""
+    if world == 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def reduce_sum(x: float, world: int, device=None) -> float:
+    if world == 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    """Samples SM clocks and throttle reasons with nvidia-smi while running."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            if self.thread is not None:
+                self.thread.join(timeout=2)
+
+    def summary(self):
+        if not self.lines:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- oracle timing
+def oracle_rows_per_sec(w, seconds: float, q_rows_src, k, v, rows):
+    """Time the CPU oracle on query rows of workload ``w`` for about ``seconds``.
+
+    Returns (flops_done, elapsed, rows_done)."""
+    import oracle
+    import torch
+    done_rows, flops, t0 = [], 0, time.perf_counter()
+    for i, r in enumerate(rows):
+        q1 = q_rows_src[:, i:i + 1]
+        oracle.prefill_rows(q1, k, v, w.w_pretrained, w.w0, w.theta, [r], q_holds_rows=True)
+        done_rows.append(r)
+        flops += row_flops(w.Hq, w.D, [r])
+        if time.perf_counter() - t0 >= seconds:
+            break
+    return flops, time.perf_counter() - t0, done_rows
+
+
+def cpu_sample_inputs(w, n_rows: int, device):
+    """Inputs of ``w`` for oracle timing: the query rows to time and K/V as fp32 numpy."""
+    import numpy as np
+    import torch
+    from zero_shot_rope_bifocal_b200.synth import prefill_inputs, sample_rows
+    x = prefill_inputs(w, device=device)
+    g = torch.Generator().manual_seed(1234)
+    rows = sorted(torch.randint(w.L // 2, w.L, (n_rows,), generator=g).tolist())
+    ridx = torch.tensor(rows, device=x.q.device)
+    q_rows = x.q.index_select(1, ridx).to("cpu", torch.float32).numpy()
+    k = x.k.to("cpu", torch.float32).numpy()
+    v = x.v.to("cpu", torch.float32).numpy()
+    del x
+    return q_rows, k, v, rows
+
+
+def threads_used() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [d.get("num_threads", 1) for d in threadpool_info() if d.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+# ---------------------------------------------------------------- reference arm
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    from zero_shot_rope_bifocal_b200.synth import WORKLOADS
+    w = WORKLOADS[PREFILL_WORKLOAD]
+    q_rows, k, v, rows = cpu_sample_inputs(w, 64, "cpu")
+    per_step = max(2.0, args.reference_seconds / max(1, args.steps + args.warmup))
+    for _ in range(args.warmup):
+        oracle_rows_per_sec(w, per_step, q_rows, k, v, rows)
+    tot_f, tot_t, nrows = 0, 0.0, 0
+    for s in range(args.steps):
+        rot = rows[s % len(rows):] + rows[:s % len(rows)]
+        qrot = q_rows[:, [rows.index(r) for r in rot]]
+        f, t, done = oracle_rows_per_sec(w, per_step, qrot, k, v, rot)
+        tot_f, tot_t, nrows = tot_f + f, tot_t + t, nrows + len(done)
+    value = tot_f / tot_t / 1e12
+    line = {
+        "impl": "reference", "metric": "bifocal-attn prefill TFLOP/s @128K (Qwen3-8B layer)",
+        "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": 1e3 * tot_t / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded N(0,1) Q/K/V, K per-channel LogNormal(0,0.5) scale)",
+        "config": {"workload": PREFILL_WORKLOAD, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D,
+                   "L": w.L, "w_pretrained": w.w_pretrained, "w0": w.w0, "rope_theta": w.theta},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads_used(),
+                         "kind": "oracle",
+                         "sample": f"{nrows} query rows (all 32 heads) of the 128K prefill, "
+                                   f"random rows in [L/2, L), ~{per_step:.0f} s per step"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------- native arm
+def run_native(args):
+    import torch
+    import torch.distributed as dist
+    from zero_shot_rope_bifocal_b200 import jetlong as jl
+    from zero_shot_rope_bifocal_b200.synth import WORKLOADS, decode_inputs, prefill_inputs
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=dev)
+    jl.lib()  # fail loudly if the library is missing
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    w = WORKLOADS[PREFILL_WORKLOAD].with_(seed=WORKLOADS[PREFILL_WORKLOAD].seed + 100 * rank)
+    x = prefill_inputs(w, device=dev)
+    B, L, Hq, Hkv, D = w.B, w.L, w.Hq, w.Hkv, w.D
+    out = torch.empty((B, L, Hq, D), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((B, Hq, L), dtype=torch.float32, device=dev)
+    ws = torch.empty(jl.jetlong_prefill_workspace_size(B, Hq, Hkv, L, D), dtype=torch.uint8,
+                     device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(ev_mid=None, ev_end=None):
+        jl.jetlong_prefill_rotate(x.q, x.k, w.w_pretrained, w.theta, ws, stream=stream)
+        if ev_mid is not None:
+            ev_mid.record(stream)
+        jl.jetlong_prefill_attend(x.v, out, lse, Hq, w.w_pretrained, w.w0, ws, stream=stream)
+        if ev_end is not None:
+            ev_end.record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    if jl.jetlong_device_status() != jl.JL_OK:
+        raise RuntimeError("device status not OK after warm-up")
+
+    ev0 = torch.cuda.Event(enable_timing=True)
+    ev1 = torch.cuda.Event(enable_timing=True)
+    mids = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    with ClockSampler(local) as clocks:
+        barrier()
+        torch.cuda.synchronize(dev)
+        ev0.record(stream)
+        for s in range(args.steps):
+            step(mids[s], ends[s])
+        ev1.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier()
+    t_ms = ev0.elapsed_time(ev1)
+    attn_ms = sum(mids[s].elapsed_time(ends[s]) for s in range(args.steps)) / args.steps
+    rot_ms = (t_ms - attn_ms * args.steps) / args.steps
+    if jl.jetlong_device_status() != jl.JL_OK:
+        raise RuntimeError("device status not OK after timing")
+    t_max = reduce_max(t_ms, world, dev)
+    flops_rank = prefill_flops(B, Hq, L, D) * args.steps
+    flops_all = reduce_sum(flops_rank, world, dev)
+    value = flops_all / (t_max * 1e-3) / 1e12
+
+    # ---- decode: 256 steps on a 128K true-position cache
+    wd = WORKLOADS[DECODE_WORKLOAD].with_(seed=WORKLOADS[DECODE_WORKLOAD].seed + 100 * rank)
+    d = decode_inputs(wd, device=dev)
+    kc = torch.empty_like(d.k_raw)
+    jl.jetlong_rope_cache(d.k_raw, kc, 0, wd.theta, stream=stream)
+    del d.k_raw
+    dq = d.q
+    dout = torch.empty((wd.B, wd.Hq, wd.D), dtype=torch.bfloat16, device=dev)
+    dlse = torch.empty((wd.B, wd.Hq), dtype=torch.float32, device=dev)
+    dws = torch.empty(jl.jetlong_decode_workspace_size(wd.B, wd.Hq, wd.Hkv, wd.L, wd.D),
+                      dtype=torch.uint8, device=dev)
+
+    def dstep():
+        jl.jetlong_decode(dq, kc, d.v, wd.L, wd.w_pretrained, wd.w0, wd.theta, out=dout, lse=dlse,
+                          workspace=dws, stream=stream)
+
+    for _ in range(max(3, args.warmup)):
+        dstep()
+    n_dec = args.decode_steps
+    with ClockSampler(local) as dclocks:
+        barrier()
+        torch.cuda.synchronize(dev)
+        ev0.record(stream)
+        for _ in range(n_dec):
+            dstep()
+        ev1.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier()
+    dec_ms = reduce_max(ev0.elapsed_time(ev1), world, dev)
+    if jl.jetlong_device_status() != jl.JL_OK:
+        raise RuntimeError("device status not OK after decode timing")
+    us_tok = 1e3 * dec_ms / n_dec
+    dec_gbs = decode_bytes(wd.B, wd.Hkv, wd.L, wd.D) / (us_tok * 1e-6) / 1e9
+
+    # ---- end to end through the public API from pinned host buffers
+    hq = x.q.cpu().pin_memory()
+    hk = x.k.cpu().pin_memory()
+    hv = x.v.cpu().pin_memory()
+    hout = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    hlse = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+    dq2, dk2, dv2 = torch.empty_like(x.q), torch.empty_like(x.k), torch.empty_like(x.v)
+    del x
+
+    def e2e_step():
+        dq2.copy_(hq, non_blocking=True)
+        dk2.copy_(hk, non_blocking=True)
+        dv2.copy_(hv, non_blocking=True)
+        jl.jetlong_prefill(dq2, dk2, dv2, w.w_pretrained, w.w0, w.theta, out=out, lse=lse,
+                           workspace=ws, stream=stream)
+        hout.copy_(out, non_blocking=True)
+        hlse.copy_(lse, non_blocking=True)
+
+    e2e_step()
+    n_e2e = max(1, min(args.steps, 3))
+    barrier()
+    torch.cuda.synchronize(dev)
+    ev0.record(stream)
+    for _ in range(n_e2e):
+        e2e_step()
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    e2e_ms = reduce_max(ev0.elapsed_time(ev1), world, dev) / n_e2e
+    e2e_val = reduce_sum(prefill_flops(B, Hq, L, D), world, dev) / (e2e_ms * 1e-3) / 1e12
+    h2d = (hq.numel() + hk.numel() + hv.numel()) * 2
+    d2h = hout.numel() * 2 + hlse.numel() * 4
+
+    # ---- CPU oracle baseline (rank 0, N=1 only)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        q_rows, kk, vv, rows = cpu_sample_inputs(w, 64, dev)
+        f, t, done = oracle_rows_per_sec(w, args.cpu_seconds, q_rows, kk, vv, rows)
+        cpu = {"value": f / t / 1e12, "unit": "TFLOP/s", "cores": threads_used(), "kind": "oracle",
+               "sample": f"{len(done)} query rows (all 32 heads) of the 128K prefill, random rows "
+                         f"in [L/2, L), {t:.1f} s of fp64 NumPy"}
+
+    if rank == 0:
+        peaks, src = load_peaks()
+        attn_tflops = prefill_flops(B, Hq, L, D) / (attn_ms * 1e-3) / 1e12
+        peak = peaks["bf16_tflops_sustained"]
+        line = {
+            "metric": "bifocal-attn prefill TFLOP/s @128K (Qwen3-8B layer); decode us/token",
+            "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": t_max / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded N(0,1) Q/K/V, K per-channel LogNormal(0,0.5) scale)",
+            "config": {"workload": PREFILL_WORKLOAD, "B": B, "Hq": Hq, "Hkv": Hkv, "D": D, "L": L,
+                       "w_pretrained": w.w_pretrained, "w0": w.w0, "rope_theta": w.theta,
+                       "G": jl.jetlong_group_size(L, w.w_pretrained),
+                       "l2": "inputs larger than L2 (q 1 GiB, k/v 256 MiB each); no flush",
+                       "parallelism": f"independent layer per rank x{world}"},
+            "roofline": {"bound": "tensor", "achieved": attn_tflops, "peak": peak,
+                         "unit": "TFLOP/s", "frac": attn_tflops / peak,
+                         "peak_source": f"{src} bf16_tflops_sustained",
+                         "nominal_frac": attn_tflops / NOMINAL["bf16_tflops"],
+                         "kernel": "bifocal_prefill_kernel<128>", "kernel_ms": attn_ms,
+                         "traffic": None},
+            "breakdown_ms": {"rotate": rot_ms, "attend": attn_ms},
+            "decode": {"workload": DECODE_WORKLOAD, "us_per_token": us_tok, "steps": n_dec,
+                       "achieved_gbs": dec_gbs, "peak_gbs": peaks["hbm_gbs"],
+                       "frac": dec_gbs / peaks["hbm_gbs"],
+                       "nominal_frac": dec_gbs / NOMINAL["hbm_gbs"],
+                       "bytes_per_token": decode_bytes(wd.B, wd.Hkv, wd.L, wd.D),
+                       "clocks": dclocks.summary()},
+            "e2e": {"value": e2e_val, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+            "gpu_launches": 2 * args.steps + 2 * n_dec,
+            "clocks": clocks.summary(),
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["native", "reference"], default="native")
+    ap.add_argument("--decode-steps", type=int, default=256)
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--reference-seconds", type=float, default=120.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    args.warmup = max(3, args.warmup)  # at least three untimed warm-up steps
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_native(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

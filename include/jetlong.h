@@ -1,0 +1,195 @@
+/*
+ * jetlong.h -- C ABI of the B200 (sm_100a) bifocal-RoPE attention library.
+ *
+ * The operation is the attention of "Jet-Long: Efficient Long-Context Extension
+ * with Dynamic Bifocal RoPE":
+ *
+ *   - schedule (§3.1, Eq. (2)):  G = max(1, ceil(L / w_pretrained)),
+ *                                f(x) = floor(x / G)   (identity when L <= w_pretrained);
+ *   - score rule (§3, display equation of S(q, k)), for query i and key j <= i:
+ *         i - j <= w0 :  S = RoPE(x_q, i)    . RoPE(x_k, j)
+ *         i - j >  w0 :  S = RoPE(x_q, f(i)) . RoPE(x_k, f(j))
+ *     scaled by 1/sqrt(D), softmax over j <= i (causal);
+ *   - the two windows are merged as in §3.3 (inclusion-exclusion of three
+ *     attention passes); the kernels compute the same sum in one online
+ *     softmax that picks the score of each pair by the rule above;
+ *   - KV cache (§3.2): keys are stored once, rotated to their true positions,
+ *     k_cache[k] = RoPE(x_k, k); decode applies the correction rotation by
+ *     Delta k = f(k) - k on the fly and never rewrites the cache.
+ *
+ * RoPE pairs channel i with channel i + D/2 and rotates the pair by the angle
+ * p * theta^(-2i/D); angles are formed in double precision and reduced before
+ * the sine/cosine, so positions up to 2^31 keep full accuracy.
+ *
+ * Conventions shared by every entry point
+ *   - Positions are 0-based.  The decode query of a cache holding L tokens
+ *     (the new one included) sits at position L - 1.
+ *   - Tensors are dense, row-major (last index fastest), BF16 unless noted,
+ *     in device memory.  Layouts are given as [dim0, dim1, ...].
+ *   - GQA: query head h reads KV head h / (Hq / Hkv).
+ *   - Supported head dims: D = 64 or 128.  Hq must be a multiple of Hkv.
+ *   - Device pointers must be 16-byte aligned.
+ *   - Ownership: the caller owns every buffer; the library keeps no buffer and
+ *     performs no device allocation.  Scratch space is passed in as a
+ *     caller-owned workspace whose size the *_workspace_size functions return.
+ *   - Execution: asynchronous on `stream` (NULL = the legacy default stream) on
+ *     the current CUDA device.  Arguments are validated on the host before
+ *     anything is launched; a call that returns an error launched nothing.
+ *   - Errors are returned as jl_status codes, never thrown.  JL_ERR_CUDA means
+ *     a launch failed (see cudaGetLastError for the CUDA code).  Every wait
+ *     inside a kernel is bounded in time; a wait that gives up records
+ *     JL_ERR_DEVICE_TIMEOUT, which jetlong_device_status() reports.
+ *   - Calls on different streams may run concurrently as long as they do not
+ *     share output or workspace buffers.
+ */
+#ifndef JETLONG_H
+#define JETLONG_H
+
+#include <stddef.h>
+
+#if defined(__GNUC__)
+#define JL_API __attribute__((visibility("default")))
+#else
+#define JL_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ABI-identical to cudaStream_t; NULL selects the legacy default stream. */
+typedef struct CUstream_st *jl_stream_t;
+
+typedef enum {
+  JL_OK = 0,
+  JL_ERR_NULL = -1,            /* a required pointer is NULL                        */
+  JL_ERR_SHAPE = -2,           /* a size is out of range or inconsistent            */
+  JL_ERR_UNSUPPORTED = -3,     /* valid but not implemented (e.g. D not 64/128)     */
+  JL_ERR_ALIGN = -4,           /* a pointer is not 16-byte aligned                  */
+  JL_ERR_WORKSPACE = -5,       /* workspace NULL or smaller than required           */
+  JL_ERR_CUDA = -6,            /* a CUDA runtime / launch error                     */
+  JL_ERR_DEVICE_TIMEOUT = -7,  /* a bounded in-kernel wait expired (device report)  */
+  JL_ERR_NO_DEVICE = -8        /* no sm_100 device is current                       */
+} jl_status;
+
+typedef enum { JL_BF16 = 0, JL_F32 = 1 } jl_dtype;
+
+/* Human-readable name of a status code (static string, never NULL). */
+JL_API const char *jetlong_status_string(int status);
+
+/* Library version as "major.minor.patch" (static string). */
+JL_API const char *jetlong_version(void);
+
+/*
+ * Dynamic group size of §3.1, Eq. (2): G = max(1, ceil(L / w_pretrained)).
+ * Host only, no CUDA call.  Returns G >= 1, or JL_ERR_SHAPE if L < 1 or
+ * w_pretrained < 1.
+ */
+JL_API int jetlong_group_size(int L, int w_pretrained);
+
+/*
+ * Bytes of workspace jetlong_prefill needs for these sizes (host only).
+ * Returns 0 if a size is invalid.
+ */
+JL_API size_t jetlong_prefill_workspace_size(int B, int Hq, int Hkv, int L, int D);
+
+/*
+ * Bifocal causal attention over a whole prompt (prefill).  One G for the call,
+ * from the prompt length L (§3.1).
+ *
+ *   q   [B, L, Hq,  D] BF16, pre-RoPE queries           (read)
+ *   k   [B, L, Hkv, D] BF16, pre-RoPE keys              (read)
+ *   v   [B, L, Hkv, D] BF16, values                     (read)
+ *   out [B, L, Hq,  D] out_dtype (JL_BF16 or JL_F32)    (written)
+ *   lse [B, Hq, L] float32, natural-log log-sum-exp of the scaled scores per
+ *       row (written; may be NULL)
+ *   w_pretrained >= 1, w0 >= 0, rope_theta > 0.
+ *   k_cache_out: NULL, or [B, k_cache_capacity, Hkv, D] BF16; rows [0, L) are
+ *       written with RoPE(x_k, k) at true positions (§3.2), the cache decode
+ *       expects.  k_cache_capacity >= L (ignored when k_cache_out is NULL).
+ *   workspace: device buffer of at least jetlong_prefill_workspace_size(...)
+ *       bytes, 256-byte aligned; contents on entry do not matter.
+ *
+ * Returns JL_OK or an error code (nothing launched on error).
+ */
+JL_API int jetlong_prefill(const void *q, const void *k, const void *v, void *out, float *lse,
+                    int B, int Hq, int Hkv, int L, int D,
+                    int w_pretrained, int w0, float rope_theta, int out_dtype,
+                    void *k_cache_out, int k_cache_capacity,
+                    void *workspace, size_t workspace_bytes, jl_stream_t stream);
+
+/*
+ * The two stages of jetlong_prefill, for callers that schedule them apart
+ * (e.g. to time the attention kernel alone, or to rotate once and attend
+ * several times).  jetlong_prefill == jetlong_prefill_rotate followed by
+ * jetlong_prefill_attend on the same workspace and stream.
+ *
+ * jetlong_prefill_rotate: RoPE in the Q/K load path.  Reads q and k, writes
+ *   the rotated operands into the workspace (queries and keys at true
+ *   positions i, j and, when G > 1, at remote positions f(i), f(j)) and, if
+ *   k_cache_out is not NULL, the true-position cache rows [0, L).
+ * jetlong_prefill_attend: the attention kernel.  Reads v and the rotated
+ *   operands a preceding jetlong_prefill_rotate with the same B, Hq, Hkv, L,
+ *   D, w_pretrained left in `workspace`; writes out and lse.
+ */
+JL_API int jetlong_prefill_rotate(const void *q, const void *k, int B, int Hq, int Hkv, int L,
+                                  int D, int w_pretrained, float rope_theta, void *k_cache_out,
+                                  int k_cache_capacity, void *workspace, size_t workspace_bytes,
+                                  jl_stream_t stream);
+
+JL_API int jetlong_prefill_attend(const void *v, void *out, float *lse, int B, int Hq, int Hkv,
+                                  int L, int D, int w_pretrained, int w0, int out_dtype,
+                                  const void *workspace, size_t workspace_bytes,
+                                  jl_stream_t stream);
+
+/*
+ * Bytes of workspace jetlong_decode needs for a cache of L tokens (host only).
+ * Non-decreasing in L: sizing it for the largest L a generation loop will reach
+ * covers every earlier step.  Returns 0 if a size is invalid.
+ */
+JL_API size_t jetlong_decode_workspace_size(int B, int Hq, int Hkv, int L, int D);
+
+/*
+ * One generation step on the true-position cache (§3.2).
+ *
+ *   q        [B, Hq, D] BF16, pre-RoPE query of the new token, at position L-1
+ *   k_cache  [B, Lcap, Hkv, D] BF16, RoPE(x_k, k) at true positions; slots
+ *            [0, L) valid (the new token's key included)
+ *   v_cache  [B, Lcap, Hkv, D] BF16; slots [0, L) valid
+ *   out      [B, Hq, D] out_dtype;   lse [B, Hq] float32 (may be NULL)
+ *   L: tokens in the cache including the new one, 1 <= L <= Lcap; G is
+ *      recomputed from this L (§3.1).  Keys with (L-1) - j <= w0 are used as
+ *      cached; older keys are rotated by Delta j = f(j) - j on the fly and
+ *      scored against RoPE(x_q, f(L-1)).
+ *   workspace: >= jetlong_decode_workspace_size(B, Hq, Hkv, L, D) bytes,
+ *      256-byte aligned; contents on entry do not matter.
+ */
+JL_API int jetlong_decode(const void *q, const void *k_cache, const void *v_cache, void *out,
+                   float *lse, int B, int Hq, int Hkv, int L, int Lcap, int D,
+                   int w_pretrained, int w0, float rope_theta, int out_dtype,
+                   void *workspace, size_t workspace_bytes, jl_stream_t stream);
+
+/*
+ * Write keys into the true-position cache (§3.2): for t < n,
+ *   k_cache[b, pos0 + t, h, :] = RoPE(k[b, t, h, :], pos0 + t).
+ *
+ *   k        [B, n, Hkv, D] BF16 pre-RoPE keys (read)
+ *   k_cache  [B, Lcap, Hkv, D] BF16 (rows [pos0, pos0 + n) written)
+ *   0 <= pos0, n >= 1, pos0 + n <= Lcap.
+ */
+JL_API int jetlong_rope_cache(const void *k, void *k_cache, int B, int n, int Hkv, int D,
+                       int pos0, int Lcap, float rope_theta, jl_stream_t stream);
+
+/*
+ * Synchronise `stream` and report kernel-side failures since the last call:
+ * JL_ERR_DEVICE_TIMEOUT if a bounded wait expired in any kernel of this
+ * library on the current device, JL_ERR_CUDA if the stream reports an error,
+ * else JL_OK.  Clears the recorded timeout.
+ */
+JL_API int jetlong_device_status(jl_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* JETLONG_H */

@@ -135,7 +135,8 @@ def _check_shapes(q, k, v):
     return B, L, Hq, Hkv, D
 
 
-def prefill_rows(q, k, v, w_pretrained: int, w0: int, theta: float, rows):
+def prefill_rows(q, k, v, w_pretrained: int, w0: int, theta: float, rows,
+                 q_holds_rows: bool = False):
     """Bifocal causal attention for the listed query rows (all heads, all batches).
 
     For query i and key j <= i (§3 score rule, §3.1 schedule, one G for the
@@ -150,13 +151,22 @@ def prefill_rows(q, k, v, w_pretrained: int, w0: int, theta: float, rows):
     per (i, j) with an explicit mask; keys are scored in one vectorised product
     per row, which is the same arithmetic as a per-pair loop.
 
+    The prompt length L (and with it G) is k.shape[1].  With
+    ``q_holds_rows`` q is [B, len(rows), Hq, D] and holds only the listed
+    rows' queries, in the order of ``rows``.
+
     Returns (o [B, len(rows), Hq, D] float64, lse [B, Hq, len(rows)] float64).
     """
     q = np.asarray(q)
     k = np.asarray(k)
     v = np.asarray(v)
-    B, L, Hq, Hkv, D = _check_shapes(q, k, v)
     rows = np.asarray(rows, dtype=np.int64)
+    if q_holds_rows:
+        if q.ndim != 4 or q.shape[1] != rows.size:
+            raise ValueError("q must be [B, len(rows), Hq, D]")
+        B, L, Hq, Hkv, D = _check_shapes(np.broadcast_to(q[:, :1], (q.shape[0], k.shape[1]) + q.shape[2:]), k, v)
+    else:
+        B, L, Hq, Hkv, D = _check_shapes(q, k, v)
     if rows.size and (rows.min() < 0 or rows.max() >= L):
         raise ValueError("row out of range")
     grp = Hq // Hkv
@@ -174,7 +184,8 @@ def prefill_rows(q, k, v, w_pretrained: int, w0: int, theta: float, rows):
             k_remote = rope(xk, remap(jpos, G), theta)  # RoPE(x_k, f(j))
             heads = np.arange(g * grp, (g + 1) * grp)
             for r, i in enumerate(rows):
-                xq = q[b, i, heads, :].astype(np.float64)           # [grp, D]
+                qi = r if q_holds_rows else i
+                xq = q[b, qi, heads, :].astype(np.float64)          # [grp, D]
                 q_true = rope(xq, np.int64(i), theta)                 # RoPE(x_q, i)
                 q_remote = rope(xq, remap(np.int64(i), G), theta)     # RoPE(x_q, f(i))
                 n = i + 1                                             # causal: j <= i

@@ -1,0 +1,142 @@
+"""C-ABI checks that need no GPU: the library loads, exports every function
+include/jetlong.h declares, answers the host-only queries, and rejects
+invalid arguments before any CUDA call."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import oracle
+from zero_shot_rope_bifocal_b200 import build as jl_build
+from zero_shot_rope_bifocal_b200 import jetlong as jl
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "jetlong.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not os.path.exists(jl.LIB_PATH):
+        jl_build.build()
+    return jl.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return re.findall(r"JL_API\s+[\w\s\*]+?\b(jetlong_\w+)\s*\(", text)
+
+
+def test_header_declares_the_api():
+    names = set(declared_functions())
+    assert {"jetlong_prefill", "jetlong_decode", "jetlong_rope_cache", "jetlong_group_size",
+            "jetlong_prefill_workspace_size", "jetlong_decode_workspace_size",
+            "jetlong_status_string", "jetlong_device_status", "jetlong_version"} <= names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+    assert set(declared_functions()) == set(jl.SIGNATURES), "binding and header disagree"
+
+
+def test_only_the_c_abi_is_exported(lib):
+    out = os.popen(f"nm -D --defined-only {jl.LIB_PATH}").read()
+    funcs = {ln.split()[-1] for ln in out.splitlines() if " T " in ln}
+    assert funcs == set(declared_functions()), funcs ^ set(declared_functions())
+
+
+def test_group_size_agrees_with_oracle(lib):
+    for w in (1, 7, 128, 32768):
+        for L in list(range(1, 3 * w + 5, max(1, w // 7))) + [98304, 98305, 131072, 2 ** 31 - 1]:
+            assert jl.jetlong_group_size(L, w) == oracle.group_size(L, w), (L, w)
+    assert lib.jetlong_group_size(0, 5) == jl.JL_ERR_SHAPE
+    assert lib.jetlong_group_size(5, 0) == jl.JL_ERR_SHAPE
+
+
+def test_workspace_sizes(lib):
+    n = jl.jetlong_prefill_workspace_size(1, 32, 8, 131072, 128)
+    assert n >= 2 * 2 * (32 + 8) * 131072 * 128
+    assert jl.jetlong_prefill_workspace_size(1, 3, 2, 100, 128) == 0  # Hq % Hkv != 0
+    assert jl.jetlong_prefill_workspace_size(1, 2, 1, 100, 96) == 0   # unsupported D
+    prev = 0
+    for L in (1, 63, 64, 65, 1000, 4096, 32768, 65536, 131072, 1 << 20):
+        cur = jl.jetlong_decode_workspace_size(1, 32, 8, L, 128)
+        assert cur >= prev and cur > 0
+        prev = cur
+
+
+def test_status_strings(lib):
+    for code in range(-8, 1):
+        assert jl.status_string(code).startswith("JL_")
+    assert jl.status_string(5) == "unknown jl_status"
+
+
+P = ctypes.c_void_p(256)  # a non-NULL, aligned stand-in pointer; never dereferenced
+
+
+def prefill_call(lib, **kw):
+    a = dict(q=P, k=P, v=P, out=P, lse=None, B=1, Hq=2, Hkv=1, L=512, D=64, wp=128, w0=32,
+             theta=1e4, od=0, kc=None, cap=0, ws=P, wsb=1 << 40, stream=None)
+    a.update(kw)
+    return lib.jetlong_prefill(a["q"], a["k"], a["v"], a["out"], a["lse"], a["B"], a["Hq"], a["Hkv"],
+                               a["L"], a["D"], a["wp"], a["w0"], a["theta"], a["od"], a["kc"],
+                               a["cap"], a["ws"], a["wsb"], a["stream"])
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(q=None), jl.JL_ERR_NULL),
+    (dict(out=None), jl.JL_ERR_NULL),
+    (dict(B=0), jl.JL_ERR_SHAPE),
+    (dict(L=0), jl.JL_ERR_SHAPE),
+    (dict(Hq=3, Hkv=2), jl.JL_ERR_SHAPE),
+    (dict(D=96), jl.JL_ERR_UNSUPPORTED),
+    (dict(D=256), jl.JL_ERR_UNSUPPORTED),
+    (dict(w0=-1), jl.JL_ERR_SHAPE),
+    (dict(wp=0), jl.JL_ERR_SHAPE),
+    (dict(theta=0.0), jl.JL_ERR_SHAPE),
+    (dict(theta=float("nan")), jl.JL_ERR_SHAPE),
+    (dict(od=2), jl.JL_ERR_UNSUPPORTED),
+    (dict(kc=P, cap=100), jl.JL_ERR_SHAPE),
+    (dict(q=ctypes.c_void_p(258)), jl.JL_ERR_ALIGN),
+    (dict(lse=ctypes.c_void_p(260)), jl.JL_ERR_ALIGN),
+    (dict(ws=None), jl.JL_ERR_WORKSPACE),
+    (dict(wsb=10), jl.JL_ERR_WORKSPACE),
+    (dict(ws=ctypes.c_void_p(272)), jl.JL_ERR_ALIGN),
+])
+def test_prefill_rejects_bad_arguments(lib, kw, status):
+    assert prefill_call(lib, **kw) == status
+
+
+def decode_call(lib, **kw):
+    a = dict(q=P, kc=P, vc=P, out=P, lse=None, B=1, Hq=32, Hkv=8, L=1000, Lcap=1000, D=128,
+             wp=32768, w0=4096, theta=1e6, od=0, ws=P, wsb=1 << 40, stream=None)
+    a.update(kw)
+    return lib.jetlong_decode(a["q"], a["kc"], a["vc"], a["out"], a["lse"], a["B"], a["Hq"],
+                              a["Hkv"], a["L"], a["Lcap"], a["D"], a["wp"], a["w0"], a["theta"],
+                              a["od"], a["ws"], a["wsb"], a["stream"])
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(kc=None), jl.JL_ERR_NULL),
+    (dict(Lcap=999), jl.JL_ERR_SHAPE),
+    (dict(L=0), jl.JL_ERR_SHAPE),
+    (dict(Hq=34, Hkv=2), jl.JL_ERR_UNSUPPORTED),   # group of 17 query heads
+    (dict(D=80), jl.JL_ERR_UNSUPPORTED),
+    (dict(w0=-5), jl.JL_ERR_SHAPE),
+    (dict(vc=ctypes.c_void_p(8)), jl.JL_ERR_ALIGN),
+    (dict(wsb=0), jl.JL_ERR_WORKSPACE),
+])
+def test_decode_rejects_bad_arguments(lib, kw, status):
+    assert decode_call(lib, **kw) == status
+
+
+@pytest.mark.parametrize("args,status", [
+    ((None, P, 1, 4, 2, 128, 0, 8, 1e4, None), jl.JL_ERR_NULL),
+    ((P, P, 1, 4, 2, 128, 5, 8, 1e4, None), jl.JL_ERR_SHAPE),     # pos0 + n > Lcap
+    ((P, P, 1, 0, 2, 128, 0, 8, 1e4, None), jl.JL_ERR_SHAPE),
+    ((P, P, 1, 4, 2, 48, 0, 8, 1e4, None), jl.JL_ERR_UNSUPPORTED),
+    ((P, P, 1, 4, 2, 128, -1, 8, 1e4, None), jl.JL_ERR_SHAPE),
+])
+def test_rope_cache_rejects_bad_arguments(lib, args, status):
+    assert lib.jetlong_rope_cache(*args) == status

@@ -286,6 +286,10 @@ def test_prefill_rows_subset_matches_full():
     o2, l2 = oracle.prefill_rows(q, k, v, w.w_pretrained, w.w0, w.theta, rows)
     np.testing.assert_allclose(o2, o[:, rows], atol=0)
     np.testing.assert_allclose(l2, lse[:, :, rows], atol=0)
+    o3, l3 = oracle.prefill_rows(q[:, rows], k, v, w.w_pretrained, w.w0, w.theta, rows,
+                                 q_holds_rows=True)
+    np.testing.assert_array_equal(o3, o2)
+    np.testing.assert_array_equal(l3, l2)
 
 
 # ---------------------------------------------------------------- decode

@@ -1,0 +1,318 @@
+// jetlong_api.cu -- the C ABI declared in include/jetlong.h: argument
+// validation, workspace carving, and the launch sequence of each call.
+//
+// Every check runs on the host before the first CUDA call, so an invalid call
+// returns its status without touching the device (and works on a machine with
+// no GPU at all).
+#include <mutex>
+
+#include "../../include/jetlong.h"
+#include "jl_common.cuh"
+
+namespace jl {
+
+// Kernel-side error word (timeouts of bounded waits).  Kernels receive its
+// device address; host code reaches it through cudaGetSymbolAddress.
+__device__ unsigned int g_device_error;
+
+namespace {
+
+constexpr size_t kAlign = 256;
+
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+struct DeviceState {
+  bool checked = false;
+  bool is_sm100 = false;
+  unsigned int *err = nullptr;
+};
+
+constexpr int kMaxDevices = 64;
+std::mutex g_mu;
+DeviceState g_dev[kMaxDevices];
+
+// Checks the current device once (compute capability 10.x) and fetches the
+// device address of the error word for it.
+int current_device(DeviceState **out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return JL_ERR_NO_DEVICE;
+  }
+  std::lock_guard<std::mutex> lk(g_mu);
+  DeviceState &st = g_dev[dev];
+  if (!st.checked) {
+    int major = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) {
+      cudaGetLastError();
+      return JL_ERR_NO_DEVICE;
+    }
+    st.is_sm100 = (major == 10);
+    if (st.is_sm100) {
+      void *p = nullptr;
+      if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) {
+        cudaGetLastError();
+        return JL_ERR_CUDA;
+      }
+      st.err = static_cast<unsigned int *>(p);
+    }
+    st.checked = true;
+  }
+  if (!st.is_sm100) return JL_ERR_NO_DEVICE;
+  *out = &st;
+  return JL_OK;
+}
+
+int check_common(int B, int Hq, int Hkv, int L, int D) {
+  if (B < 1 || Hq < 1 || Hkv < 1 || L < 1) return JL_ERR_SHAPE;
+  if (Hq % Hkv != 0) return JL_ERR_SHAPE;
+  if (D != 64 && D != 128) return JL_ERR_UNSUPPORTED;
+  // Sizes must keep every element index inside 2^31 tokens x heads x D math.
+  if (static_cast<long long>(B) * L * Hq > (1ll << 31)) return JL_ERR_SHAPE;
+  return JL_OK;
+}
+
+int check_method(int w_pretrained, int w0, float theta) {
+  if (w_pretrained < 1 || w0 < 0) return JL_ERR_SHAPE;
+  if (!(theta > 0.f) || theta != theta) return JL_ERR_SHAPE;
+  return JL_OK;
+}
+
+size_t prefill_ws_bytes(int B, int Hq, int Hkv, int L, int D) {
+  const size_t q = static_cast<size_t>(B) * Hq * L * D * 2;
+  const size_t k = static_cast<size_t>(B) * Hkv * L * D * 2;
+  return 2 * align_up(q) + 2 * align_up(k);
+}
+
+size_t decode_ws_bytes(int B, int Hq, int Hkv, int L, int D) {
+  int ns = 0, ch = 0;
+  decode_plan(B, Hkv, L, &ns, &ch);
+  return align_up(static_cast<size_t>(B) * Hq * ns * (D + 2) * sizeof(float));
+}
+
+}  // namespace
+}  // namespace jl
+
+using namespace jl;
+
+extern "C" {
+
+const char *jetlong_status_string(int s) {
+  switch (s) {
+    case JL_OK: return "JL_OK";
+    case JL_ERR_NULL: return "JL_ERR_NULL: a required pointer is NULL";
+    case JL_ERR_SHAPE: return "JL_ERR_SHAPE: a size is out of range or inconsistent";
+    case JL_ERR_UNSUPPORTED: return "JL_ERR_UNSUPPORTED: configuration not implemented";
+    case JL_ERR_ALIGN: return "JL_ERR_ALIGN: a pointer is not 16-byte aligned";
+    case JL_ERR_WORKSPACE: return "JL_ERR_WORKSPACE: workspace missing or too small";
+    case JL_ERR_CUDA: return "JL_ERR_CUDA: a CUDA call or launch failed";
+    case JL_ERR_DEVICE_TIMEOUT: return "JL_ERR_DEVICE_TIMEOUT: a bounded in-kernel wait expired";
+    case JL_ERR_NO_DEVICE: return "JL_ERR_NO_DEVICE: no sm_100 device is current";
+    default: return "unknown jl_status";
+  }
+}
+
+const char *jetlong_version(void) { return "0.1.0"; }
+
+int jetlong_group_size(int L, int w_pretrained) {
+  if (L < 1 || w_pretrained < 1) return JL_ERR_SHAPE;
+  return group_size(L, w_pretrained);
+}
+
+size_t jetlong_prefill_workspace_size(int B, int Hq, int Hkv, int L, int D) {
+  if (check_common(B, Hq, Hkv, L, D) != JL_OK) return 0;
+  return prefill_ws_bytes(B, Hq, Hkv, L, D);
+}
+
+}  // extern "C"
+
+namespace {
+
+// Validation shared by the prefill entry points.  Pointers that a stage does
+// not use are passed as a non-NULL placeholder by the caller.
+int prepare_prefill(const void *q, const void *k, const void *v, void *out, float *lse, int B,
+                    int Hq, int Hkv, int L, int D, int w_pretrained, int w0, float rope_theta,
+                    int out_dtype, void *k_cache_out, int k_cache_capacity, void *workspace,
+                    size_t workspace_bytes, PrefillArgs *a) {
+  if (!q || !k || !v || !out) return JL_ERR_NULL;
+  int st = check_common(B, Hq, Hkv, L, D);
+  if (st != JL_OK) return st;
+  if ((st = check_method(w_pretrained, w0, rope_theta)) != JL_OK) return st;
+  if (out_dtype != JL_BF16 && out_dtype != JL_F32) return JL_ERR_UNSUPPORTED;
+  if (k_cache_out && k_cache_capacity < L) return JL_ERR_SHAPE;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) ||
+      (lse && !aligned16(lse)) || (k_cache_out && !aligned16(k_cache_out)))
+    return JL_ERR_ALIGN;
+  const size_t need = prefill_ws_bytes(B, Hq, Hkv, L, D);
+  if (!workspace || workspace_bytes < need) return JL_ERR_WORKSPACE;
+  if (reinterpret_cast<uintptr_t>(workspace) % kAlign) return JL_ERR_ALIGN;
+
+  DeviceState *dev = nullptr;
+  if ((st = current_device(&dev)) != JL_OK) return st;
+
+  *a = PrefillArgs{};
+  a->q = static_cast<const __nv_bfloat16 *>(q);
+  a->k = static_cast<const __nv_bfloat16 *>(k);
+  a->v = static_cast<const __nv_bfloat16 *>(v);
+  a->out = out;
+  a->lse = lse;
+  a->out_f32 = out_dtype == JL_F32;
+  a->k_cache_out = static_cast<__nv_bfloat16 *>(k_cache_out);
+  a->k_cache_capacity = k_cache_out ? k_cache_capacity : 0;
+  uint8_t *ws = static_cast<uint8_t *>(workspace);
+  const size_t qb = align_up(static_cast<size_t>(B) * Hq * L * D * 2);
+  const size_t kb = align_up(static_cast<size_t>(B) * Hkv * L * D * 2);
+  a->q_true = reinterpret_cast<__nv_bfloat16 *>(ws);
+  a->q_remote = reinterpret_cast<__nv_bfloat16 *>(ws + qb);
+  a->k_true = reinterpret_cast<__nv_bfloat16 *>(ws + 2 * qb);
+  a->k_remote = reinterpret_cast<__nv_bfloat16 *>(ws + 2 * qb + kb);
+  a->B = B;
+  a->Hq = Hq;
+  a->Hkv = Hkv;
+  a->L = L;
+  a->D = D;
+  a->w_pretrained = w_pretrained;
+  a->w0 = w0;
+  a->G = group_size(L, w_pretrained);
+  a->theta = rope_theta;
+  a->dev_error = dev->err;
+  return JL_OK;
+}
+
+// Stand-in for a pointer a stage does not read (never dereferenced).
+void *const kUnused = reinterpret_cast<void *>(static_cast<uintptr_t>(256));
+
+}  // namespace
+
+extern "C" {
+
+int jetlong_prefill(const void *q, const void *k, const void *v, void *out, float *lse, int B,
+                    int Hq, int Hkv, int L, int D, int w_pretrained, int w0, float rope_theta,
+                    int out_dtype, void *k_cache_out, int k_cache_capacity, void *workspace,
+                    size_t workspace_bytes, jl_stream_t stream) {
+  PrefillArgs a;
+  const int st = prepare_prefill(q, k, v, out, lse, B, Hq, Hkv, L, D, w_pretrained, w0,
+                                 rope_theta, out_dtype, k_cache_out, k_cache_capacity, workspace,
+                                 workspace_bytes, &a);
+  if (st != JL_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (launch_rope_qk(a, s) != cudaSuccess) return JL_ERR_CUDA;
+  if (launch_prefill_attention(a, s) != cudaSuccess) return JL_ERR_CUDA;
+  return JL_OK;
+}
+
+int jetlong_prefill_rotate(const void *q, const void *k, int B, int Hq, int Hkv, int L, int D,
+                           int w_pretrained, float rope_theta, void *k_cache_out,
+                           int k_cache_capacity, void *workspace, size_t workspace_bytes,
+                           jl_stream_t stream) {
+  PrefillArgs a;
+  const int st = prepare_prefill(q, k, kUnused, kUnused, nullptr, B, Hq, Hkv, L, D, w_pretrained,
+                                 0, rope_theta, JL_BF16, k_cache_out, k_cache_capacity, workspace,
+                                 workspace_bytes, &a);
+  if (st != JL_OK) return st;
+  if (launch_rope_qk(a, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return JL_ERR_CUDA;
+  return JL_OK;
+}
+
+int jetlong_prefill_attend(const void *v, void *out, float *lse, int B, int Hq, int Hkv, int L,
+                           int D, int w_pretrained, int w0, int out_dtype, const void *workspace,
+                           size_t workspace_bytes, jl_stream_t stream) {
+  PrefillArgs a;
+  const int st = prepare_prefill(kUnused, kUnused, v, out, lse, B, Hq, Hkv, L, D, w_pretrained, w0,
+                                 1.0f, out_dtype, nullptr, 0, const_cast<void *>(workspace),
+                                 workspace_bytes, &a);
+  if (st != JL_OK) return st;
+  if (launch_prefill_attention(a, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return JL_ERR_CUDA;
+  return JL_OK;
+}
+
+size_t jetlong_decode_workspace_size(int B, int Hq, int Hkv, int L, int D) {
+  if (check_common(B, Hq, Hkv, L, D) != JL_OK) return 0;
+  return decode_ws_bytes(B, Hq, Hkv, L, D);
+}
+
+int jetlong_decode(const void *q, const void *k_cache, const void *v_cache, void *out, float *lse,
+                   int B, int Hq, int Hkv, int L, int Lcap, int D, int w_pretrained, int w0,
+                   float rope_theta, int out_dtype, void *workspace, size_t workspace_bytes,
+                   jl_stream_t stream) {
+  if (!q || !k_cache || !v_cache || !out) return JL_ERR_NULL;
+  int st = check_common(B, Hq, Hkv, L, D);
+  if (st != JL_OK) return st;
+  if (Lcap < L) return JL_ERR_SHAPE;
+  if (Hq / Hkv > decode_max_group()) return JL_ERR_UNSUPPORTED;
+  if ((st = check_method(w_pretrained, w0, rope_theta)) != JL_OK) return st;
+  if (out_dtype != JL_BF16 && out_dtype != JL_F32) return JL_ERR_UNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out) ||
+      (lse && !aligned16(lse)))
+    return JL_ERR_ALIGN;
+  const size_t need = decode_ws_bytes(B, Hq, Hkv, L, D);
+  if (!workspace || workspace_bytes < need) return JL_ERR_WORKSPACE;
+  if (reinterpret_cast<uintptr_t>(workspace) % kAlign) return JL_ERR_ALIGN;
+
+  DeviceState *dev = nullptr;
+  if ((st = current_device(&dev)) != JL_OK) return st;
+
+  DecodeArgs a{};
+  a.q = static_cast<const __nv_bfloat16 *>(q);
+  a.k_cache = static_cast<const __nv_bfloat16 *>(k_cache);
+  a.v_cache = static_cast<const __nv_bfloat16 *>(v_cache);
+  a.out = out;
+  a.lse = lse;
+  a.out_f32 = out_dtype == JL_F32;
+  a.partial = static_cast<float *>(workspace);
+  a.B = B;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.L = L;
+  a.Lcap = Lcap;
+  a.D = D;
+  a.w_pretrained = w_pretrained;
+  a.w0 = w0;
+  a.G = group_size(L, w_pretrained);
+  a.theta = rope_theta;
+  decode_plan(B, Hkv, L, &a.n_split, &a.chunk);
+  a.dev_error = dev->err;
+  if (launch_decode(a, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return JL_ERR_CUDA;
+  return JL_OK;
+}
+
+int jetlong_rope_cache(const void *k, void *k_cache, int B, int n, int Hkv, int D, int pos0,
+                       int Lcap, float rope_theta, jl_stream_t stream) {
+  if (!k || !k_cache) return JL_ERR_NULL;
+  if (B < 1 || n < 1 || Hkv < 1 || pos0 < 0 || Lcap < 1) return JL_ERR_SHAPE;
+  if (static_cast<long long>(pos0) + n > Lcap) return JL_ERR_SHAPE;
+  if (D != 64 && D != 128) return JL_ERR_UNSUPPORTED;
+  if (!(rope_theta > 0.f)) return JL_ERR_SHAPE;
+  if (!aligned16(k) || !aligned16(k_cache)) return JL_ERR_ALIGN;
+  DeviceState *dev = nullptr;
+  int st = current_device(&dev);
+  if (st != JL_OK) return st;
+  if (launch_rope_cache(static_cast<const __nv_bfloat16 *>(k), static_cast<__nv_bfloat16 *>(k_cache),
+                        B, n, Hkv, D, pos0, Lcap, rope_theta,
+                        reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return JL_ERR_CUDA;
+  return JL_OK;
+}
+
+int jetlong_device_status(jl_stream_t stream) {
+  DeviceState *dev = nullptr;
+  int st = current_device(&dev);
+  if (st != JL_OK) return st;
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) {
+    cudaGetLastError();
+    return JL_ERR_CUDA;
+  }
+  unsigned int flag = 0;
+  if (cudaMemcpyFromSymbol(&flag, g_device_error, sizeof(flag)) != cudaSuccess) return JL_ERR_CUDA;
+  if (flag != kDevOk) {
+    const unsigned int zero = 0;
+    if (cudaMemcpyToSymbol(g_device_error, &zero, sizeof(zero)) != cudaSuccess) return JL_ERR_CUDA;
+    return JL_ERR_DEVICE_TIMEOUT;
+  }
+  return JL_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,101 @@
+// jl_common.cuh -- definitions shared by the library's translation units:
+// the schedule of §3.1, RoPE angle evaluation, bf16 helpers, and the
+// launcher interfaces between the C-ABI layer and the kernels.
+#pragma once
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <climits>
+#include <cstdint>
+
+namespace jl {
+
+// Kernel-side error codes written to the device error word.
+enum : unsigned int {
+  kDevOk = 0u,
+  kDevTimeout = 1u,
+};
+
+// Time limit for any single in-kernel wait.  Every legitimate wait in these
+// kernels lasts micro- to milliseconds; two seconds means a lost arrival.
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+
+// §3.1, Eq. (2): G = max(1, ceil(L / w_pretrained)), integer arithmetic.
+__host__ __device__ __forceinline__ int group_size(int L, int w_pretrained) {
+  const long long g = (static_cast<long long>(L) + w_pretrained - 1) / w_pretrained;
+  return g < 1 ? 1 : static_cast<int>(g);
+}
+
+// §3.1: remote position f(x) = floor(x / G) for x >= 0.
+__host__ __device__ __forceinline__ int remap(int x, int G) { return x / G; }
+
+// RoPE frequency theta^(-2i/D) in double precision.
+__device__ __forceinline__ double rope_freq(int i, int D, double theta) {
+  return exp(-2.0 * static_cast<double>(i) / static_cast<double>(D) * log(theta));
+}
+
+// cos / sin of the RoPE angle pos * freq.  The product is formed in double,
+// reduced by the nearest multiple of 2*pi (split into a double head and tail
+// so the reduction stays exact to ~1e-16 relative for |angle| < 2^40), and the
+// reduced angle in [-pi, pi] goes to the single-precision sine/cosine.
+__device__ __forceinline__ void rope_cos_sin(long long pos, double freq, float &c, float &s) {
+  const double two_pi_hi = 6.283185307179586232;   // nearest double to 2*pi
+  const double two_pi_lo = 2.4492935982947064e-16; // 2*pi - two_pi_hi
+  const double a = static_cast<double>(pos) * freq;
+  const double n = rint(a * 0.15915494309189533577);  // a / (2*pi), rounded
+  double r = fma(-n, two_pi_hi, a);
+  r = fma(-n, two_pi_lo, r);
+  sincosf(static_cast<float>(r), &s, &c);
+}
+
+__device__ __forceinline__ float bf2f(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+// ---------------------------------------------------------------- launchers
+struct PrefillArgs {
+  // caller buffers
+  const __nv_bfloat16 *q, *k, *v;
+  void *out;
+  float *lse;
+  int out_f32;
+  __nv_bfloat16 *k_cache_out;
+  int k_cache_capacity;
+  // rotated operands in the workspace, head-major [B, H, L, D]
+  __nv_bfloat16 *q_true, *q_remote, *k_true, *k_remote;
+  // sizes and method parameters
+  int B, Hq, Hkv, L, D, w_pretrained, w0, G;
+  float theta;
+  unsigned int *dev_error;
+};
+
+// Rotates q and k into the four operand arrays (and the optional cache).
+cudaError_t launch_rope_qk(const PrefillArgs &a, cudaStream_t stream);
+
+// The attention kernel proper (tcgen05 / TMEM / TMA).
+cudaError_t launch_prefill_attention(const PrefillArgs &a, cudaStream_t stream);
+
+struct DecodeArgs {
+  const __nv_bfloat16 *q, *k_cache, *v_cache;
+  void *out;
+  float *lse;
+  int out_f32;
+  float *partial;  // workspace: [B, Hq, n_split, D + 2]
+  int B, Hq, Hkv, L, Lcap, D, w_pretrained, w0, G;
+  float theta;
+  int n_split, chunk;
+  unsigned int *dev_error;
+};
+
+// Split-KV plan: number of key chunks and chunk length for a cache of L tokens.
+void decode_plan(int B, int Hkv, int L, int *n_split, int *chunk);
+
+// Largest Hq / Hkv the decode kernel supports.
+int decode_max_group();
+
+cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t stream);
+
+cudaError_t launch_rope_cache(const __nv_bfloat16 *k, __nv_bfloat16 *k_cache, int B, int n,
+                              int Hkv, int D, int pos0, int Lcap, float theta,
+                              cudaStream_t stream);
+
+}  // namespace jl

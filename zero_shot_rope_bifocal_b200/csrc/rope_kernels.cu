@@ -1,0 +1,151 @@
+// rope_kernels.cu -- RoPE in the Q/K load path of the bifocal attention.
+//
+// Prefill operand pass (Jet-Long paper, §3 score rule and §3.2): for every
+// token the queries are rotated to the true position i and to the remote
+// position f(i), the keys to j and to f(j):
+//
+//   q_true[b,h,i]  = RoPE(x_q, i)      q_remote[b,h,i] = RoPE(x_q, f(i))
+//   k_true[b,g,j]  = RoPE(x_k, j)      k_remote[b,g,j] = RoPE(x_k, f(j))
+//
+// k_true is exactly the true-position KV cache of §3.2, and k_remote equals
+// the correction rotation by Delta j = f(j) - j applied to it.  The outputs are
+// head-major [B, H, L, D] BF16 so that the attention kernel's TMA fetches each
+// 128-token tile as one contiguous block.  When G == 1 (L <= w_pretrained,
+// the native-window case of Appendix H) f is the identity and only the
+// true-position arrays are written.
+//
+// Cache writer (§3.2): k_cache[b, pos0 + t] = RoPE(k[b, t], pos0 + t).
+//
+// Each CTA evaluates cos/sin once per (position, frequency) into shared
+// memory and applies it to every head of that position; channel pairs are
+// (i, i + D/2), processed two pairs per thread with BF16x2 loads and stores.
+#include "jl_common.cuh"
+
+namespace jl {
+namespace {
+
+constexpr int kRopeThreads = 256;
+constexpr int kPosPerCta = 4;
+
+// Rotate BF16 pairs (a[i], a[i+D/2]) and (a[i+1], a[i+1+D/2]) of one head row.
+__device__ __forceinline__ void rotate2(const __nv_bfloat16 *src, __nv_bfloat16 *dst, int i, int half,
+                                        float2 cs0, float2 cs1) {
+  const __nv_bfloat162 lo = *reinterpret_cast<const __nv_bfloat162 *>(src + i);
+  const __nv_bfloat162 hi = *reinterpret_cast<const __nv_bfloat162 *>(src + i + half);
+  const float a0 = __low2float(lo), a1 = __high2float(lo);
+  const float b0 = __low2float(hi), b1 = __high2float(hi);
+  // cs = (cos, sin)
+  const float r0 = a0 * cs0.x - b0 * cs0.y, s0 = a0 * cs0.y + b0 * cs0.x;
+  const float r1 = a1 * cs1.x - b1 * cs1.y, s1 = a1 * cs1.y + b1 * cs1.x;
+  *reinterpret_cast<__nv_bfloat162 *>(dst + i) = __floats2bfloat162_rn(r0, r1);
+  *reinterpret_cast<__nv_bfloat162 *>(dst + i + half) = __floats2bfloat162_rn(s0, s1);
+}
+
+__global__ void __launch_bounds__(kRopeThreads)
+rope_qk_kernel(PrefillArgs a) {
+  extern __shared__ float2 cs_smem[];  // [2][kPosPerCta][D/2] (cos, sin)
+  const int half = a.D / 2;
+  const int b = blockIdx.y;
+  const int p_begin = blockIdx.x * kPosPerCta;
+  const int npos = min(kPosPerCta, a.L - p_begin);
+  const bool two = a.G > 1;
+  float2 *cs_true = cs_smem;
+  float2 *cs_remote = cs_smem + kPosPerCta * half;
+
+  const double theta = static_cast<double>(a.theta);
+  for (int idx = threadIdx.x; idx < npos * half * (two ? 2 : 1); idx += blockDim.x) {
+    const int var = idx / (npos * half);
+    const int rem = idx - var * npos * half;
+    const int t = rem / half, i = rem - t * half;
+    const int pos = p_begin + t;
+    const long long ppos = var == 0 ? pos : remap(pos, a.G);
+    float c, s;
+    rope_cos_sin(ppos, rope_freq(i, a.D, theta), c, s);
+    (var == 0 ? cs_true : cs_remote)[t * half + i] = make_float2(c, s);
+  }
+  __syncthreads();
+
+  const int quarter = a.D / 4;  // pairs of channel pairs per head row
+  // queries
+  for (int idx = threadIdx.x; idx < npos * a.Hq * quarter; idx += blockDim.x) {
+    const int t = idx / (a.Hq * quarter);
+    const int rem = idx - t * a.Hq * quarter;
+    const int h = rem / quarter;
+    const int i = (rem - h * quarter) * 2;
+    const int pos = p_begin + t;
+    const __nv_bfloat16 *src = a.q + ((static_cast<size_t>(b) * a.L + pos) * a.Hq + h) * a.D;
+    const size_t drow = ((static_cast<size_t>(b) * a.Hq + h) * a.L + pos) * a.D;
+    rotate2(src, a.q_true + drow, i, half, cs_true[t * half + i], cs_true[t * half + i + 1]);
+    if (two)
+      rotate2(src, a.q_remote + drow, i, half, cs_remote[t * half + i],
+              cs_remote[t * half + i + 1]);
+  }
+  // keys (+ optional true-position cache)
+  for (int idx = threadIdx.x; idx < npos * a.Hkv * quarter; idx += blockDim.x) {
+    const int t = idx / (a.Hkv * quarter);
+    const int rem = idx - t * a.Hkv * quarter;
+    const int g = rem / quarter;
+    const int i = (rem - g * quarter) * 2;
+    const int pos = p_begin + t;
+    const __nv_bfloat16 *src = a.k + ((static_cast<size_t>(b) * a.L + pos) * a.Hkv + g) * a.D;
+    const size_t drow = ((static_cast<size_t>(b) * a.Hkv + g) * a.L + pos) * a.D;
+    rotate2(src, a.k_true + drow, i, half, cs_true[t * half + i], cs_true[t * half + i + 1]);
+    if (two)
+      rotate2(src, a.k_remote + drow, i, half, cs_remote[t * half + i],
+              cs_remote[t * half + i + 1]);
+    if (a.k_cache_out) {
+      __nv_bfloat16 *crow =
+          a.k_cache_out + ((static_cast<size_t>(b) * a.k_cache_capacity + pos) * a.Hkv + g) * a.D;
+      rotate2(src, crow, i, half, cs_true[t * half + i], cs_true[t * half + i + 1]);
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kRopeThreads)
+rope_cache_kernel(const __nv_bfloat16 *__restrict__ k, __nv_bfloat16 *__restrict__ k_cache, int n,
+                  int Hkv, int D, int pos0, int Lcap, float theta_f) {
+  extern __shared__ float2 cs_smem[];  // [kPosPerCta][D/2]
+  const int half = D / 2;
+  const int b = blockIdx.y;
+  const int t_begin = blockIdx.x * kPosPerCta;
+  const int npos = min(kPosPerCta, n - t_begin);
+  const double theta = static_cast<double>(theta_f);
+  for (int idx = threadIdx.x; idx < npos * half; idx += blockDim.x) {
+    const int t = idx / half, i = idx - t * half;
+    float c, s;
+    rope_cos_sin(static_cast<long long>(pos0) + t_begin + t, rope_freq(i, D, theta), c, s);
+    cs_smem[t * half + i] = make_float2(c, s);
+  }
+  __syncthreads();
+  const int quarter = D / 4;
+  for (int idx = threadIdx.x; idx < npos * Hkv * quarter; idx += blockDim.x) {
+    const int t = idx / (Hkv * quarter);
+    const int rem = idx - t * Hkv * quarter;
+    const int g = rem / quarter;
+    const int i = (rem - g * quarter) * 2;
+    const __nv_bfloat16 *src = k + ((static_cast<size_t>(b) * n + t_begin + t) * Hkv + g) * D;
+    __nv_bfloat16 *dst =
+        k_cache + ((static_cast<size_t>(b) * Lcap + pos0 + t_begin + t) * Hkv + g) * D;
+    rotate2(src, dst, i, half, cs_smem[t * half + i], cs_smem[t * half + i + 1]);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_rope_qk(const PrefillArgs &a, cudaStream_t stream) {
+  const dim3 grid((a.L + kPosPerCta - 1) / kPosPerCta, a.B);
+  const size_t smem = 2 * kPosPerCta * (a.D / 2) * sizeof(float2);
+  rope_qk_kernel<<<grid, kRopeThreads, smem, stream>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_rope_cache(const __nv_bfloat16 *k, __nv_bfloat16 *k_cache, int B, int n,
+                              int Hkv, int D, int pos0, int Lcap, float theta,
+                              cudaStream_t stream) {
+  const dim3 grid((n + kPosPerCta - 1) / kPosPerCta, B);
+  const size_t smem = kPosPerCta * (D / 2) * sizeof(float2);
+  rope_cache_kernel<<<grid, kRopeThreads, smem, stream>>>(k, k_cache, n, Hkv, D, pos0, Lcap, theta);
+  return cudaGetLastError();
+}
+
+}  // namespace jl
