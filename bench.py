@@ -265,10 +265,10 @@ def run_native(args):
     stream = torch.cuda.current_stream(dev)
 
     def step(ev_mid=None, ev_end=None):
-        jl.jetlong_prefill_rotate(x.q, x.k, w.w_pretrained, w.theta, ws, stream=stream)
+        jl.jetlong_prefill_rotate(x.q, x.k, x.v, w.w_pretrained, w.theta, ws, stream=stream)
         if ev_mid is not None:
             ev_mid.record(stream)
-        jl.jetlong_prefill_attend(x.v, out, lse, Hq, w.w_pretrained, w.w0, ws, stream=stream)
+        jl.jetlong_prefill_attend(out, lse, Hkv, w.w_pretrained, w.w0, ws, stream=stream)
         if ev_end is not None:
             ev_end.record(stream)
 

@@ -39,6 +39,12 @@
  *     a launch failed (see cudaGetLastError for the CUDA code).  Every wait
  *     inside a kernel is bounded in time; a wait that gives up records
  *     JL_ERR_DEVICE_TIMEOUT, which jetlong_device_status() reports.
+ *   - Precision: BF16 inputs; the prefill's tensor-core operands (rotated
+ *     Q/K, V, and the probabilities P) are FP16, which holds the rotated
+ *     values with three more mantissa bits than BF16; accumulation, softmax
+ *     statistics and LSE are FP32.  Inputs must stay inside the FP16 range
+ *     (|x| <= 65504 after rotation); a prefill that meets a larger value
+ *     records JL_ERR_RANGE for jetlong_device_status().
  *   - Calls on different streams may run concurrently as long as they do not
  *     share output or workspace buffers.
  */
@@ -69,7 +75,9 @@ typedef enum {
   JL_ERR_WORKSPACE = -5,       /* workspace NULL or smaller than required           */
   JL_ERR_CUDA = -6,            /* a CUDA runtime / launch error                     */
   JL_ERR_DEVICE_TIMEOUT = -7,  /* a bounded in-kernel wait expired (device report)  */
-  JL_ERR_NO_DEVICE = -8        /* no sm_100 device is current                       */
+  JL_ERR_NO_DEVICE = -8,       /* no sm_100 device is current                       */
+  JL_ERR_RANGE = -9            /* an input exceeds the FP16 range of the MMA operands
+                                  (|x| > 65504 after rotation; device report)        */
 } jl_status;
 
 typedef enum { JL_BF16 = 0, JL_F32 = 1 } jl_dtype;
@@ -124,23 +132,24 @@ JL_API int jetlong_prefill(const void *q, const void *k, const void *v, void *ou
  * several times).  jetlong_prefill == jetlong_prefill_rotate followed by
  * jetlong_prefill_attend on the same workspace and stream.
  *
- * jetlong_prefill_rotate: RoPE in the Q/K load path.  Reads q and k, writes
- *   the rotated operands into the workspace (queries and keys at true
- *   positions i, j and, when G > 1, at remote positions f(i), f(j)) and, if
- *   k_cache_out is not NULL, the true-position cache rows [0, L).
- * jetlong_prefill_attend: the attention kernel.  Reads v and the rotated
- *   operands a preceding jetlong_prefill_rotate with the same B, Hq, Hkv, L,
- *   D, w_pretrained left in `workspace`; writes out and lse.
+ * jetlong_prefill_rotate: RoPE in the Q/K load path.  Reads q, k, v (layouts
+ *   as for jetlong_prefill) and writes the tensor-core operands into the
+ *   workspace: queries and keys rotated to true positions i, j and, when
+ *   G > 1, to remote positions f(i), f(j), plus the values, all FP16
+ *   head-major; if k_cache_out is not NULL it also writes the BF16
+ *   true-position cache rows [0, L) (§3.2).
+ * jetlong_prefill_attend: the attention kernel.  Reads the operands a
+ *   preceding jetlong_prefill_rotate with the same B, Hq, Hkv, L, D,
+ *   w_pretrained left in `workspace`; writes out and lse (lse may be NULL).
  */
-JL_API int jetlong_prefill_rotate(const void *q, const void *k, int B, int Hq, int Hkv, int L,
-                                  int D, int w_pretrained, float rope_theta, void *k_cache_out,
-                                  int k_cache_capacity, void *workspace, size_t workspace_bytes,
-                                  jl_stream_t stream);
+JL_API int jetlong_prefill_rotate(const void *q, const void *k, const void *v, int B, int Hq,
+                                  int Hkv, int L, int D, int w_pretrained, float rope_theta,
+                                  void *k_cache_out, int k_cache_capacity, void *workspace,
+                                  size_t workspace_bytes, jl_stream_t stream);
 
-JL_API int jetlong_prefill_attend(const void *v, void *out, float *lse, int B, int Hq, int Hkv,
-                                  int L, int D, int w_pretrained, int w0, int out_dtype,
-                                  const void *workspace, size_t workspace_bytes,
-                                  jl_stream_t stream);
+JL_API int jetlong_prefill_attend(void *out, float *lse, int B, int Hq, int Hkv, int L, int D,
+                                  int w_pretrained, int w0, int out_dtype, const void *workspace,
+                                  size_t workspace_bytes, jl_stream_t stream);
 
 /*
  * Bytes of workspace jetlong_decode needs for a cache of L tokens (host only).
@@ -183,8 +192,9 @@ JL_API int jetlong_rope_cache(const void *k, void *k_cache, int B, int n, int Hk
 /*
  * Synchronise `stream` and report kernel-side failures since the last call:
  * JL_ERR_DEVICE_TIMEOUT if a bounded wait expired in any kernel of this
- * library on the current device, JL_ERR_CUDA if the stream reports an error,
- * else JL_OK.  Clears the recorded timeout.
+ * library on the current device, JL_ERR_RANGE if a prefill met an input
+ * outside the FP16 operand range, JL_ERR_CUDA if the stream reports an error,
+ * else JL_OK.  Clears the recorded report.
  */
 JL_API int jetlong_device_status(jl_stream_t stream);
 

@@ -56,7 +56,7 @@ def test_group_size_agrees_with_oracle(lib):
 
 def test_workspace_sizes(lib):
     n = jl.jetlong_prefill_workspace_size(1, 32, 8, 131072, 128)
-    assert n >= 2 * 2 * (32 + 8) * 131072 * 128
+    assert n >= 2 * (2 * 32 + 3 * 8) * 131072 * 128
     assert jl.jetlong_prefill_workspace_size(1, 3, 2, 100, 128) == 0  # Hq % Hkv != 0
     assert jl.jetlong_prefill_workspace_size(1, 2, 1, 100, 96) == 0   # unsupported D
     prev = 0
@@ -67,7 +67,7 @@ def test_workspace_sizes(lib):
 
 
 def test_status_strings(lib):
-    for code in range(-8, 1):
+    for code in range(-9, 1):
         assert jl.status_string(code).startswith("JL_")
     assert jl.status_string(5) == "unknown jl_status"
 
@@ -140,3 +140,18 @@ def test_decode_rejects_bad_arguments(lib, kw, status):
 ])
 def test_rope_cache_rejects_bad_arguments(lib, args, status):
     assert lib.jetlong_rope_cache(*args) == status
+
+
+def test_stage_entry_points_check_their_own_buffers(lib):
+    # rotate needs q, k, v; attend needs out; neither accepts a short workspace
+    rot = lambda q=P, k=P, v=P, ws=P, wsb=1 << 40: lib.jetlong_prefill_rotate(
+        q, k, v, 1, 2, 1, 512, 64, 128, 1e4, None, 0, ws, wsb, None)
+    att = lambda out=P, lse=None, ws=P, wsb=1 << 40: lib.jetlong_prefill_attend(
+        out, lse, 1, 2, 1, 512, 64, 128, 32, 0, ws, wsb, None)
+    assert rot(v=None) == jl.JL_ERR_NULL
+    assert rot(k=None) == jl.JL_ERR_NULL
+    assert rot(v=ctypes.c_void_p(264)) == jl.JL_ERR_ALIGN
+    assert rot(wsb=100) == jl.JL_ERR_WORKSPACE
+    assert att(out=None) == jl.JL_ERR_NULL
+    assert att(lse=ctypes.c_void_p(260)) == jl.JL_ERR_ALIGN
+    assert att(ws=None) == jl.JL_ERR_WORKSPACE

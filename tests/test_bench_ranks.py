@@ -1,0 +1,60 @@
+"""The benchmark's multi-rank host logic on CPU (gloo, world size 2).
+
+Each rank runs an independent problem; the report takes the max of the ranks'
+device times and the sum of their work.  No collective touches the data path.
+"""
+import os
+import socket
+
+import pytest
+import torch.multiprocessing as mp
+
+import bench
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, q):
+    import torch.distributed as dist
+    os.environ.update(RANK=str(rank), WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank,
+                            world_size=world)
+    r, w, lr = bench.dist_env()
+    t = bench.reduce_max(10.0 + 5 * rank, w)
+    f = bench.reduce_sum(bench.prefill_flops(1, 32, 1024 * (rank + 1), 128), w)
+    q.put((r, w, lr, t, f))
+    dist.destroy_process_group()
+
+
+def test_two_rank_reductions():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+        assert p.exitcode == 0
+    res = sorted(q.get(timeout=10) for _ in range(2))
+    want_f = bench.prefill_flops(1, 32, 1024, 128) + bench.prefill_flops(1, 32, 2048, 128)
+    for rank, (r, w, lr, t, f) in enumerate(res):
+        assert (r, w, lr) == (rank, 2, rank)
+        assert t == 15.0
+        assert f == want_f
+
+
+def test_single_rank_is_identity():
+    assert bench.reduce_max(3.5, 1) == 3.5
+    assert bench.reduce_sum(7.0, 1) == 7.0
+
+
+def test_work_accounting():
+    # 4 * B * Hq * D * L(L+1)/2 at the headline point
+    assert bench.prefill_flops(1, 32, 131072, 128) == 4 * 32 * 128 * 131072 * 131073 // 2
+    assert bench.decode_bytes(1, 8, 131072, 128) == 2 * 131072 * 8 * 128 * 2
+    assert bench.row_flops(32, 128, [0, 9]) == 4 * 32 * 128 * (1 + 10)

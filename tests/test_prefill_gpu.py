@@ -143,3 +143,30 @@ def test_bad_arguments_launch_nothing():
         jl.jetlong_prefill(q, k, v, w.w_pretrained, w.w0, w.theta, workspace=small)
     assert ei.value.status == jl.JL_ERR_WORKSPACE
     assert jl.jetlong_device_status() == jl.JL_OK
+
+
+def test_staged_calls_equal_the_fused_call():
+    w = WORKLOADS["tiny"].with_(L=900, w_pretrained=256, w0=50)
+    x = prefill_inputs(w)
+    q, k, v = (t.cuda() for t in (x.q, x.k, x.v))
+    out1, lse1 = jl.jetlong_prefill(q, k, v, w.w_pretrained, w.w0, w.theta, out_dtype=torch.float32)
+    ws = torch.empty(jl.jetlong_prefill_workspace_size(w.B, w.Hq, w.Hkv, w.L, w.D),
+                     dtype=torch.uint8, device="cuda")
+    out2 = torch.empty_like(out1)
+    lse2 = torch.empty_like(lse1)
+    jl.jetlong_prefill_rotate(q, k, v, w.w_pretrained, w.theta, ws)
+    jl.jetlong_prefill_attend(out2, lse2, w.Hkv, w.w_pretrained, w.w0, ws)
+    assert jl.jetlong_device_status() == jl.JL_OK
+    assert torch.equal(out1, out2) and torch.equal(lse1, lse2)
+
+
+def test_values_beyond_fp16_range_are_reported():
+    w = WORKLOADS["tiny"]
+    x = prefill_inputs(w)
+    q = x.q.clone()
+    q[0, 5, 1, 3] = 1.0e5  # beyond the FP16 operand range
+    jl.jetlong_prefill(q.cuda(), x.k.cuda(), x.v.cuda(), w.w_pretrained, w.w0, w.theta)
+    assert jl.jetlong_device_status() == jl.JL_ERR_RANGE
+    # the report is cleared once read, and a clean call reports OK again
+    run(w, x=x)
+    assert jl.jetlong_device_status() == jl.JL_OK

@@ -83,7 +83,7 @@ int check_method(int w_pretrained, int w0, float theta) {
 size_t prefill_ws_bytes(int B, int Hq, int Hkv, int L, int D) {
   const size_t q = static_cast<size_t>(B) * Hq * L * D * 2;
   const size_t k = static_cast<size_t>(B) * Hkv * L * D * 2;
-  return 2 * align_up(q) + 2 * align_up(k);
+  return 2 * align_up(q) + 3 * align_up(k);  // q_true, q_remote, k_true, k_remote, v
 }
 
 size_t decode_ws_bytes(int B, int Hq, int Hkv, int L, int D) {
@@ -110,6 +110,7 @@ const char *jetlong_status_string(int s) {
     case JL_ERR_CUDA: return "JL_ERR_CUDA: a CUDA call or launch failed";
     case JL_ERR_DEVICE_TIMEOUT: return "JL_ERR_DEVICE_TIMEOUT: a bounded in-kernel wait expired";
     case JL_ERR_NO_DEVICE: return "JL_ERR_NO_DEVICE: no sm_100 device is current";
+    case JL_ERR_RANGE: return "JL_ERR_RANGE: an input value exceeds the FP16 operand range";
     default: return "unknown jl_status";
   }
 }
@@ -130,21 +131,28 @@ size_t jetlong_prefill_workspace_size(int B, int Hq, int Hkv, int L, int D) {
 
 namespace {
 
-// Validation shared by the prefill entry points.  Pointers that a stage does
-// not use are passed as a non-NULL placeholder by the caller.
-int prepare_prefill(const void *q, const void *k, const void *v, void *out, float *lse, int B,
-                    int Hq, int Hkv, int L, int D, int w_pretrained, int w0, float rope_theta,
-                    int out_dtype, void *k_cache_out, int k_cache_capacity, void *workspace,
-                    size_t workspace_bytes, PrefillArgs *a) {
-  if (!q || !k || !v || !out) return JL_ERR_NULL;
+// Which buffers a prefill entry point reads or writes.
+enum PrefillStage : int { kStageRotate = 1, kStageAttend = 2, kStageBoth = 3 };
+
+// Validation shared by the prefill entry points.  A stage's pointers must be
+// non-NULL and aligned; pointers of the other stage must be NULL and are
+// never handed to a kernel.
+int prepare_prefill(int stage, const void *q, const void *k, const void *v, void *out, float *lse,
+                    int B, int Hq, int Hkv, int L, int D, int w_pretrained, int w0,
+                    float rope_theta, int out_dtype, void *k_cache_out, int k_cache_capacity,
+                    void *workspace, size_t workspace_bytes, PrefillArgs *a) {
+  const bool rot = stage & kStageRotate, att = stage & kStageAttend;
+  if (rot && (!q || !k || !v)) return JL_ERR_NULL;
+  if (att && !out) return JL_ERR_NULL;
   int st = check_common(B, Hq, Hkv, L, D);
   if (st != JL_OK) return st;
   if ((st = check_method(w_pretrained, w0, rope_theta)) != JL_OK) return st;
-  if (out_dtype != JL_BF16 && out_dtype != JL_F32) return JL_ERR_UNSUPPORTED;
-  if (k_cache_out && k_cache_capacity < L) return JL_ERR_SHAPE;
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out) ||
-      (lse && !aligned16(lse)) || (k_cache_out && !aligned16(k_cache_out)))
+  if (att && out_dtype != JL_BF16 && out_dtype != JL_F32) return JL_ERR_UNSUPPORTED;
+  if (rot && k_cache_out && k_cache_capacity < L) return JL_ERR_SHAPE;
+  if (rot && (!aligned16(q) || !aligned16(k) || !aligned16(v) ||
+              (k_cache_out && !aligned16(k_cache_out))))
     return JL_ERR_ALIGN;
+  if (att && (!aligned16(out) || (lse && !aligned16(lse)))) return JL_ERR_ALIGN;
   const size_t need = prefill_ws_bytes(B, Hq, Hkv, L, D);
   if (!workspace || workspace_bytes < need) return JL_ERR_WORKSPACE;
   if (reinterpret_cast<uintptr_t>(workspace) % kAlign) return JL_ERR_ALIGN;
@@ -153,21 +161,22 @@ int prepare_prefill(const void *q, const void *k, const void *v, void *out, floa
   if ((st = current_device(&dev)) != JL_OK) return st;
 
   *a = PrefillArgs{};
-  a->q = static_cast<const __nv_bfloat16 *>(q);
-  a->k = static_cast<const __nv_bfloat16 *>(k);
-  a->v = static_cast<const __nv_bfloat16 *>(v);
-  a->out = out;
-  a->lse = lse;
+  a->q = rot ? static_cast<const __nv_bfloat16 *>(q) : nullptr;
+  a->k = rot ? static_cast<const __nv_bfloat16 *>(k) : nullptr;
+  a->v = rot ? static_cast<const __nv_bfloat16 *>(v) : nullptr;
+  a->out = att ? out : nullptr;
+  a->lse = att ? lse : nullptr;
   a->out_f32 = out_dtype == JL_F32;
-  a->k_cache_out = static_cast<__nv_bfloat16 *>(k_cache_out);
-  a->k_cache_capacity = k_cache_out ? k_cache_capacity : 0;
+  a->k_cache_out = rot ? static_cast<__nv_bfloat16 *>(k_cache_out) : nullptr;
+  a->k_cache_capacity = a->k_cache_out ? k_cache_capacity : 0;
   uint8_t *ws = static_cast<uint8_t *>(workspace);
   const size_t qb = align_up(static_cast<size_t>(B) * Hq * L * D * 2);
   const size_t kb = align_up(static_cast<size_t>(B) * Hkv * L * D * 2);
-  a->q_true = reinterpret_cast<__nv_bfloat16 *>(ws);
-  a->q_remote = reinterpret_cast<__nv_bfloat16 *>(ws + qb);
-  a->k_true = reinterpret_cast<__nv_bfloat16 *>(ws + 2 * qb);
-  a->k_remote = reinterpret_cast<__nv_bfloat16 *>(ws + 2 * qb + kb);
+  a->q_true = reinterpret_cast<__half *>(ws);
+  a->q_remote = reinterpret_cast<__half *>(ws + qb);
+  a->k_true = reinterpret_cast<__half *>(ws + 2 * qb);
+  a->k_remote = reinterpret_cast<__half *>(ws + 2 * qb + kb);
+  a->v_op = reinterpret_cast<__half *>(ws + 2 * qb + 2 * kb);
   a->B = B;
   a->Hq = Hq;
   a->Hkv = Hkv;
@@ -181,9 +190,6 @@ int prepare_prefill(const void *q, const void *k, const void *v, void *out, floa
   return JL_OK;
 }
 
-// Stand-in for a pointer a stage does not read (never dereferenced).
-void *const kUnused = reinterpret_cast<void *>(static_cast<uintptr_t>(256));
-
 }  // namespace
 
 extern "C" {
@@ -193,9 +199,9 @@ int jetlong_prefill(const void *q, const void *k, const void *v, void *out, floa
                     int out_dtype, void *k_cache_out, int k_cache_capacity, void *workspace,
                     size_t workspace_bytes, jl_stream_t stream) {
   PrefillArgs a;
-  const int st = prepare_prefill(q, k, v, out, lse, B, Hq, Hkv, L, D, w_pretrained, w0,
-                                 rope_theta, out_dtype, k_cache_out, k_cache_capacity, workspace,
-                                 workspace_bytes, &a);
+  const int st = prepare_prefill(kStageBoth, q, k, v, out, lse, B, Hq, Hkv, L, D, w_pretrained,
+                                 w0, rope_theta, out_dtype, k_cache_out, k_cache_capacity,
+                                 workspace, workspace_bytes, &a);
   if (st != JL_OK) return st;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (launch_rope_qk(a, s) != cudaSuccess) return JL_ERR_CUDA;
@@ -203,26 +209,26 @@ int jetlong_prefill(const void *q, const void *k, const void *v, void *out, floa
   return JL_OK;
 }
 
-int jetlong_prefill_rotate(const void *q, const void *k, int B, int Hq, int Hkv, int L, int D,
-                           int w_pretrained, float rope_theta, void *k_cache_out,
+int jetlong_prefill_rotate(const void *q, const void *k, const void *v, int B, int Hq, int Hkv,
+                           int L, int D, int w_pretrained, float rope_theta, void *k_cache_out,
                            int k_cache_capacity, void *workspace, size_t workspace_bytes,
                            jl_stream_t stream) {
   PrefillArgs a;
-  const int st = prepare_prefill(q, k, kUnused, kUnused, nullptr, B, Hq, Hkv, L, D, w_pretrained,
-                                 0, rope_theta, JL_BF16, k_cache_out, k_cache_capacity, workspace,
-                                 workspace_bytes, &a);
+  const int st = prepare_prefill(kStageRotate, q, k, v, nullptr, nullptr, B, Hq, Hkv, L, D,
+                                 w_pretrained, 0, rope_theta, JL_BF16, k_cache_out,
+                                 k_cache_capacity, workspace, workspace_bytes, &a);
   if (st != JL_OK) return st;
   if (launch_rope_qk(a, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return JL_ERR_CUDA;
   return JL_OK;
 }
 
-int jetlong_prefill_attend(const void *v, void *out, float *lse, int B, int Hq, int Hkv, int L,
-                           int D, int w_pretrained, int w0, int out_dtype, const void *workspace,
+int jetlong_prefill_attend(void *out, float *lse, int B, int Hq, int Hkv, int L, int D,
+                           int w_pretrained, int w0, int out_dtype, const void *workspace,
                            size_t workspace_bytes, jl_stream_t stream) {
   PrefillArgs a;
-  const int st = prepare_prefill(kUnused, kUnused, v, out, lse, B, Hq, Hkv, L, D, w_pretrained, w0,
-                                 1.0f, out_dtype, nullptr, 0, const_cast<void *>(workspace),
-                                 workspace_bytes, &a);
+  const int st = prepare_prefill(kStageAttend, nullptr, nullptr, nullptr, out, lse, B, Hq, Hkv, L,
+                                 D, w_pretrained, w0, 1.0f, out_dtype, nullptr, 0,
+                                 const_cast<void *>(workspace), workspace_bytes, &a);
   if (st != JL_OK) return st;
   if (launch_prefill_attention(a, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
     return JL_ERR_CUDA;
@@ -310,7 +316,7 @@ int jetlong_device_status(jl_stream_t stream) {
   if (flag != kDevOk) {
     const unsigned int zero = 0;
     if (cudaMemcpyToSymbol(g_device_error, &zero, sizeof(zero)) != cudaSuccess) return JL_ERR_CUDA;
-    return JL_ERR_DEVICE_TIMEOUT;
+    return (flag & kDevTimeout) ? JL_ERR_DEVICE_TIMEOUT : JL_ERR_RANGE;
   }
   return JL_OK;
 }

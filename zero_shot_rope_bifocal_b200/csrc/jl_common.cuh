@@ -4,6 +4,7 @@
 #pragma once
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 #include <climits>
@@ -11,15 +12,17 @@
 
 namespace jl {
 
-// Kernel-side error codes written to the device error word.
+// Kernel-side error bits written to the device error word.
 enum : unsigned int {
   kDevOk = 0u,
-  kDevTimeout = 1u,
+  kDevTimeout = 1u,   // a bounded wait expired
+  kDevRange = 2u,     // an operand left the FP16 range of the MMA operands
 };
 
 // Time limit for any single in-kernel wait.  Every legitimate wait in these
-// kernels lasts micro- to milliseconds; two seconds means a lost arrival.
-constexpr uint64_t kWaitLimitNs = 2000000000ull;
+// kernels (a TMA tile landing, an MMA group finishing) lasts microseconds;
+// a quarter of a second means a lost arrival.
+constexpr uint64_t kWaitLimitNs = 250000000ull;
 
 // §3.1, Eq. (2): G = max(1, ceil(L / w_pretrained)), integer arithmetic.
 __host__ __device__ __forceinline__ int group_size(int L, int w_pretrained) {
@@ -60,8 +63,9 @@ struct PrefillArgs {
   int out_f32;
   __nv_bfloat16 *k_cache_out;
   int k_cache_capacity;
-  // rotated operands in the workspace, head-major [B, H, L, D]
-  __nv_bfloat16 *q_true, *q_remote, *k_true, *k_remote;
+  // MMA operands in the workspace, FP16 head-major [B, H, L, D]: queries and
+  // keys rotated to true / remote positions, and the values
+  __half *q_true, *q_remote, *k_true, *k_remote, *v_op;
   // sizes and method parameters
   int B, Hq, Hkv, L, D, w_pretrained, w0, G;
   float theta;

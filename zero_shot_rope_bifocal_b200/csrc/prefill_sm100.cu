@@ -20,21 +20,26 @@
 // G == 1 (L <= w_pretrained) f is the identity and every tile is a plain
 // causal "local" visit: the native-window case of Appendix H.
 //
+// Operands: the RoPE pass leaves q/k (both variants) and v in the workspace as
+// FP16, head-major [B, H, L, D].  FP16 keeps three more mantissa bits than
+// BF16 for the rotated values the tensor core must consume in 16 bits.
+//
 // Hardware mapping (one CTA = one 128-row query tile of one head; 4 warps):
 //   * TMA (128-byte swizzle) loads the query tile once per variant and K / V
 //     tiles into a two-slot ring; mbarriers with expect-tx track arrival;
 //   * thread 0 issues tcgen05.mma: S = Q K^T (M=128, N=128, K=D) into TMEM,
 //     later O += P V with P read from TMEM (M=128, N=D, K=128);
 //   * every thread owns one query row = one TMEM lane: it loads its S row,
-//     applies the mask, runs the online softmax in base 2 (fp32 statistics,
-//     BF16 P as the pages' precision statement in Appendix H), rescales its O
-//     row only when the running max grew by more than 2^8, and stores P;
+//     applies the mask, runs the online softmax in base 2 (fp32 statistics),
+//     rescales its O row only when the running max grew by more than 2^8
+//     (decided per warp, since TMEM loads and stores are warp-collective),
+//     and stores P (FP16) to TMEM;
 //   * the epilogue divides O by the row sum and writes O and the natural-log
 //     LSE.
-// Each wait is bounded in time (see jl::kWaitLimitNs); on expiry the CTA
-// records a device error, drains its own MMAs, frees TMEM and exits.
+// Each wait is bounded in time (jl::kWaitLimitNs); on expiry the CTA records a
+// device error, drains its own MMAs, frees TMEM and exits, and CTAs that start
+// after a recorded error skip their work.
 #include <cmath>
-#include <cstdio>
 
 #include "jl_common.cuh"
 #include "sm100_ptx.cuh"
@@ -46,10 +51,11 @@ constexpr int BM = 128;  // query rows per tile (= TMEM lanes)
 constexpr int BN = 128;  // keys per tile
 constexpr int kThreads = 128;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
+constexpr uint32_t kF16 = 0;               // operand format code of kind::f16
 
 template <int D>
 struct Layout {
-  static constexpr int TILE = BM * D * 2;       // bytes of one 128 x D BF16 tile
+  static constexpr int TILE = BM * D * 2;       // bytes of one 128 x D 16-bit tile
   static constexpr int BOX = 128 * 128;         // bytes of one 128-row x 64-col swizzled box
   static constexpr int Q = 0;
   static constexpr int K0 = TILE;
@@ -94,6 +100,7 @@ bifocal_prefill_kernel(const __grid_constant__ CUtensorMap tm_qt,
   const uint32_t bar_s = sb + LY::BAR + 24;
   const uint32_t bar_o = sb + LY::BAR + 32;
   const uint32_t tmem_slot = sb + LY::BAR + 40;
+  volatile uint32_t *skip_flag = reinterpret_cast<volatile uint32_t *>(smem + LY::BAR + 44);
 
   const int tid = threadIdx.x, warp = tid >> 5;
   const int qt = prm.n_qt - 1 - static_cast<int>(blockIdx.x);  // longest rows first
@@ -106,7 +113,8 @@ bifocal_prefill_kernel(const __grid_constant__ CUtensorMap tm_qt,
   const int w0 = prm.w0eff;
 
   // Visit plan: remote visits of key tiles [0, n_rem), then local visits of
-  // key tiles [kl0, n_kt).
+  // key tiles [kl0, n_kt).  Every causal pair of the tile is kept by exactly
+  // one visit.
   const int n_kt = p1 / BN + 1;
   int n_rem = 0, kl0 = 0;
   if (prm.G > 1) {
@@ -114,6 +122,13 @@ bifocal_prefill_kernel(const __grid_constant__ CUtensorMap tm_qt,
     kl0 = max(0, p0 - w0) / BN;
   }
   const int nv = n_rem + (n_kt - kl0);
+
+  // Once any CTA has recorded a failure, the others skip their work, so a
+  // broken launch ends after one wait limit instead of one per CTA wave.
+  // Thread 0 reads the word and the whole CTA follows its answer.
+  if (tid == 0) *skip_flag = *reinterpret_cast<volatile unsigned int *>(prm.dev_error);
+  __syncthreads();
+  if (*skip_flag != kDevOk) return;
 
   if (tid == 0) {
     mbar_init(bar_q, 1);
@@ -137,13 +152,13 @@ bifocal_prefill_kernel(const __grid_constant__ CUtensorMap tm_qt,
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(smem + LY::BAR + 40);
-  const uint32_t tS = tmem;          // S: 128 columns fp32
-  const uint32_t tO = tmem + 128;    // O: D columns fp32
-  const uint32_t tP = tmem + 128 + D; // P: 64 columns of packed BF16 pairs
+  const uint32_t tS = tmem;            // S: 128 columns fp32
+  const uint32_t tO = tmem + 128;      // O: D columns fp32
+  const uint32_t tP = tmem + 128 + D;  // P: 64 columns of packed FP16 pairs
   const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
 
-  constexpr uint32_t IDESC_QK = idesc_bf16_f32(BM, BN, false, false);
-  constexpr uint32_t IDESC_PV = idesc_bf16_f32(BM, D, false, true);
+  constexpr uint32_t IDESC_QK = idesc_f16kind_f32(BM, BN, kF16, false, false);
+  constexpr uint32_t IDESC_PV = idesc_f16kind_f32(BM, D, kF16, false, true);
   constexpr int NBOX = D / 64;
 
   auto load_q = [&](bool remote) {
@@ -158,7 +173,7 @@ bifocal_prefill_kernel(const __grid_constant__ CUtensorMap tm_qt,
     for (int c = 0; c < NBOX; ++c) {
       tma_load_3d(sK[slot] + c * LY::BOX, remote ? &tm_kr : &tm_kt, bar_kv[slot], c * 64, kt * BN,
                   b * prm.Hkv + hk);
-      tma_load_4d(sV[slot] + c * LY::BOX, &tm_v, bar_kv[slot], c * 64, hk, kt * BN, b);
+      tma_load_3d(sV[slot] + c * LY::BOX, &tm_v, bar_kv[slot], c * 64, kt * BN, b * prm.Hkv + hk);
     }
   };
 
@@ -177,14 +192,15 @@ bifocal_prefill_kernel(const __grid_constant__ CUtensorMap tm_qt,
     const int slot = vt & 1;
     if (tid == 0 && ok) {
       if (vt == 0 || vt == n_rem) ok = mbar_wait_bounded(bar_q, vt == 0 ? 0u : 1u, kWaitLimitNs);
-      if (ok) ok = mbar_wait_bounded(bar_kv[slot], static_cast<uint32_t>(vt >> 1) & 1u, kWaitLimitNs);
+      if (ok)
+        ok = mbar_wait_bounded(bar_kv[slot], static_cast<uint32_t>(vt >> 1) & 1u, kWaitLimitNs);
       if (ok) {
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * LY::BOX + (kk & 3) * 32;
-          mma_bf16_ss(tS, smem_desc_sw128(sQ + off, 16, 1024), smem_desc_sw128(sK[slot] + off, 16, 1024),
-                      IDESC_QK, kk > 0 ? 1u : 0u);
+          mma_f16kind_ss(tS, smem_desc_sw128(sQ + off, 16, 1024),
+                         smem_desc_sw128(sK[slot] + off, 16, 1024), IDESC_QK, kk > 0 ? 1u : 0u);
         }
         mma_commit(bar_s);
       }
@@ -202,7 +218,8 @@ bifocal_prefill_kernel(const __grid_constant__ CUtensorMap tm_qt,
       load_kv(vt + 1, slot ^ 1);
     }
 
-    // ---- softmax on this thread's row
+    // ---- softmax on this thread's row (TMEM accesses are warp-collective:
+    // every branch around them below is warp-uniform)
     float x[BN];
     {
       uint32_t r[BN / 32][32];
@@ -233,25 +250,27 @@ bifocal_prefill_kernel(const __grid_constant__ CUtensorMap tm_qt,
     float tmax = -INFINITY;
 #pragma unroll
     for (int c = 0; c < BN; ++c) tmax = fmaxf(tmax, x[c]);
-    if (tmax > m_used + kRescaleThreshold || (m_used == -INFINITY && tmax > -INFINITY)) {
-      const float m_new = tmax;
-      if (m_used != -INFINITY) {
-        const float alpha = exp2f(m_used - m_new);
-        l_sum *= alpha;
-        if (vt > 0) {
+    const bool grow = tmax > m_used + kRescaleThreshold || (m_used == -INFINITY && tmax > -INFINITY);
+    float alpha = 1.f;  // factor applied to this row's O and l
+    if (grow) {
+      if (m_used != -INFINITY) alpha = exp2f(m_used - tmax);
+      m_used = tmax;
+    }
+    l_sum *= alpha;
+    // O holds data from visit 1 on (visit 0 overwrites it); rows whose max was
+    // -inf have O = 0 there, so alpha = 1 keeps them exact.
+    if (vt > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+      __syncwarp();
 #pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t r[32];
-            tmem_ld32(tO + lane_base + c * 32, r);
-            tmem_wait_ld();
-            reg_fence(r);
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t r[32];
+        tmem_ld32(tO + lane_base + c * 32, r);
+        tmem_wait_ld();
+        reg_fence(r);
 #pragma unroll
-            for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(u2f(r[e]) * alpha);
-            tmem_st32(tO + lane_base + c * 32, r);
-          }
-        }
+        for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(u2f(r[e]) * alpha);
+        tmem_st32(tO + lane_base + c * 32, r);
       }
-      m_used = m_new;
     }
     float lsum = 0.f;
     if (m_used == -INFINITY) {
@@ -265,12 +284,13 @@ bifocal_prefill_kernel(const __grid_constant__ CUtensorMap tm_qt,
       }
     }
     l_sum += lsum;
+    __syncwarp();
 #pragma unroll
     for (int c = 0; c < BN / 64; ++c) {
       uint32_t r[32];
 #pragma unroll
       for (int e = 0; e < 32; ++e) {
-        const __nv_bfloat162 pr = __floats2bfloat162_rn(x[c * 64 + 2 * e], x[c * 64 + 2 * e + 1]);
+        const __half2 pr = __floats2half2_rn(x[c * 64 + 2 * e], x[c * 64 + 2 * e + 1]);
         r[e] = *reinterpret_cast<const uint32_t *>(&pr);
       }
       tmem_st32(tP + lane_base + c * 32, r);
@@ -282,8 +302,8 @@ bifocal_prefill_kernel(const __grid_constant__ CUtensorMap tm_qt,
       tc_fence_after();
 #pragma unroll
       for (int kk = 0; kk < BN / 16; ++kk)
-        mma_bf16_ts(tO, tP + kk * 8, smem_desc_sw128(sV[slot] + kk * 16 * 128, LY::BOX, 1024),
-                    IDESC_PV, (vt > 0 || kk > 0) ? 1u : 0u);
+        mma_f16kind_ts(tO, tP + kk * 8, smem_desc_sw128(sV[slot] + kk * 16 * 128, LY::BOX, 1024),
+                       IDESC_PV, (vt > 0 || kk > 0) ? 1u : 0u);
     }
   }
 
@@ -291,17 +311,20 @@ bifocal_prefill_kernel(const __grid_constant__ CUtensorMap tm_qt,
   if (tid == 0) mma_commit(bar_o);
   const bool drained = mbar_wait_bounded(bar_o, 0u, kWaitLimitNs);
   tc_fence_after();
-  if (!ok || !drained) {
+  const bool good = __syncthreads_and(ok && drained);
+  if (!good) {
     if (tid == 0) atomicOr(prm.dev_error, kDevTimeout);
-  } else if (row_ok) {
-    const float inv_l = 1.f / l_sum;
+  } else {
+    const float inv_l = row_ok ? 1.f / l_sum : 0.f;
     const size_t obase = ((static_cast<size_t>(b) * prm.L + row) * prm.Hq + h) * D;
 #pragma unroll
     for (int c = 0; c < D / 32; ++c) {
       uint32_t r[32];
-      tmem_ld32(tO + lane_base + c * 32, r);
+      __syncwarp();
+      tmem_ld32(tO + lane_base + c * 32, r);  // whole warp, valid row or not
       tmem_wait_ld();
       reg_fence(r);
+      if (!row_ok) continue;
       if (prm.out_f32) {
         float4 *dst = reinterpret_cast<float4 *>(reinterpret_cast<float *>(prm.out) + obase + c * 32);
 #pragma unroll
@@ -323,7 +346,7 @@ bifocal_prefill_kernel(const __grid_constant__ CUtensorMap tm_qt,
         }
       }
     }
-    if (prm.lse)
+    if (row_ok && prm.lse)
       prm.lse[(static_cast<size_t>(b) * prm.Hq + h) * prm.L + row] =
           (m_used + log2f(l_sum)) * 0.69314718055994531f;
   }
@@ -350,7 +373,7 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// Head-major operand [BH, L, D] BF16: box = 64 channels x 128 tokens of one head.
+// Head-major operand [BH, L, D] FP16: box = 64 channels x 128 tokens of one head.
 bool encode_head_major(CUtensorMap *tm, const void *base, int BH, int L, int D) {
   const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(L),
                               static_cast<cuuint64_t>(BH)};
@@ -358,21 +381,7 @@ bool encode_head_major(CUtensorMap *tm, const void *base, int BH, int L, int D) 
                                  static_cast<cuuint64_t>(L) * D * 2};
   const cuuint32_t box[3] = {64, 128, 1};
   const cuuint32_t estr[3] = {1, 1, 1};
-  return encode_fn()(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides,
-                     box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
-         CUDA_SUCCESS;
-}
-
-// Caller's V [B, L, Hkv, D] BF16: box = 64 channels x 1 head x 128 tokens.
-bool encode_token_major(CUtensorMap *tm, const void *base, int B, int L, int H, int D) {
-  const cuuint64_t dims[4] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(H),
-                              static_cast<cuuint64_t>(L), static_cast<cuuint64_t>(B)};
-  const cuuint64_t strides[3] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(H) * D * 2,
-                                 static_cast<cuuint64_t>(L) * H * D * 2};
-  const cuuint32_t box[4] = {64, 1, 128, 1};
-  const cuuint32_t estr[4] = {1, 1, 1, 1};
-  return encode_fn()(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void *>(base), dims, strides,
+  return encode_fn()(tm, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, const_cast<void *>(base), dims, strides,
                      box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                      CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
          CUDA_SUCCESS;
@@ -387,7 +396,7 @@ cudaError_t launch_d(const PrefillArgs &a, cudaStream_t stream) {
       !encode_head_major(&tqr, two ? a.q_remote : a.q_true, a.B * a.Hq, a.L, D) ||
       !encode_head_major(&tkt, a.k_true, a.B * a.Hkv, a.L, D) ||
       !encode_head_major(&tkr, two ? a.k_remote : a.k_true, a.B * a.Hkv, a.L, D) ||
-      !encode_token_major(&tv, a.v, a.B, a.L, a.Hkv, D))
+      !encode_head_major(&tv, a.v_op, a.B * a.Hkv, a.L, D))
     return cudaErrorInvalidValue;
   Params prm;
   prm.B = a.B;

@@ -8,9 +8,13 @@
 //   k_true[b,g,j]  = RoPE(x_k, j)      k_remote[b,g,j] = RoPE(x_k, f(j))
 //
 // k_true is exactly the true-position KV cache of §3.2, and k_remote equals
-// the correction rotation by Delta j = f(j) - j applied to it.  The outputs are
-// head-major [B, H, L, D] BF16 so that the attention kernel's TMA fetches each
-// 128-token tile as one contiguous block.  When G == 1 (L <= w_pretrained,
+// the correction rotation by Delta j = f(j) - j applied to it.  The outputs
+// (and a copy of v) are the tensor-core operands: FP16, head-major
+// [B, H, L, D], so that the attention kernel's TMA fetches each 128-token tile
+// as one contiguous block.  FP16 holds the rotated values with three more
+// mantissa bits than BF16; a value beyond the FP16 range (|x| > 65504) is
+// reported through the device error word.  The optional cache output keeps
+// the caller's BF16 format.  When G == 1 (L <= w_pretrained,
 // the native-window case of Appendix H) f is the identity and only the
 // true-position arrays are written.
 //
@@ -27,18 +31,36 @@ namespace {
 constexpr int kRopeThreads = 256;
 constexpr int kPosPerCta = 4;
 
-// Rotate BF16 pairs (a[i], a[i+D/2]) and (a[i+1], a[i+1+D/2]) of one head row.
-__device__ __forceinline__ void rotate2(const __nv_bfloat16 *src, __nv_bfloat16 *dst, int i, int half,
-                                        float2 cs0, float2 cs1) {
+// Rotated pairs (a[i], a[i+D/2]) and (a[i+1], a[i+1+D/2]) of one BF16 head row,
+// in fp32: returns (r0, r1) for channels i, i+1 and (s0, s1) for i+D/2, i+1+D/2.
+struct Rot2 {
+  float r0, r1, s0, s1;
+};
+
+__device__ __forceinline__ Rot2 rotate2(const __nv_bfloat16 *src, int i, int half, float2 cs0,
+                                        float2 cs1) {
   const __nv_bfloat162 lo = *reinterpret_cast<const __nv_bfloat162 *>(src + i);
   const __nv_bfloat162 hi = *reinterpret_cast<const __nv_bfloat162 *>(src + i + half);
   const float a0 = __low2float(lo), a1 = __high2float(lo);
   const float b0 = __low2float(hi), b1 = __high2float(hi);
   // cs = (cos, sin)
-  const float r0 = a0 * cs0.x - b0 * cs0.y, s0 = a0 * cs0.y + b0 * cs0.x;
-  const float r1 = a1 * cs1.x - b1 * cs1.y, s1 = a1 * cs1.y + b1 * cs1.x;
-  *reinterpret_cast<__nv_bfloat162 *>(dst + i) = __floats2bfloat162_rn(r0, r1);
-  *reinterpret_cast<__nv_bfloat162 *>(dst + i + half) = __floats2bfloat162_rn(s0, s1);
+  return {a0 * cs0.x - b0 * cs0.y, a1 * cs1.x - b1 * cs1.y, a0 * cs0.y + b0 * cs0.x,
+          a1 * cs1.y + b1 * cs1.x};
+}
+
+__device__ __forceinline__ void store_bf16(__nv_bfloat16 *dst, int i, int half, const Rot2 &v) {
+  *reinterpret_cast<__nv_bfloat162 *>(dst + i) = __floats2bfloat162_rn(v.r0, v.r1);
+  *reinterpret_cast<__nv_bfloat162 *>(dst + i + half) = __floats2bfloat162_rn(v.s0, v.s1);
+}
+
+// FP16 MMA operand; returns false if a value left the FP16 range.
+__device__ __forceinline__ bool store_f16(__half *dst, int i, int half, const Rot2 &v) {
+  const __half2 lo = __floats2half2_rn(v.r0, v.r1);
+  const __half2 hi = __floats2half2_rn(v.s0, v.s1);
+  *reinterpret_cast<__half2 *>(dst + i) = lo;
+  *reinterpret_cast<__half2 *>(dst + i + half) = hi;
+  return !(__hisinf(__low2half(lo)) | __hisinf(__high2half(lo)) | __hisinf(__low2half(hi)) |
+           __hisinf(__high2half(hi)));
 }
 
 __global__ void __launch_bounds__(kRopeThreads)
@@ -65,6 +87,7 @@ rope_qk_kernel(PrefillArgs a) {
   }
   __syncthreads();
 
+  bool in_range = true;
   const int quarter = a.D / 4;  // pairs of channel pairs per head row
   // queries
   for (int idx = threadIdx.x; idx < npos * a.Hq * quarter; idx += blockDim.x) {
@@ -75,30 +98,37 @@ rope_qk_kernel(PrefillArgs a) {
     const int pos = p_begin + t;
     const __nv_bfloat16 *src = a.q + ((static_cast<size_t>(b) * a.L + pos) * a.Hq + h) * a.D;
     const size_t drow = ((static_cast<size_t>(b) * a.Hq + h) * a.L + pos) * a.D;
-    rotate2(src, a.q_true + drow, i, half, cs_true[t * half + i], cs_true[t * half + i + 1]);
+    in_range &= store_f16(a.q_true + drow, i, half,
+                          rotate2(src, i, half, cs_true[t * half + i], cs_true[t * half + i + 1]));
     if (two)
-      rotate2(src, a.q_remote + drow, i, half, cs_remote[t * half + i],
-              cs_remote[t * half + i + 1]);
+      in_range &= store_f16(a.q_remote + drow, i, half,
+                            rotate2(src, i, half, cs_remote[t * half + i],
+                                    cs_remote[t * half + i + 1]));
   }
-  // keys (+ optional true-position cache)
+  // keys (+ optional true-position cache) and values
   for (int idx = threadIdx.x; idx < npos * a.Hkv * quarter; idx += blockDim.x) {
     const int t = idx / (a.Hkv * quarter);
     const int rem = idx - t * a.Hkv * quarter;
     const int g = rem / quarter;
     const int i = (rem - g * quarter) * 2;
     const int pos = p_begin + t;
-    const __nv_bfloat16 *src = a.k + ((static_cast<size_t>(b) * a.L + pos) * a.Hkv + g) * a.D;
+    const size_t srow = ((static_cast<size_t>(b) * a.L + pos) * a.Hkv + g) * a.D;
+    const __nv_bfloat16 *src = a.k + srow;
     const size_t drow = ((static_cast<size_t>(b) * a.Hkv + g) * a.L + pos) * a.D;
-    rotate2(src, a.k_true + drow, i, half, cs_true[t * half + i], cs_true[t * half + i + 1]);
+    const Rot2 kt = rotate2(src, i, half, cs_true[t * half + i], cs_true[t * half + i + 1]);
+    in_range &= store_f16(a.k_true + drow, i, half, kt);
     if (two)
-      rotate2(src, a.k_remote + drow, i, half, cs_remote[t * half + i],
-              cs_remote[t * half + i + 1]);
-    if (a.k_cache_out) {
-      __nv_bfloat16 *crow =
-          a.k_cache_out + ((static_cast<size_t>(b) * a.k_cache_capacity + pos) * a.Hkv + g) * a.D;
-      rotate2(src, crow, i, half, cs_true[t * half + i], cs_true[t * half + i + 1]);
-    }
+      in_range &= store_f16(a.k_remote + drow, i, half,
+                            rotate2(src, i, half, cs_remote[t * half + i],
+                                    cs_remote[t * half + i + 1]));
+    if (a.k_cache_out)
+      store_bf16(a.k_cache_out + ((static_cast<size_t>(b) * a.k_cache_capacity + pos) * a.Hkv + g) * a.D,
+                 i, half, kt);
+    // values: the identity rotation, i.e. a BF16 -> FP16 copy into head-major order
+    in_range &= store_f16(a.v_op + drow, i, half,
+                          rotate2(a.v + srow, i, half, make_float2(1.f, 0.f), make_float2(1.f, 0.f)));
   }
+  if (!in_range) atomicOr(a.dev_error, kDevRange);
 }
 
 __global__ void __launch_bounds__(kRopeThreads)
@@ -126,7 +156,7 @@ rope_cache_kernel(const __nv_bfloat16 *__restrict__ k, __nv_bfloat16 *__restrict
     const __nv_bfloat16 *src = k + ((static_cast<size_t>(b) * n + t_begin + t) * Hkv + g) * D;
     __nv_bfloat16 *dst =
         k_cache + ((static_cast<size_t>(b) * Lcap + pos0 + t_begin + t) * Hkv + g) * D;
-    rotate2(src, dst, i, half, cs_smem[t * half + i], cs_smem[t * half + i + 1]);
+    store_bf16(dst, i, half, rotate2(src, i, half, cs_smem[t * half + i], cs_smem[t * half + i + 1]));
   }
 }
 

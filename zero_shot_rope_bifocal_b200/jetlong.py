@@ -28,6 +28,7 @@ JL_ERR_WORKSPACE = -5
 JL_ERR_CUDA = -6
 JL_ERR_DEVICE_TIMEOUT = -7
 JL_ERR_NO_DEVICE = -8
+JL_ERR_RANGE = -9
 JL_BF16 = 0
 JL_F32 = 1
 
@@ -40,8 +41,9 @@ SIGNATURES = {
     "jetlong_prefill_workspace_size": (_SZ, [_I, _I, _I, _I, _I]),
     "jetlong_prefill": (_I, [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _I, _F, _I,
                              _VP, _I, _VP, _SZ, _VP]),
-    "jetlong_prefill_rotate": (_I, [_VP, _VP, _I, _I, _I, _I, _I, _I, _F, _VP, _I, _VP, _SZ, _VP]),
-    "jetlong_prefill_attend": (_I, [_VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _I, _I, _VP, _SZ, _VP]),
+    "jetlong_prefill_rotate": (_I, [_VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _F, _VP, _I, _VP, _SZ,
+                                    _VP]),
+    "jetlong_prefill_attend": (_I, [_VP, _VP, _I, _I, _I, _I, _I, _I, _I, _I, _VP, _SZ, _VP]),
     "jetlong_decode_workspace_size": (_SZ, [_I, _I, _I, _I, _I]),
     "jetlong_decode": (_I, [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _I, _I, _F, _I,
                             _VP, _SZ, _VP]),
@@ -173,31 +175,33 @@ def jetlong_prefill(q, k, v, w_pretrained: int, w0: int, rope_theta: float, *,
     return out, lse
 
 
-def jetlong_prefill_rotate(q, k, w_pretrained: int, rope_theta: float, workspace, *,
+def jetlong_prefill_rotate(q, k, v, w_pretrained: int, rope_theta: float, workspace, *,
                            k_cache_out=None, stream=None):
-    """Stage 1 of jetlong_prefill: rotated Q/K operands into ``workspace``."""
+    """Stage 1 of jetlong_prefill: the FP16 tensor-core operands into ``workspace``."""
     B, L, Hq, D = q.shape
     Hkv = k.shape[2]
     _require(q, "q", (B, L, Hq, D), torch.bfloat16)
     _require(k, "k", (B, L, Hkv, D), torch.bfloat16)
+    _require(v, "v", (B, L, Hkv, D), torch.bfloat16)
     cap = 0 if k_cache_out is None else k_cache_out.shape[1]
     if k_cache_out is not None:
         _require(k_cache_out, "k_cache_out", (B, cap, Hkv, D), torch.bfloat16)
-    st = lib().jetlong_prefill_rotate(_ptr(q), _ptr(k), B, Hq, Hkv, L, D, int(w_pretrained),
-                                      float(rope_theta), _ptr(k_cache_out), cap, _ptr(workspace),
-                                      workspace.numel(), _stream_ptr(stream))
+    st = lib().jetlong_prefill_rotate(_ptr(q), _ptr(k), _ptr(v), B, Hq, Hkv, L, D,
+                                      int(w_pretrained), float(rope_theta), _ptr(k_cache_out), cap,
+                                      _ptr(workspace), workspace.numel(), _stream_ptr(stream))
     _check("jetlong_prefill_rotate", st)
 
 
-def jetlong_prefill_attend(v, out, lse, Hq: int, w_pretrained: int, w0: int, workspace, *,
+def jetlong_prefill_attend(out, lse, Hkv: int, w_pretrained: int, w0: int, workspace, *,
                            stream=None):
-    """Stage 2 of jetlong_prefill: the attention kernel on the rotated operands."""
-    B, L, Hkv, D = v.shape
-    _require(v, "v", (B, L, Hkv, D), torch.bfloat16)
+    """Stage 2 of jetlong_prefill: the attention kernel on the operands in ``workspace``."""
+    if out.dim() != 4:
+        raise ValueError("out must be [B, L, Hq, D]")
+    B, L, Hq, D = out.shape
     _require(out, "out", (B, L, Hq, D), out.dtype)
     if lse is not None:
         _require(lse, "lse", (B, Hq, L), torch.float32)
-    st = lib().jetlong_prefill_attend(_ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, L, D,
+    st = lib().jetlong_prefill_attend(_ptr(out), _ptr(lse), B, Hq, int(Hkv), L, D,
                                       int(w_pretrained), int(w0), _out_dtype(out.dtype),
                                       _ptr(workspace), workspace.numel(), _stream_ptr(stream))
     _check("jetlong_prefill_attend", st)
