@@ -172,6 +172,7 @@ JL_API size_t jetlong_decode_workspace_size(int B, int Hq, int Hkv, int L, int D
  *      scored against RoPE(x_q, f(L-1)).
  *   workspace: >= jetlong_decode_workspace_size(B, Hq, Hkv, L, D) bytes,
  *      256-byte aligned; contents on entry do not matter.
+ *   Hq / Hkv must be 1, 2, 4 or 8 (JL_ERR_UNSUPPORTED otherwise).
  */
 JL_API int jetlong_decode(const void *q, const void *k_cache, const void *v_cache, void *out,
                    float *lse, int B, int Hq, int Hkv, int L, int Lcap, int D,

@@ -122,6 +122,8 @@ def decode_call(lib, **kw):
     (dict(Lcap=999), jl.JL_ERR_SHAPE),
     (dict(L=0), jl.JL_ERR_SHAPE),
     (dict(Hq=34, Hkv=2), jl.JL_ERR_UNSUPPORTED),   # group of 17 query heads
+    (dict(Hq=48, Hkv=8), jl.JL_ERR_UNSUPPORTED),   # group of 6 query heads
+    (dict(Hq=32, Hkv=2), jl.JL_ERR_UNSUPPORTED),   # group of 16 query heads
     (dict(D=80), jl.JL_ERR_UNSUPPORTED),
     (dict(w0=-5), jl.JL_ERR_SHAPE),
     (dict(vc=ctypes.c_void_p(8)), jl.JL_ERR_ALIGN),

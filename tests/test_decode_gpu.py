@@ -46,8 +46,9 @@ def test_tiny_decode_lengths(L):
 
 
 @pytest.mark.parametrize("Hq,Hkv,D,wp,w0,L", [
-    (8, 2, 128, 64, 0, 1000), (3, 3, 64, 100, 7, 777), (16, 1, 128, 512, 600, 2048),
-    (32, 8, 128, 1024, 100, 5000), (4, 2, 64, 1, 3, 200)])
+    (8, 2, 128, 64, 0, 1000), (3, 3, 64, 100, 7, 777), (8, 1, 128, 512, 600, 2048),
+    (32, 8, 128, 1024, 100, 5000), (4, 2, 64, 1, 3, 200), (16, 16, 128, 300, 50, 3000),
+    (64, 8, 128, 2048, 1000, 9000), (24, 12, 64, 500, 20, 4100), (8, 8, 128, 128, 10, 17)])
 def test_decode_shapes(Hq, Hkv, D, wp, w0, L):
     w = Workload("dec", 2, Hq, Hkv, D, L, wp, w0, 1e6, 30 + L, False, kind="decode")
     d = decode_inputs(w, Lcap=L + 5)

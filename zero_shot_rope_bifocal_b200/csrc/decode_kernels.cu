@@ -3,218 +3,348 @@
 // correction rotation"; score rule of §3; schedule of §3.1 with L = tokens in
 // the cache including the new one, query at p = L - 1).
 //
-// Split-KV: the key range [0, L) is cut into n_split chunks; CTA (s, g, b)
-// streams chunk s of KV head g for every query head of that group and keeps
-// an online softmax per head.  Keys with p - j <= w0 are scored as cached
-// against RoPE(x_q, p); older keys are rotated in shared memory by
-// Delta j = f(j) - j (the correction rotation, so the cache is never
-// rewritten) and scored against RoPE(x_q, f(p)).  Each CTA writes its
-// unnormalised partial output with its running max and sum to the workspace;
-// a second kernel merges the partials by log-sum-exp, one warp per head.
+// Split-KV: CTA (s, c, b) streams key chunk s of KV heads [8c, 8c + 8) of
+// batch b through a three-stage shared-memory ring filled by bulk async copies
+// (cp.async.bulk + mbarrier transaction counts): each stage holds P tokens of
+// K and V for the CTA's heads, which are contiguous in the cache.  Warp w owns
+// KV head 8c + w and its Hq/Hkv query heads; lane l holds channel pairs
+// (i, i + D/2) for i in {2l, 2l+1} (D = 128) or {l} (D = 64), so the
+// correction rotation of a pair is lane-local.
 //
-// Traffic: the kernel reads K and V once (2 * L * Hkv * D * 2 bytes per
-// token); everything else is O(Hq * D * n_split).
+// Per token j: keys with p - j <= w0 are scored as cached against
+// RoPE(x_q, p); older keys are first rotated by Delta j = f(j) - j (the
+// correction rotation, so the cache is never rewritten) and scored against
+// RoPE(x_q, f(p)).  cos/sin of Delta j * theta_i are evaluated once per token
+// per CTA (double-precision angle, reduced, then the hardware sine/cosine on
+// [-pi, pi]) and shared by all heads.  The partial dot products of a batch of
+// tokens x query heads (32 values per lane) are summed across the warp by a
+// reduce-scatter that leaves one (token, head) score per lane; an online
+// softmax per head then weights V.  Each CTA writes its unnormalised partial
+// output with its running max and sum; a second kernel merges the partials by
+// log-sum-exp, one warp per head.
+//
+// Traffic: K and V once (2 * L * Hkv * D * 2 bytes per token of output);
+// everything else is O(Hq * D * n_split).
 #include <cmath>
 
 #include "jl_common.cuh"
+#include "sm100_ptx.cuh"
 
 namespace jl {
 namespace {
 
-constexpr int kDecThreads = 128;
-constexpr int kKeyBlock = 64;
-constexpr int kMaxGrp = 16;
+constexpr int kDecWarps = 8;  // = KV heads per CTA
+constexpr int kDecThreads = kDecWarps * 32;
+constexpr int kStages = 3;
+constexpr int kMaxGrp = 8;
 constexpr float kLog2e = 1.4426950408889634f;
 
 template <int D>
-struct DecodeSmem {
-  static constexpr int KS = D + 4;  // padded fp32 row of K (bank-conflict free float4 reads)
-  static size_t bytes(int grp) {
-    return sizeof(float) * (2 * grp * D + kKeyBlock * KS + kKeyBlock * D + grp * kKeyBlock +
-                            3 * grp) +
-           sizeof(double) * (D / 2) + 16;
-  }
+struct DecCfg {
+  static constexpr int P = D == 128 ? 16 : 32;     // tokens per stage
+  static constexpr int EPL = D / 32;               // channels per lane
+  static constexpr int HEAD_BYTES = D * 2;         // one head's K (or V) row
+  static constexpr int STAGE_HALF = P * kDecWarps * HEAD_BYTES;  // K (or V) of a stage
+  static constexpr int STAGE = 2 * STAGE_HALF;
+  static constexpr int CS = kStages * STAGE;                     // cos/sin table [P][D/2]
+  static constexpr int BAR = CS + P * (D / 2) * 8;
+  static constexpr int BYTES = BAR + 8 * kStages + 16;
 };
 
+// Channel held by slot e of lane l: slots [0, EPL/2) are the first members of
+// the lane's channel pairs, slots [EPL/2, EPL) their partners (+ D/2).
 template <int D>
-__global__ void __launch_bounds__(kDecThreads)
+__device__ __forceinline__ int chan(int l, int e) {
+  if constexpr (D == 128) return (e & 1) + 2 * l + (e >> 1) * 64;  // 2l, 2l+1, 64+2l, 65+2l
+  else return l + e * 32;                                          // l, 32+l
+}
+
+// The lane's EPL channels of one BF16 head row in shared memory, as fp32.
+template <int D>
+__device__ __forceinline__ void load_row(const __nv_bfloat16 *row, int lane, float (&x)[D / 32]) {
+  if constexpr (D == 128) {
+    const __nv_bfloat162 lo = *reinterpret_cast<const __nv_bfloat162 *>(row + 2 * lane);
+    const __nv_bfloat162 hi = *reinterpret_cast<const __nv_bfloat162 *>(row + 64 + 2 * lane);
+    x[0] = __low2float(lo);
+    x[1] = __high2float(lo);
+    x[2] = __low2float(hi);
+    x[3] = __high2float(hi);
+  } else {
+    x[0] = bf2f(row[lane]);
+    x[1] = bf2f(row[lane + 32]);
+  }
+}
+
+__device__ __forceinline__ void bulk_copy(uint32_t dst, const void *src, uint32_t bytes,
+                                          uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+      "l"(src), "r"(bytes), "r"(bar)
+      : "memory");
+}
+
+// Sum 32 per-lane values across the warp so that lane l ends with the total of
+// value l (reduce-scatter by halving).  With `half_only` the values 16..31 are
+// absent: lanes l and l + 16 both end with the total of value l & 15.
+template <bool kHalfOnly>
+__device__ __forceinline__ float reduce_scatter(float (&v)[32], int lane) {
+  if constexpr (kHalfOnly) {
+#pragma unroll
+    for (int k = 0; k < 16; ++k) v[k] += __shfl_xor_sync(0xffffffffu, v[k], 16);
+  } else {
+    const bool up = lane & 16;
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      const float send = up ? v[k] : v[k + 16];
+      const float keep = up ? v[k + 16] : v[k];
+      v[k] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
+    }
+  }
+#pragma unroll
+  for (int o = 8; o >= 1; o >>= 1) {
+    const bool up = lane & o;
+#pragma unroll
+    for (int k = 0; k < o; ++k) {
+      const float send = up ? v[k] : v[k + o];
+      const float keep = up ? v[k + o] : v[k];
+      v[k] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+    }
+  }
+  return v[0];
+}
+
+template <int D, int GRP>
+__global__ void __launch_bounds__(kDecThreads, 1)
 decode_split_kernel(DecodeArgs a) {
-  constexpr int KS = DecodeSmem<D>::KS;
-  constexpr int HALF = D / 2;
-  const int s = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int grp = a.Hq / a.Hkv;
+  using C = DecCfg<D>;
+  constexpr int P = C::P, EPL = C::EPL, HALF = D / 2;
+  constexpr int NB = (32 / GRP) < P ? (32 / GRP) : P;  // tokens per score batch
+  constexpr int NV = NB * GRP;                         // values per batch: 16 or 32
+  static_assert(NV == 16 || NV == 32, "batch must fill 16 or 32 lanes");
+  static_assert(P % NB == 0, "batches tile a stage");
+
+  extern __shared__ __align__(128) uint8_t dsm[];
+  const uint32_t sb = smem_u32(dsm);
+  float2 *cs_tab = reinterpret_cast<float2 *>(dsm + C::CS);  // [P][D/2] (cos, sin)
+  volatile uint32_t *abort = reinterpret_cast<volatile uint32_t *>(dsm + C::BAR + 8 * kStages);
+
+  const int s = blockIdx.x, chunk_id = blockIdx.y, b = blockIdx.z;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int g0 = chunk_id * kDecWarps;
+  const int nh = min(kDecWarps, a.Hkv - g0);  // KV heads of this CTA
+  const int g = g0 + warp;
+  const bool wactive = warp < nh;
   const int p = a.L - 1;
   const int G = a.G;
-  const int fp = remap(p, G);
   const int w0eff = (G == 1) ? INT_MAX : a.w0;
   const int j_begin = s * a.chunk;
   const int j_end = min(a.L, j_begin + a.chunk);
+  const int n_stage = (j_end - j_begin + P - 1) / P;
+  const uint32_t row_bytes = static_cast<uint32_t>(nh) * C::HEAD_BYTES;  // one token, CTA heads
+  const size_t cache_row = static_cast<size_t>(a.Hkv) * D;               // elements per token
 
-  extern __shared__ __align__(16) unsigned char dsm[];
-  double *freq = reinterpret_cast<double *>(dsm);
-  float *q_true = reinterpret_cast<float *>(dsm + sizeof(double) * HALF);  // [grp][D]
-  float *q_rem = q_true + grp * D;                                         // [grp][D]
-  float *Ks = q_rem + grp * D;                                             // [kKeyBlock][KS]
-  float *Vs = Ks + kKeyBlock * KS;                                         // [kKeyBlock][D]
-  float *sc = Vs + kKeyBlock * D;                                          // [grp][kKeyBlock]
-  float *m_run = sc + grp * kKeyBlock;                                     // [grp]
-  float *l_run = m_run + grp;
-  float *alpha = l_run + grp;
+  if (tid == 0) {
+    for (int i = 0; i < kStages; ++i) mbar_init(sb + C::BAR + 8 * i, 1);
+    *abort = 0u;
+    fence_mbar_init();
+  }
+  __syncthreads();
 
+  auto issue = [&](int t) {
+    const int slot = t % kStages;
+    const int jt = j_begin + t * P;
+    const int n = min(P, j_end - jt);
+    const uint32_t bar = sb + C::BAR + 8 * slot;
+    const uint32_t kdst = sb + slot * C::STAGE, vdst = kdst + C::STAGE_HALF;
+    mbar_arrive_expect_tx(bar, 2u * n * row_bytes);
+    const __nv_bfloat16 *ks = a.k_cache + (static_cast<size_t>(b) * a.Lcap + jt) * cache_row + g0 * D;
+    const __nv_bfloat16 *vs = a.v_cache + (static_cast<size_t>(b) * a.Lcap + jt) * cache_row + g0 * D;
+    if (nh == a.Hkv) {  // the CTA's rows of consecutive tokens are contiguous
+      bulk_copy(kdst, ks, n * row_bytes, bar);
+      bulk_copy(vdst, vs, n * row_bytes, bar);
+    } else {
+      for (int t2 = 0; t2 < n; ++t2) {
+        bulk_copy(kdst + t2 * row_bytes, ks + t2 * cache_row, row_bytes, bar);
+        bulk_copy(vdst + t2 * row_bytes, vs + t2 * cache_row, row_bytes, bar);
+      }
+    }
+  };
+  if (tid == 0)
+    for (int t = 0; t < kStages && t < n_stage; ++t) issue(t);
+
+  // Queries of this warp's heads at the true position p and the remote
+  // position f(p), for the lane's channels, pre-scaled by log2(e)/sqrt(D).
   const double theta = static_cast<double>(a.theta);
-  for (int i = tid; i < HALF; i += kDecThreads) freq[i] = rope_freq(i, D, theta);
-  for (int h = tid; h < grp; h += kDecThreads) {
-    m_run[h] = -INFINITY;
-    l_run[h] = 0.f;
-  }
-  __syncthreads();
-
-  // Queries at the true position p and the remote position f(p), pre-scaled by
-  // log2(e)/sqrt(D) so the softmax runs in base 2.
   const float qscale = kLog2e / sqrtf(static_cast<float>(D));
-  for (int idx = tid; idx < grp * HALF; idx += kDecThreads) {
-    const int h = idx / HALF, i = idx - h * HALF;
-    const __nv_bfloat16 *qrow = a.q + (static_cast<size_t>(b) * a.Hq + g * grp + h) * D;
-    const float x = bf2f(qrow[i]), y = bf2f(qrow[i + HALF]);
-    float c, sn;
-    rope_cos_sin(p, freq[i], c, sn);
-    q_true[h * D + i] = (x * c - y * sn) * qscale;
-    q_true[h * D + i + HALF] = (x * sn + y * c) * qscale;
-    rope_cos_sin(fp, freq[i], c, sn);
-    q_rem[h * D + i] = (x * c - y * sn) * qscale;
-    q_rem[h * D + i + HALF] = (x * sn + y * c) * qscale;
-  }
-
-  constexpr int kMaxOut = kMaxGrp * D / kDecThreads;
-  float acc[kMaxOut];
+  float qt[GRP][EPL], qr[GRP][EPL];
+  double freq[EPL / 2];
 #pragma unroll
-  for (int r = 0; r < kMaxOut; ++r) acc[r] = 0.f;
-  const int n_out = grp * D;
-
-  const size_t row_stride = static_cast<size_t>(a.Hkv) * D;
-  const __nv_bfloat16 *kbase = a.k_cache + (static_cast<size_t>(b) * a.Lcap * a.Hkv + g) * D;
-  const __nv_bfloat16 *vbase = a.v_cache + (static_cast<size_t>(b) * a.Lcap * a.Hkv + g) * D;
-
-  for (int jb = j_begin; jb < j_end; jb += kKeyBlock) {
-    const int nk = min(kKeyBlock, j_end - jb);
-    __syncthreads();  // previous block fully consumed
-    // Stage K and V rows (8 BF16 per 16-byte load) as fp32.
-    for (int idx = tid; idx < kKeyBlock * (D / 8); idx += kDecThreads) {
-      const int t = idx / (D / 8), c8 = (idx - t * (D / 8)) * 8;
-      float kv[8], vv[8];
-      if (t < nk) {
-        const uint4 kr = *reinterpret_cast<const uint4 *>(kbase + (jb + t) * row_stride + c8);
-        const uint4 vr = *reinterpret_cast<const uint4 *>(vbase + (jb + t) * row_stride + c8);
-        const __nv_bfloat162 *k2 = reinterpret_cast<const __nv_bfloat162 *>(&kr);
-        const __nv_bfloat162 *v2 = reinterpret_cast<const __nv_bfloat162 *>(&vr);
+  for (int e = 0; e < EPL / 2; ++e) freq[e] = rope_freq(chan<D>(lane, e), D, theta);
+  {
+    float ct[EPL / 2], st[EPL / 2], cr[EPL / 2], sr[EPL / 2];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          kv[2 * e] = __low2float(k2[e]);
-          kv[2 * e + 1] = __high2float(k2[e]);
-          vv[2 * e] = __low2float(v2[e]);
-          vv[2 * e + 1] = __high2float(v2[e]);
-        }
-      } else {
+    for (int e = 0; e < EPL / 2; ++e) {
+      rope_cos_sin(p, freq[e], ct[e], st[e]);
+      rope_cos_sin(remap(p, G), freq[e], cr[e], sr[e]);
+    }
 #pragma unroll
-        for (int e = 0; e < 8; ++e) kv[e] = vv[e] = 0.f;
-      }
+    for (int h = 0; h < GRP; ++h) {
+      const int hq = (wactive ? g : g0) * GRP + h;
+      const __nv_bfloat16 *qrow = a.q + (static_cast<size_t>(b) * a.Hq + hq) * D;
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        Ks[t * KS + c8 + e] = kv[e];
-        Vs[t * D + c8 + e] = vv[e];
+      for (int e = 0; e < EPL / 2; ++e) {
+        const float x = bf2f(qrow[chan<D>(lane, e)]), y = bf2f(qrow[chan<D>(lane, e) + HALF]);
+        qt[h][e] = (x * ct[e] - y * st[e]) * qscale;
+        qt[h][e + EPL / 2] = (x * st[e] + y * ct[e]) * qscale;
+        qr[h][e] = (x * cr[e] - y * sr[e]) * qscale;
+        qr[h][e + EPL / 2] = (x * sr[e] + y * cr[e]) * qscale;
       }
     }
-    __syncthreads();
-    // Correction rotation of the remote keys (p - j > w0): R(Delta j), Delta j = f(j) - j.
-    if (p - jb > w0eff) {
-      for (int idx = tid; idx < nk * HALF; idx += kDecThreads) {
-        const int t = idx / HALF, i = idx - t * HALF;
-        const int j = jb + t;
+  }
+  // Channel e of the lane: e < EPL/2 are the first members of the pairs,
+  // e >= EPL/2 their partners (+D/2).
+
+  float acc[GRP][EPL];
+#pragma unroll
+  for (int h = 0; h < GRP; ++h)
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) acc[h][e] = 0.f;
+  float m_mine = -INFINITY, l_mine = 0.f;  // state of head (lane % GRP)
+
+  bool ok = true;
+  int t_fail = 0;
+  for (int t = 0; t < n_stage; ++t) {
+    const int slot = t % kStages;
+    const int jt = j_begin + t * P;
+    const int n = min(P, j_end - jt);
+    // cos/sin of the correction angles of this stage's remote tokens
+    if (p - jt > w0eff) {
+      for (int idx = tid; idx < n * HALF; idx += kDecThreads) {
+        const int tt = idx / HALF, i = idx - tt * HALF;
+        const int j = jt + tt;
+        float c = 1.f, sn = 0.f;
         if (p - j > w0eff) {
-          float c, sn;
-          rope_cos_sin(static_cast<long long>(remap(j, G)) - j, freq[i], c, sn);
-          const float x = Ks[t * KS + i], y = Ks[t * KS + i + HALF];
-          Ks[t * KS + i] = x * c - y * sn;
-          Ks[t * KS + i + HALF] = x * sn + y * c;
+          const double ang = static_cast<double>(remap(j, G) - j) *
+                             rope_freq(i, D, theta);  // Delta j * theta_i
+          const double r = ang - rint(ang * 0.15915494309189533577) * 6.283185307179586232;
+          __sincosf(static_cast<float>(r), &sn, &c);
+        }
+        cs_tab[tt * HALF + i] = make_float2(c, sn);
+      }
+    }
+    const uint32_t bar = sb + C::BAR + 8 * slot;
+    ok = mbar_wait_bounded(bar, static_cast<uint32_t>(t / kStages) & 1u, kWaitLimitNs);
+    if (__syncthreads_or(!ok)) {
+      ok = false;
+      t_fail = t;
+      break;
+    }
+    if (wactive) {
+      const uint8_t *kst = dsm + slot * C::STAGE + warp * C::HEAD_BYTES;
+      const uint8_t *vst = kst + C::STAGE_HALF;
+#pragma unroll 1
+      for (int tb = 0; tb < P; tb += NB) {
+        if (tb >= n) break;
+        // partial scores of NB tokens x GRP heads
+        float part[32];
+#pragma unroll
+        for (int k = 0; k < 32; ++k) part[k] = 0.f;
+#pragma unroll
+        for (int pb = 0; pb < NB; ++pb) {
+          const int tt = tb + pb;
+          if (tt < n) {
+            const int j = jt + tt;
+            const __nv_bfloat16 *krow =
+                reinterpret_cast<const __nv_bfloat16 *>(kst + tt * row_bytes);
+            float kv[EPL];
+            load_row<D>(krow, lane, kv);
+            const bool remote = p - j > w0eff;
+            if (remote) {
+#pragma unroll
+              for (int e = 0; e < EPL / 2; ++e) {
+                const float2 cs = cs_tab[tt * HALF + chan<D>(lane, e)];
+                const float x = kv[e], y = kv[e + EPL / 2];
+                kv[e] = x * cs.x - y * cs.y;
+                kv[e + EPL / 2] = x * cs.y + y * cs.x;
+              }
+            }
+#pragma unroll
+            for (int h = 0; h < GRP; ++h) {
+              float d = 0.f;
+#pragma unroll
+              for (int e = 0; e < EPL; ++e) d = fmaf(remote ? qr[h][e] : qt[h][e], kv[e], d);
+              part[pb * GRP + h] = d;
+            }
+          }
+        }
+        const float sc = reduce_scatter<NV == 16>(part, lane);
+        const int my_pb = (lane % NV) / GRP;
+        const bool valid = tb + my_pb < n;
+        const float sv = valid ? sc : -INFINITY;
+        // online softmax for head (lane % GRP) over the batch
+        float bm = sv;
+#pragma unroll
+        for (int o = GRP; o < NV; o <<= 1) bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, o));
+        const float m_new = fmaxf(m_mine, bm);  // finite: the batch holds a valid token
+        const float alpha_mine = exp2f(m_mine - m_new);
+        const float pm = exp2f(sv - m_new);
+        float ps = pm;
+#pragma unroll
+        for (int o = GRP; o < NV; o <<= 1) ps += __shfl_xor_sync(0xffffffffu, ps, o);
+        l_mine = l_mine * alpha_mine + ps;
+        m_mine = m_new;
+#pragma unroll
+        for (int h = 0; h < GRP; ++h) {
+          const float al = __shfl_sync(0xffffffffu, alpha_mine, h);
+#pragma unroll
+          for (int e = 0; e < EPL; ++e) acc[h][e] *= al;
+        }
+#pragma unroll
+        for (int pb = 0; pb < NB; ++pb) {
+          const int tt = tb + pb;
+          if (tt < n) {
+            const __nv_bfloat16 *vrow =
+                reinterpret_cast<const __nv_bfloat16 *>(vst + tt * row_bytes);
+            float vv[EPL];
+            load_row<D>(vrow, lane, vv);
+#pragma unroll
+            for (int h = 0; h < GRP; ++h) {
+              const float pr = __shfl_sync(0xffffffffu, pm, pb * GRP + h);
+#pragma unroll
+              for (int e = 0; e < EPL; ++e) acc[h][e] = fmaf(pr, vv[e], acc[h][e]);
+            }
+          }
         }
       }
-      __syncthreads();
     }
-    // Scores for (key t, head h).
-    for (int idx = tid; idx < kKeyBlock * grp; idx += kDecThreads) {
-      const int t = idx % kKeyBlock, h = idx / kKeyBlock;
-      const int j = jb + t;
-      float sres = -INFINITY;
-      if (t < nk) {
-        const float *qv = (p - j > w0eff) ? q_rem + h * D : q_true + h * D;
-        const float *kv = Ks + t * KS;
-        float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
-#pragma unroll 8
-        for (int d = 0; d < D; d += 4) {
-          const float4 k4 = *reinterpret_cast<const float4 *>(kv + d);
-          const float4 q4 = *reinterpret_cast<const float4 *>(qv + d);
-          acc0 = fmaf(k4.x, q4.x, acc0);
-          acc1 = fmaf(k4.y, q4.y, acc1);
-          acc2 = fmaf(k4.z, q4.z, acc2);
-          acc3 = fmaf(k4.w, q4.w, acc3);
-        }
-        sres = (acc0 + acc1) + (acc2 + acc3);
-      }
-      sc[h * kKeyBlock + t] = sres;
-    }
-    __syncthreads();
-    // Online softmax per head (one warp per head).
-    for (int h = warp; h < grp; h += kDecThreads / 32) {
-      float v0 = sc[h * kKeyBlock + lane], v1 = sc[h * kKeyBlock + lane + 32];
-      float mx = fmaxf(v0, v1);
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-      const float m_old = m_run[h];
-      const float m_new = fmaxf(m_old, mx);  // finite: every block holds a valid key
-      const float e0 = exp2f(v0 - m_new), e1 = exp2f(v1 - m_new);
-      sc[h * kKeyBlock + lane] = e0;
-      sc[h * kKeyBlock + lane + 32] = e1;
-      float sum = e0 + e1;
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-      __syncwarp();
-      if (lane == 0) {
-        const float al = exp2f(m_old - m_new);  // 0 when m_old = -inf
-        alpha[h] = al;
-        l_run[h] = l_run[h] * al + sum;
-        m_run[h] = m_new;
-      }
-    }
-    __syncthreads();
-    // O[h, d] = alpha[h] * O[h, d] + sum_t p[h, t] V[t, d]
-#pragma unroll
-    for (int r = 0; r < kMaxOut; ++r) {
-      const int o = tid + r * kDecThreads;
-      if (o < n_out) {
-        const int h = o / D, d = o - h * D;
-        const float *ph = sc + h * kKeyBlock;
-        float x = acc[r] * alpha[h];
-#pragma unroll 8
-        for (int t = 0; t < kKeyBlock; ++t) x = fmaf(ph[t], Vs[t * D + d], x);
-        acc[r] = x;
-      }
-    }
+    __syncthreads();  // stage slot and cos/sin table free again
+    if (tid == 0 && t + kStages < n_stage) issue(t + kStages);
   }
-  __syncthreads();
+  if (!ok) {
+    // Stages t_fail .. t_fail + kStages - 1 may still be in flight: let them
+    // land (bounded) before the CTA exits, then report.
+    if (tid == 0) {
+      for (int u = t_fail; u < n_stage && u < t_fail + kStages; ++u)
+        mbar_wait_bounded(sb + C::BAR + 8 * (u % kStages), static_cast<uint32_t>(u / kStages) & 1u,
+                          kWaitLimitNs);
+      atomicOr(a.dev_error, kDevTimeout);
+    }
+    return;
+  }
+  if (!wactive) return;
   // Partial record: [D] unnormalised output, then the running max (base 2) and sum.
 #pragma unroll
-  for (int r = 0; r < kMaxOut; ++r) {
-    const int o = tid + r * kDecThreads;
-    if (o < n_out) {
-      const int h = o / D, d = o - h * D;
-      float *rec = a.partial + ((static_cast<size_t>(b) * a.Hq + g * grp + h) * a.n_split + s) * (D + 2);
-      rec[d] = acc[r];
-      if (d == 0) {
-        rec[D] = m_run[h];
-        rec[D + 1] = l_run[h];
-      }
-    }
+  for (int h = 0; h < GRP; ++h) {
+    float *rec = a.partial +
+                 ((static_cast<size_t>(b) * a.Hq + g * GRP + h) * a.n_split + s) * (D + 2);
+#pragma unroll
+    for (int e = 0; e < EPL; ++e) rec[chan<D>(lane, e)] = acc[h][e];
+  }
+  if (lane < GRP) {
+    float *rec = a.partial +
+                 ((static_cast<size_t>(b) * a.Hq + g * GRP + lane) * a.n_split + s) * (D + 2);
+    rec[D] = m_mine;
+    rec[D + 1] = l_mine;
   }
 }
 
@@ -258,16 +388,27 @@ decode_combine_kernel(DecodeArgs a) {
   if (lane == 0 && a.lse) a.lse[bh] = (M + log2f(lsum)) * 0.69314718055994531f;
 }
 
+template <int D, int GRP>
+cudaError_t launch_split(const DecodeArgs &a, cudaStream_t stream) {
+  const int smem = DecCfg<D>::BYTES;
+  cudaError_t e = cudaFuncSetAttribute(decode_split_kernel<D, GRP>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  const int n_chunk = (a.Hkv + kDecWarps - 1) / kDecWarps;
+  decode_split_kernel<D, GRP><<<dim3(a.n_split, n_chunk, a.B), kDecThreads, smem, stream>>>(a);
+  return cudaGetLastError();
+}
+
 template <int D>
 cudaError_t launch_decode_d(const DecodeArgs &a, cudaStream_t stream) {
-  const int grp = a.Hq / a.Hkv;
-  const size_t smem = DecodeSmem<D>::bytes(grp);
-  cudaError_t e = cudaFuncSetAttribute(decode_split_kernel<D>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
-  if (e != cudaSuccess) return e;
-  decode_split_kernel<D><<<dim3(a.n_split, a.Hkv, a.B), kDecThreads, smem, stream>>>(a);
-  e = cudaGetLastError();
+  cudaError_t e;
+  switch (a.Hq / a.Hkv) {
+    case 1: e = launch_split<D, 1>(a, stream); break;
+    case 2: e = launch_split<D, 2>(a, stream); break;
+    case 4: e = launch_split<D, 4>(a, stream); break;
+    case 8: e = launch_split<D, 8>(a, stream); break;
+    default: return cudaErrorInvalidValue;
+  }
   if (e != cudaSuccess) return e;
   const int nbh = a.B * a.Hq;
   decode_combine_kernel<D><<<(nbh + 3) / 4, 128, 0, stream>>>(a);
@@ -277,22 +418,22 @@ cudaError_t launch_decode_d(const DecodeArgs &a, cudaStream_t stream) {
 }  // namespace
 
 void decode_plan(int B, int Hkv, int L, int *n_split, int *chunk) {
-  // Aim for about four resident CTAs per SM over the 148 SMs of a B200; the
-  // split count is non-decreasing in L, so workspace sized for the largest L
-  // of a generation loop covers every step.
-  const int target = 4 * 148;
-  const int units = B * Hkv;
-  int ns = (target + units - 1) / units;
-  const int max_ns = (L + kKeyBlock - 1) / kKeyBlock;
+  // One CTA per SM (each holds a 3-stage ring) over the 148 SMs of a B200;
+  // chunks are whole stages of 16 tokens.  The split count is non-decreasing
+  // in L, so workspace sized for the largest L of a generation loop covers
+  // every step.
+  const int units = B * ((Hkv + kDecWarps - 1) / kDecWarps);
+  int ns = (148 + units - 1) / units;
+  const int max_ns = (L + 15) / 16;
   if (ns > max_ns) ns = max_ns;
   if (ns < 1) ns = 1;
   int ch = (L + ns - 1) / ns;
-  ch = (ch + kKeyBlock - 1) / kKeyBlock * kKeyBlock;
+  ch = (ch + 31) / 32 * 32;  // a whole number of stages for both head dims
   *chunk = ch;
   *n_split = (L + ch - 1) / ch;
 }
 
-int decode_max_group() { return kMaxGrp; }
+bool decode_supports_group(int grp) { return grp == 1 || grp == 2 || grp == 4 || grp == 8; }
 
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t stream) {
   if (a.D == 128) return launch_decode_d<128>(a, stream);

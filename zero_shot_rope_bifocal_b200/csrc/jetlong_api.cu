@@ -248,7 +248,7 @@ int jetlong_decode(const void *q, const void *k_cache, const void *v_cache, void
   int st = check_common(B, Hq, Hkv, L, D);
   if (st != JL_OK) return st;
   if (Lcap < L) return JL_ERR_SHAPE;
-  if (Hq / Hkv > decode_max_group()) return JL_ERR_UNSUPPORTED;
+  if (!decode_supports_group(Hq / Hkv)) return JL_ERR_UNSUPPORTED;
   if ((st = check_method(w_pretrained, w0, rope_theta)) != JL_OK) return st;
   if (out_dtype != JL_BF16 && out_dtype != JL_F32) return JL_ERR_UNSUPPORTED;
   if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out) ||

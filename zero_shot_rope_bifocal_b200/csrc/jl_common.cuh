@@ -93,8 +93,8 @@ struct DecodeArgs {
 // Split-KV plan: number of key chunks and chunk length for a cache of L tokens.
 void decode_plan(int B, int Hkv, int L, int *n_split, int *chunk);
 
-// Largest Hq / Hkv the decode kernel supports.
-int decode_max_group();
+// Query heads per KV head (Hq / Hkv) the decode kernel is built for: 1, 2, 4, 8.
+bool decode_supports_group(int grp);
 
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t stream);
 

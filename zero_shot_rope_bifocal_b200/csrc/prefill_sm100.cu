@@ -24,21 +24,24 @@
 // FP16, head-major [B, H, L, D].  FP16 keeps three more mantissa bits than
 // BF16 for the rotated values the tensor core must consume in 16 bits.
 //
-// Hardware mapping (one CTA = one 128-row query tile of one head; 4 warps):
-//   * TMA (128-byte swizzle) loads the query tile once per variant and K / V
-//     tiles into a two-slot ring; mbarriers with expect-tx track arrival;
-//   * thread 0 issues tcgen05.mma: S = Q K^T (M=128, N=128, K=D) into TMEM,
-//     later O += P V with P read from TMEM (M=128, N=D, K=128);
-//   * every thread owns one query row = one TMEM lane: it loads its S row,
-//     applies the mask, runs the online softmax in base 2 (fp32 statistics),
-//     rescales its O row only when the running max grew by more than 2^8
-//     (decided per warp, since TMEM loads and stores are warp-collective),
-//     and stores P (FP16) to TMEM;
-//   * the epilogue divides O by the row sum and writes O and the natural-log
-//     LSE.
-// Each wait is bounded in time (jl::kWaitLimitNs); on expiry the CTA records a
-// device error, drains its own MMAs, frees TMEM and exits, and CTAs that start
-// after a recorded error skip their work.
+// CTA = two 128-row query tiles of the same 128 positions, for two query
+// heads of one KV group (GQA packing: each K/V tile staged in shared memory
+// serves 256 query rows).  Warp-specialised, 12 warps:
+//   * warps 0-3 / 4-7: softmax for query tile 0 / 1 (one thread per row =
+//     one TMEM lane); they also rescale their O rows when needed and run the
+//     epilogue;
+//   * warp 8: TMA producer (queries once per variant, K and V tiles through a
+//     four-slot ring);
+//   * warp 9: tcgen05.mma issuer, in the order
+//       S0(j+1) = Q0 K(j+1)^T after O0 += P0(j) V(j), and likewise for tile 1,
+//     so the tensor core works on one tile while the other tile's softmax
+//     runs;
+//   * warps 10-11 hold no role.
+// TMEM (512 columns): S0 | S1 | O0 | O1; P of each tile overwrites the first
+// 64 columns of its S as packed FP16 once the S row is in registers.
+// Each wait is bounded in time (jl::kWaitLimitNs) and also gives up when
+// another role has given up; the CTA then records a device error, drains its
+// MMAs and in-flight copies, frees TMEM and exits.
 #include <cmath>
 
 #include "jl_common.cuh"
@@ -49,28 +52,38 @@ namespace {
 
 constexpr int BM = 128;  // query rows per tile (= TMEM lanes)
 constexpr int BN = 128;  // keys per tile
-constexpr int kThreads = 128;
+constexpr int NS = 4;    // K/V ring slots (one K or V tile each)
+constexpr int kWarps = 12;
+constexpr int kThreads = kWarps * 32;
+constexpr int kProducerWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr int kSoftmaxRegs = 200;
+constexpr int kOtherRegs = 96;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 constexpr uint32_t kF16 = 0;               // operand format code of kind::f16
 
 template <int D>
 struct Layout {
-  static constexpr int TILE = BM * D * 2;       // bytes of one 128 x D 16-bit tile
-  static constexpr int BOX = 128 * 128;         // bytes of one 128-row x 64-col swizzled box
-  static constexpr int Q = 0;
-  static constexpr int K0 = TILE;
-  static constexpr int V0 = 3 * TILE;
-  static constexpr int BAR = 5 * TILE;
-  static constexpr int BYTES = BAR + 64;
-  static constexpr int ALLOC = BYTES + 1024;    // slack to align the base to 1024
-  // TMEM columns: S (128) + O (D) + P (64), rounded up to a power of two.
-  // D = 128 uses all 512 columns and its shared memory keeps one CTA per SM;
-  // D = 64 fits two CTAs per SM in both.
-  static constexpr uint32_t TMEM_COLS = D == 128 ? 512u : 256u;
+  static constexpr int TILE = BM * D * 2;  // bytes of one 128 x D FP16 tile
+  static constexpr int BOX = 128 * 128;    // bytes of one 128-row x 64-col swizzled box
+  static constexpr int Q0 = 0;
+  static constexpr int RING = 2 * TILE;
+  static constexpr int BAR = RING + NS * TILE;
+  // barrier indices (8 bytes each)
+  static constexpr int kQFull = 0, kQEmpty = 2, kKvFull = 4, kKvEmpty = 4 + NS,
+                       kSFull = 4 + 2 * NS, kPFull = 6 + 2 * NS, kOFull = 8 + 2 * NS,
+                       kDrain = 10 + 2 * NS, kNumBars = 11 + 2 * NS;
+  static constexpr int TMEM_SLOT = BAR + 8 * kNumBars;
+  static constexpr int ABORT = TMEM_SLOT + 4;
+  static constexpr int SKIP = TMEM_SLOT + 8;
+  static constexpr int BYTES = TMEM_SLOT + 16;
+  // 1024 B of slack to align the base; D = 64 asks for enough shared memory
+  // to keep one CTA per SM, since each CTA holds all 512 TMEM columns.
+  static constexpr int ALLOC = (BYTES + 1024 > 120 * 1024) ? BYTES + 1024 : 120 * 1024;
 };
 
 struct Params {
-  int B, Hq, Hkv, L, G, w0eff, n_qt;
+  int B, Hq, Hkv, L, G, w0eff, n_qt, grp, npair;
   float scale_log2;
   void *out;
   float *lse;
@@ -79,6 +92,30 @@ struct Params {
 };
 
 __device__ __forceinline__ float u2f(uint32_t u) { return __uint_as_float(u); }
+
+__device__ __forceinline__ void set_regs_softmax() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftmaxRegs));
+}
+__device__ __forceinline__ void set_regs_other() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kOtherRegs));
+}
+
+// Bounded wait that also gives up once another role has raised `abort`.
+__device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t parity,
+                                              volatile uint32_t *abort) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 63u) == 0u) {
+      if (*abort) return false;
+      if (global_timer_ns() - t0 > kWaitLimitNs) {
+        *abort = 1u;
+        return false;
+      }
+    }
+  }
+}
 
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -92,24 +129,19 @@ bifocal_prefill_kernel(const __grid_constant__ CUtensorMap tm_qt,
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const uint32_t sb = smem_u32(smem);
-  const uint32_t sQ = sb + LY::Q;
-  const uint32_t sK[2] = {sb + LY::K0, sb + LY::K0 + LY::TILE};
-  const uint32_t sV[2] = {sb + LY::V0, sb + LY::V0 + LY::TILE};
-  const uint32_t bar_q = sb + LY::BAR;
-  const uint32_t bar_kv[2] = {sb + LY::BAR + 8, sb + LY::BAR + 16};
-  const uint32_t bar_s = sb + LY::BAR + 24;
-  const uint32_t bar_o = sb + LY::BAR + 32;
-  const uint32_t tmem_slot = sb + LY::BAR + 40;
-  volatile uint32_t *skip_flag = reinterpret_cast<volatile uint32_t *>(smem + LY::BAR + 44);
+  auto bar = [&](int i) { return sb + LY::BAR + 8u * static_cast<uint32_t>(i); };
+  volatile uint32_t *abort = reinterpret_cast<volatile uint32_t *>(smem + LY::ABORT);
+  volatile uint32_t *skip = reinterpret_cast<volatile uint32_t *>(smem + LY::SKIP);
 
-  const int tid = threadIdx.x, warp = tid >> 5;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int qt = prm.n_qt - 1 - static_cast<int>(blockIdx.x);  // longest rows first
-  const int h = blockIdx.y, b = blockIdx.z;
-  const int hk = h / (prm.Hq / prm.Hkv);
+  const int g = static_cast<int>(blockIdx.y) / prm.npair;
+  const int pr = static_cast<int>(blockIdx.y) - g * prm.npair;
+  const int b = blockIdx.z;
+  const int head0 = g * prm.grp + 2 * pr;
+  const bool has1 = 2 * pr + 1 < prm.grp;
   const int p0 = qt * BM;
   const int p1 = min(p0 + BM, prm.L) - 1;
-  const int row = p0 + tid;
-  const bool row_ok = row < prm.L;
   const int w0 = prm.w0eff;
 
   // Visit plan: remote visits of key tiles [0, n_rem), then local visits of
@@ -122,21 +154,25 @@ bifocal_prefill_kernel(const __grid_constant__ CUtensorMap tm_qt,
     kl0 = max(0, p0 - w0) / BN;
   }
   const int nv = n_rem + (n_kt - kl0);
+  const bool switch_q = n_rem > 0 && n_rem < nv;
 
-  // Once any CTA has recorded a failure, the others skip their work, so a
-  // broken launch ends after one wait limit instead of one per CTA wave.
-  // Thread 0 reads the word and the whole CTA follows its answer.
-  if (tid == 0) *skip_flag = *reinterpret_cast<volatile unsigned int *>(prm.dev_error);
+  // A launch that already recorded a failure ends quickly: thread 0 reads the
+  // error word and the whole CTA follows its answer.
+  if (tid == 0) {
+    *skip = *reinterpret_cast<volatile unsigned int *>(prm.dev_error);
+    *abort = 0u;
+  }
   __syncthreads();
-  if (*skip_flag != kDevOk) return;
+  if (*skip != kDevOk) return;
 
   if (tid == 0) {
-    mbar_init(bar_q, 1);
-    mbar_init(bar_kv[0], 1);
-    mbar_init(bar_kv[1], 1);
-    mbar_init(bar_s, 1);
-    mbar_init(bar_o, 1);
+    // P-ready barriers take one arrival from every softmax thread of the
+    // tile; all others one arrival (plus transaction bytes for TMA).
+    for (int i = 0; i < LY::kNumBars; ++i)
+      mbar_init(bar(i), (i == LY::kPFull || i == LY::kPFull + 1) ? BM : 1);
     fence_mbar_init();
+  }
+  if (warp == kProducerWarp && lane == 0) {
     prefetch_tmap(&tm_qt);
     prefetch_tmap(&tm_qr);
     prefetch_tmap(&tm_kt);
@@ -144,215 +180,304 @@ bifocal_prefill_kernel(const __grid_constant__ CUtensorMap tm_qt,
     prefetch_tmap(&tm_v);
   }
   __syncthreads();
-  if (warp == 0) {
-    tmem_alloc(tmem_slot, LY::TMEM_COLS);
+  if (warp == kMmaWarp) {
+    tmem_alloc(sb + LY::TMEM_SLOT, 512);
     tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(smem + LY::BAR + 40);
-  const uint32_t tS = tmem;            // S: 128 columns fp32
-  const uint32_t tO = tmem + 128;      // O: D columns fp32
-  const uint32_t tP = tmem + 128 + D;  // P: 64 columns of packed FP16 pairs
-  const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(smem + LY::TMEM_SLOT);
+  // TMEM columns: S0 [0,128) S1 [128,256) O0 [256,256+D) O1 [256+D,256+2D)
+  auto tS = [&](int s) { return tmem + 128u * static_cast<uint32_t>(s); };
+  auto tO = [&](int s) { return tmem + 256u + static_cast<uint32_t>(D * s); };
 
   constexpr uint32_t IDESC_QK = idesc_f16kind_f32(BM, BN, kF16, false, false);
   constexpr uint32_t IDESC_PV = idesc_f16kind_f32(BM, D, kF16, false, true);
   constexpr int NBOX = D / 64;
 
-  auto load_q = [&](bool remote) {
-    mbar_arrive_expect_tx(bar_q, LY::TILE);
-    for (int c = 0; c < NBOX; ++c)
-      tma_load_3d(sQ + c * LY::BOX, remote ? &tm_qr : &tm_qt, bar_q, c * 64, p0, b * prm.Hq + h);
-  };
-  auto load_kv = [&](int vt, int slot) {
-    const bool remote = vt < n_rem;
-    const int kt = remote ? vt : kl0 + (vt - n_rem);
-    mbar_arrive_expect_tx(bar_kv[slot], 2 * LY::TILE);
-    for (int c = 0; c < NBOX; ++c) {
-      tma_load_3d(sK[slot] + c * LY::BOX, remote ? &tm_kr : &tm_kt, bar_kv[slot], c * 64, kt * BN,
-                  b * prm.Hkv + hk);
-      tma_load_3d(sV[slot] + c * LY::BOX, &tm_v, bar_kv[slot], c * 64, kt * BN, b * prm.Hkv + hk);
-    }
-  };
-
-  if (tid == 0) {
-    load_q(n_rem > 0);
-    load_kv(0, 0);
-  }
-
-  float m_used = -INFINITY;  // reference max of this row (base 2)
-  float l_sum = 0.f;
-  bool ok = true;
-
-  for (int vt = 0; vt < nv; ++vt) {
-    const bool remote = vt < n_rem;
-    const int kt = remote ? vt : kl0 + (vt - n_rem);
-    const int slot = vt & 1;
-    if (tid == 0 && ok) {
-      if (vt == 0 || vt == n_rem) ok = mbar_wait_bounded(bar_q, vt == 0 ? 0u : 1u, kWaitLimitNs);
-      if (ok)
-        ok = mbar_wait_bounded(bar_kv[slot], static_cast<uint32_t>(vt >> 1) & 1u, kWaitLimitNs);
-      if (ok) {
-        tc_fence_after();
+  if (warp >= 8) {
+    set_regs_other();
+    if (warp == kProducerWarp && lane == 0) {
+      // ---------------------------------------------------------- producer
+      auto load_q = [&](int s, bool remote) {
+        mbar_arrive_expect_tx(bar(LY::kQFull + s), LY::TILE);
+        for (int c = 0; c < NBOX; ++c)
+          tma_load_3d(sb + LY::Q0 + s * LY::TILE + c * LY::BOX, remote ? &tm_qr : &tm_qt,
+                      bar(LY::kQFull + s), c * 64, p0, b * prm.Hq + head0 + s);
+      };
+      load_q(0, n_rem > 0);
+      if (has1) load_q(1, n_rem > 0);
+      int r = 0;
+      bool ok = true;
+      uint32_t issued[NS] = {0, 0, 0, 0};  // uses issued per slot
+      for (int j = 0; j < nv && ok; ++j) {
+        const bool remote = j < n_rem;
+        const int kt = remote ? j : kl0 + (j - n_rem);
+        for (int part = 0; part < 2 && ok; ++part, ++r) {
+          const int slot = r % NS;
+          const uint32_t use = static_cast<uint32_t>(r / NS);
+          ok = wait_or_abort(bar(LY::kKvEmpty + slot), (use & 1u) ^ 1u, abort);
+          if (!ok) break;
+          const uint32_t dst = sb + LY::RING + slot * LY::TILE;
+          mbar_arrive_expect_tx(bar(LY::kKvFull + slot), LY::TILE);
+          const CUtensorMap *tm = part == 0 ? (remote ? &tm_kr : &tm_kt) : &tm_v;
+          for (int c = 0; c < NBOX; ++c)
+            tma_load_3d(dst + c * LY::BOX, tm, bar(LY::kKvFull + slot), c * 64, kt * BN,
+                        b * prm.Hkv + g);
+          issued[slot] = use + 1;
+        }
+        if (ok && switch_q && j == n_rem - 1) {
+          ok = wait_or_abort(bar(LY::kQEmpty + 0), 0u, abort);
+          if (ok) load_q(0, false);
+          if (ok && has1) {
+            ok = wait_or_abort(bar(LY::kQEmpty + 1), 0u, abort);
+            if (ok) load_q(1, false);
+          }
+        }
+      }
+      if (!ok) {
+        // Let copies already in flight land before the CTA exits (bounded).
+        for (int s = 0; s < NS; ++s)
+          if (issued[s] > 0) mbar_wait_bounded(bar(LY::kKvFull + s), (issued[s] - 1u) & 1u, kWaitLimitNs);
+      }
+    } else if (warp == kMmaWarp && lane == 0) {
+      // ---------------------------------------------------------- MMA issuer
+      auto qk = [&](int s, uint32_t kslot) {
+        const uint32_t qa = sb + LY::Q0 + s * LY::TILE;
+        const uint32_t kb = sb + LY::RING + kslot * LY::TILE;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * LY::BOX + (kk & 3) * 32;
-          mma_f16kind_ss(tS, smem_desc_sw128(sQ + off, 16, 1024),
-                         smem_desc_sw128(sK[slot] + off, 16, 1024), IDESC_QK, kk > 0 ? 1u : 0u);
+          mma_f16kind_ss(tS(s), smem_desc_sw128(qa + off, 16, 1024), smem_desc_sw128(kb + off, 16, 1024),
+                         IDESC_QK, kk > 0 ? 1u : 0u);
         }
-        mma_commit(bar_s);
+        mma_commit(bar(LY::kSFull + s));
+      };
+      auto pv = [&](int s, uint32_t vslot, bool acc) {
+        const uint32_t vb = sb + LY::RING + vslot * LY::TILE;
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk)
+          mma_f16kind_ts(tO(s), tS(s) + kk * 8, smem_desc_sw128(vb + kk * 16 * 128, LY::BOX, 1024),
+                         IDESC_PV, (acc || kk > 0) ? 1u : 0u);
+      };
+      bool ok = wait_or_abort(bar(LY::kQFull + 0), 0u, abort);
+      if (ok && has1) ok = wait_or_abort(bar(LY::kQFull + 1), 0u, abort);
+      int r = 0;
+      // visit 0: S0, S1
+      int kslot = 0;
+      if (ok) {
+        kslot = r % NS;
+        ok = wait_or_abort(bar(LY::kKvFull + kslot), static_cast<uint32_t>(r / NS) & 1u, abort);
+        ++r;
       }
-    }
-    if (ok) ok = mbar_wait_bounded(bar_s, static_cast<uint32_t>(vt) & 1u, kWaitLimitNs);
-    if (__syncthreads_or(!ok)) {
-      ok = false;
-      break;
-    }
-    tc_fence_after();
-    // S(vt) is complete, and with it every earlier MMA: the Q buffer (if this
-    // was the last remote visit) and the other K/V slot are free.
-    if (tid == 0 && vt + 1 < nv) {
-      if (vt + 1 == n_rem) load_q(false);
-      load_kv(vt + 1, slot ^ 1);
-    }
-
-    // ---- softmax on this thread's row (TMEM accesses are warp-collective:
-    // every branch around them below is warp-uniform)
-    float x[BN];
-    {
-      uint32_t r[BN / 32][32];
-#pragma unroll
-      for (int c = 0; c < BN / 32; ++c) tmem_ld32(tS + lane_base + c * 32, r[c]);
-      tmem_wait_ld();
-#pragma unroll
-      for (int c = 0; c < BN / 32; ++c) {
-        reg_fence(r[c]);
-#pragma unroll
-        for (int e = 0; e < 32; ++e) x[c * 32 + e] = u2f(r[c][e]) * prm.scale_log2;
+      if (ok) {
+        tc_fence_after();
+        qk(0, kslot);
+        if (switch_q && n_rem == 1) mma_commit(bar(LY::kQEmpty + 0));
+        if (has1) {
+          qk(1, kslot);
+          if (switch_q && n_rem == 1) mma_commit(bar(LY::kQEmpty + 1));
+        }
+        mma_commit(bar(LY::kKvEmpty + kslot));
       }
-    }
-    const int k0 = kt * BN;
-    bool whole;
-    if (remote)
-      whole = row_ok && (row - (k0 + BN - 1) > w0);
-    else
-      whole = row_ok && (k0 + BN - 1 <= row) && (row - k0 <= w0);
-    if (!whole) {
-#pragma unroll
-      for (int c = 0; c < BN; ++c) {
-        const int d = row - (k0 + c);
-        const bool valid = row_ok && d >= 0 && (remote ? (d > w0) : (d <= w0));
-        if (!valid) x[c] = -INFINITY;
+      for (int j = 0; j < nv && ok; ++j) {
+        const int vslot = r % NS;
+        ok = wait_or_abort(bar(LY::kKvFull + vslot), static_cast<uint32_t>(r / NS) & 1u, abort);
+        ++r;
+        if (!ok) break;
+        // tile 0: O0 += P0(j) V(j), then S0(j+1)
+        ok = wait_or_abort(bar(LY::kPFull + 0), static_cast<uint32_t>(j) & 1u, abort);
+        if (!ok) break;
+        tc_fence_after();
+        pv(0, vslot, j > 0);
+        const bool more = j + 1 < nv;
+        if (more) {
+          kslot = r % NS;
+          ok = wait_or_abort(bar(LY::kKvFull + kslot), static_cast<uint32_t>(r / NS) & 1u, abort);
+          ++r;
+          if (ok && switch_q && j + 1 == n_rem) ok = wait_or_abort(bar(LY::kQFull + 0), 1u, abort);
+          if (!ok) break;
+          tc_fence_after();
+          qk(0, kslot);
+          if (switch_q && j + 2 == n_rem) mma_commit(bar(LY::kQEmpty + 0));
+        }
+        // tile 1: O1 += P1(j) V(j), then S1(j+1)
+        if (has1) {
+          ok = wait_or_abort(bar(LY::kPFull + 1), static_cast<uint32_t>(j) & 1u, abort);
+          if (!ok) break;
+          tc_fence_after();
+          pv(1, vslot, j > 0);
+        }
+        mma_commit(bar(LY::kKvEmpty + vslot));
+        if (more) {
+          if (has1) {
+            if (switch_q && j + 1 == n_rem) ok = wait_or_abort(bar(LY::kQFull + 1), 1u, abort);
+            if (!ok) break;
+            tc_fence_after();
+            qk(1, kslot);
+            if (switch_q && j + 2 == n_rem) mma_commit(bar(LY::kQEmpty + 1));
+          }
+          mma_commit(bar(LY::kKvEmpty + kslot));
+        }
       }
+      if (ok) {
+        mma_commit(bar(LY::kOFull + 0));
+        if (has1) mma_commit(bar(LY::kOFull + 1));
+      }
+      // Every MMA issued here completes before TMEM is read out or freed.
+      mma_commit(bar(LY::kDrain));
+      const uint64_t t0 = global_timer_ns();
+      while (!mbar_try_wait(bar(LY::kDrain), 0u))
+        if (global_timer_ns() - t0 > kWaitLimitNs) {
+          *abort = 1u;
+          break;
+        }
     }
-    float tmax = -INFINITY;
+  } else {
+    // ------------------------------------------------------------ softmax
+    set_regs_softmax();
+    const int s = warp >> 2;             // query tile of this warpgroup
+    const int wq = warp & 3;             // TMEM lane quarter
+    const int rloc = tid & (BM - 1);     // row inside the tile
+    const int row = p0 + rloc;
+    const bool active = s == 0 || has1;
+    const bool row_ok = active && row < prm.L;
+    const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
+    float m_used = -INFINITY;  // reference max of this row (base 2)
+    float l_sum = 0.f;
+    bool ok = active;
+    for (int j = 0; j < nv && ok; ++j) {
+      const bool remote = j < n_rem;
+      const int kt = remote ? j : kl0 + (j - n_rem);
+      ok = wait_or_abort(bar(LY::kSFull + s), static_cast<uint32_t>(j) & 1u, abort);
+      if (__any_sync(0xffffffffu, !ok)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      float x[BN];
+      {
+        uint32_t(&xr)[BN] = reinterpret_cast<uint32_t(&)[BN]>(x);
 #pragma unroll
-    for (int c = 0; c < BN; ++c) tmax = fmaxf(tmax, x[c]);
-    const bool grow = tmax > m_used + kRescaleThreshold || (m_used == -INFINITY && tmax > -INFINITY);
-    float alpha = 1.f;  // factor applied to this row's O and l
-    if (grow) {
-      if (m_used != -INFINITY) alpha = exp2f(m_used - tmax);
-      m_used = tmax;
-    }
-    l_sum *= alpha;
-    // O holds data from visit 1 on (visit 0 overwrites it); rows whose max was
-    // -inf have O = 0 there, so alpha = 1 keeps them exact.
-    if (vt > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
-      __syncwarp();
-#pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t r[32];
-        tmem_ld32(tO + lane_base + c * 32, r);
+        for (int c = 0; c < BN / 32; ++c)
+          tmem_ld32(tS(s) + lane_base + c * 32, reinterpret_cast<uint32_t(&)[32]>(xr[c * 32]));
         tmem_wait_ld();
-        reg_fence(r);
 #pragma unroll
-        for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(u2f(r[e]) * alpha);
-        tmem_st32(tO + lane_base + c * 32, r);
+        for (int c = 0; c < BN / 32; ++c) reg_fence(reinterpret_cast<uint32_t(&)[32]>(xr[c * 32]));
       }
-    }
-    float lsum = 0.f;
-    if (m_used == -INFINITY) {
+      const int k0 = kt * BN;
+      bool whole;
+      if (remote)
+        whole = row_ok && (row - (k0 + BN - 1) > w0);
+      else
+        whole = row_ok && (k0 + BN - 1 <= row) && (row - k0 <= w0);
+      if (!whole) {
 #pragma unroll
-      for (int c = 0; c < BN; ++c) x[c] = 0.f;
-    } else {
+        for (int c = 0; c < BN; ++c) {
+          const int d = row - (k0 + c);
+          const bool valid = row_ok && d >= 0 && (remote ? (d > w0) : (d <= w0));
+          if (!valid) x[c] = -INFINITY;
+        }
+      }
+      float tmax = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < BN; ++c) tmax = fmaxf(tmax, x[c]);
+      tmax *= prm.scale_log2;  // raw scores; the scale is positive
+      const bool grow =
+          tmax > m_used + kRescaleThreshold || (m_used == -INFINITY && tmax > -INFINITY);
+      float alpha = 1.f;
+      if (grow) {
+        if (m_used != -INFINITY) alpha = exp2f(m_used - tmax);
+        m_used = tmax;
+      }
+      l_sum *= alpha;
+      // O of this tile holds visits 0..j-1 (all complete: S(j) was issued
+      // after P(j-1) V(j-1)); rows whose max was -inf hold 0 there.
+      if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+        __syncwarp();
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t rr[32];
+          tmem_ld32(tO(s) + lane_base + c * 32, rr);
+          tmem_wait_ld();
+          reg_fence(rr);
+#pragma unroll
+          for (int e = 0; e < 32; ++e) rr[e] = __float_as_uint(u2f(rr[e]) * alpha);
+          tmem_st32(tO(s) + lane_base + c * 32, rr);
+        }
+      }
+      float lsum = 0.f;
+      const float neg_m = m_used == -INFINITY ? 0.f : -m_used;
 #pragma unroll
       for (int c = 0; c < BN; ++c) {
-        x[c] = exp2f(x[c] - m_used);
+        // masked entries are -inf and give 0; a row with nothing valid yet
+        // has all entries -inf
+        x[c] = exp2f(fmaf(x[c], prm.scale_log2, neg_m));
         lsum += x[c];
       }
-    }
-    l_sum += lsum;
-    __syncwarp();
+      l_sum += lsum;
+      __syncwarp();
 #pragma unroll
-    for (int c = 0; c < BN / 64; ++c) {
-      uint32_t r[32];
+      for (int c = 0; c < BN / 64; ++c) {
+        uint32_t rr[32];
 #pragma unroll
-      for (int e = 0; e < 32; ++e) {
-        const __half2 pr = __floats2half2_rn(x[c * 64 + 2 * e], x[c * 64 + 2 * e + 1]);
-        r[e] = *reinterpret_cast<const uint32_t *>(&pr);
+        for (int e = 0; e < 32; ++e) {
+          const __half2 h2 = __floats2half2_rn(x[c * 64 + 2 * e], x[c * 64 + 2 * e + 1]);
+          rr[e] = *reinterpret_cast<const uint32_t *>(&h2);
+        }
+        tmem_st32(tS(s) + lane_base + c * 32, rr);
       }
-      tmem_st32(tP + lane_base + c * 32, r);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar(LY::kPFull + s));
     }
-    tmem_wait_st();
-    tc_fence_before();
-    __syncthreads();
-    if (tid == 0) {
+    // ---- epilogue
+    if (ok) ok = wait_or_abort(bar(LY::kOFull + s), 0u, abort);
+    if (__all_sync(0xffffffffu, ok) && active) {
       tc_fence_after();
+      const float inv_l = row_ok ? 1.f / l_sum : 0.f;
+      const int head = head0 + s;
+      const size_t obase = ((static_cast<size_t>(b) * prm.L + row) * prm.Hq + head) * D;
 #pragma unroll
-      for (int kk = 0; kk < BN / 16; ++kk)
-        mma_f16kind_ts(tO, tP + kk * 8, smem_desc_sw128(sV[slot] + kk * 16 * 128, LY::BOX, 1024),
-                       IDESC_PV, (vt > 0 || kk > 0) ? 1u : 0u);
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t rr[32];
+        __syncwarp();
+        tmem_ld32(tO(s) + lane_base + c * 32, rr);  // whole warp, valid row or not
+        tmem_wait_ld();
+        reg_fence(rr);
+        if (!row_ok) continue;
+        if (prm.out_f32) {
+          float4 *dst = reinterpret_cast<float4 *>(reinterpret_cast<float *>(prm.out) + obase + c * 32);
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            dst[e] = make_float4(u2f(rr[4 * e]) * inv_l, u2f(rr[4 * e + 1]) * inv_l,
+                                 u2f(rr[4 * e + 2]) * inv_l, u2f(rr[4 * e + 3]) * inv_l);
+        } else {
+          uint4 *dst = reinterpret_cast<uint4 *>(reinterpret_cast<__nv_bfloat16 *>(prm.out) + obase + c * 32);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            uint32_t wv[4];
+#pragma unroll
+            for (int f = 0; f < 4; ++f) {
+              const __nv_bfloat162 h2 = __floats2bfloat162_rn(u2f(rr[8 * e + 2 * f]) * inv_l,
+                                                              u2f(rr[8 * e + 2 * f + 1]) * inv_l);
+              wv[f] = *reinterpret_cast<const uint32_t *>(&h2);
+            }
+            dst[e] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+          }
+        }
+      }
+      if (row_ok && prm.lse)
+        prm.lse[(static_cast<size_t>(b) * prm.Hq + head) * prm.L + row] =
+            (m_used + log2f(l_sum)) * 0.69314718055994531f;
     }
   }
 
-  // Drain: every MMA issued by thread 0 completes before O is read / TMEM freed.
-  if (tid == 0) mma_commit(bar_o);
-  const bool drained = mbar_wait_bounded(bar_o, 0u, kWaitLimitNs);
-  tc_fence_after();
-  const bool good = __syncthreads_and(ok && drained);
-  if (!good) {
-    if (tid == 0) atomicOr(prm.dev_error, kDevTimeout);
-  } else {
-    const float inv_l = row_ok ? 1.f / l_sum : 0.f;
-    const size_t obase = ((static_cast<size_t>(b) * prm.L + row) * prm.Hq + h) * D;
-#pragma unroll
-    for (int c = 0; c < D / 32; ++c) {
-      uint32_t r[32];
-      __syncwarp();
-      tmem_ld32(tO + lane_base + c * 32, r);  // whole warp, valid row or not
-      tmem_wait_ld();
-      reg_fence(r);
-      if (!row_ok) continue;
-      if (prm.out_f32) {
-        float4 *dst = reinterpret_cast<float4 *>(reinterpret_cast<float *>(prm.out) + obase + c * 32);
-#pragma unroll
-        for (int e = 0; e < 8; ++e)
-          dst[e] = make_float4(u2f(r[4 * e]) * inv_l, u2f(r[4 * e + 1]) * inv_l,
-                               u2f(r[4 * e + 2]) * inv_l, u2f(r[4 * e + 3]) * inv_l);
-      } else {
-        uint4 *dst = reinterpret_cast<uint4 *>(reinterpret_cast<__nv_bfloat16 *>(prm.out) + obase + c * 32);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          uint32_t w[4];
-#pragma unroll
-          for (int f = 0; f < 4; ++f) {
-            const __nv_bfloat162 pr = __floats2bfloat162_rn(u2f(r[8 * e + 2 * f]) * inv_l,
-                                                            u2f(r[8 * e + 2 * f + 1]) * inv_l);
-            w[f] = *reinterpret_cast<const uint32_t *>(&pr);
-          }
-          dst[e] = make_uint4(w[0], w[1], w[2], w[3]);
-        }
-      }
-    }
-    if (row_ok && prm.lse)
-      prm.lse[(static_cast<size_t>(b) * prm.Hq + h) * prm.L + row] =
-          (m_used + log2f(l_sum)) * 0.69314718055994531f;
-  }
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) tmem_dealloc(tmem, LY::TMEM_COLS);
+  if (tid == 0 && *abort) atomicOr(prm.dev_error, kDevTimeout);
+  if (warp == kMmaWarp) tmem_dealloc(tmem, 512);
 }
 
 // ---------------------------------------------------------------- host side
@@ -406,6 +531,8 @@ cudaError_t launch_d(const PrefillArgs &a, cudaStream_t stream) {
   prm.G = a.G;
   prm.w0eff = a.G == 1 ? INT_MAX : a.w0;
   prm.n_qt = (a.L + BM - 1) / BM;
+  prm.grp = a.Hq / a.Hkv;
+  prm.npair = (prm.grp + 1) / 2;
   prm.scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(D));
   prm.out = a.out;
   prm.lse = a.lse;
@@ -415,7 +542,7 @@ cudaError_t launch_d(const PrefillArgs &a, cudaStream_t stream) {
   cudaError_t e = cudaFuncSetAttribute(bifocal_prefill_kernel<D>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  const dim3 grid(prm.n_qt, a.Hq, a.B);
+  const dim3 grid(prm.n_qt, a.Hkv * prm.npair, a.B);
   bifocal_prefill_kernel<D><<<grid, kThreads, smem, stream>>>(tqt, tqr, tkt, tkr, tv, prm);
   return cudaGetLastError();
 }
