@@ -180,6 +180,32 @@ JL_API int jetlong_decode(const void *q, const void *k_cache, const void *v_cach
                    void *workspace, size_t workspace_bytes, jl_stream_t stream);
 
 /*
+ * jetlong_decode without a workspace argument, for callers that cannot
+ * allocate device memory for one: processes whose device memory belongs to a
+ * single arena or caching allocator, or generation loops that must not call
+ * cudaMalloc because an allocation would stall the device.  (The paper has no
+ * counterpart; this is a property of the library, not of the method.)
+ *
+ * Same arguments, layouts and results as jetlong_decode.  The split partials
+ * live in a fixed 4 MiB buffer inside the library's device image, which every
+ * GPU that loads the library holds until the process exits; the call
+ * allocates nothing.  Sizes whose workspace
+ * (jetlong_decode_workspace_size(B, Hq, Hkv, L, D)) exceeds 4 MiB are
+ * rejected with JL_ERR_WORKSPACE before anything is launched.
+ *   - The first call on each device looks up the buffer's device address on
+ *     the host (once per device, with that device current); make that first
+ *     call before any stream capture on that device.
+ *   - All calls share the one buffer, and each call fully overwrites the part
+ *     it reads, so nothing needs clearing between calls; but calls whose
+ *     kernels overlap on the GPU (different streams, or different host
+ *     threads) race on the buffer and must be serialised by the caller.
+ */
+JL_API int jetlong_decode_noalloc(const void *q, const void *k_cache, const void *v_cache,
+                                  void *out, float *lse, int B, int Hq, int Hkv, int L, int Lcap,
+                                  int D, int w_pretrained, int w0, float rope_theta, int out_dtype,
+                                  jl_stream_t stream);
+
+/*
  * Write keys into the true-position cache (§3.2): for t < n,
  *   k_cache[b, pos0 + t, h, :] = RoPE(k[b, t, h, :], pos0 + t).
  *

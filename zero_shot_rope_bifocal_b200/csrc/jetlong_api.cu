@@ -322,3 +322,60 @@ int jetlong_device_status(jl_stream_t stream) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Decode without any device allocation.
+//
+// Some callers cannot hand this library a workspace: their process forbids
+// cudaMalloc outside start-up (a serving loop whose device memory is owned by
+// one arena or caching allocator, or a latency-critical generation loop where
+// an allocation would stall the device).  jetlong_decode_noalloc gives them
+// the decode step with its split partials kept in a fixed buffer that lives in
+// this library's device image instead.  Every GPU that loads the library holds
+// this buffer until the process exits.
+namespace jl {
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;  // 4 MiB
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+std::mutex g_noalloc_mu;
+void *g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of the scratch buffer on the current device.  The first call
+// on a device looks it up (with that device current) and keeps it.
+int noalloc_scratch(void **out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return JL_ERR_NO_DEVICE;
+  }
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void *ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr) {
+      cudaGetLastError();
+      return JL_ERR_CUDA;
+    }
+    g_noalloc_ptr[dev] = ptr;
+  }
+  *out = g_noalloc_ptr[dev];
+  return JL_OK;
+}
+
+}  // namespace
+}  // namespace jl
+
+extern "C" int jetlong_decode_noalloc(const void *q, const void *k_cache, const void *v_cache,
+                                      void *out, float *lse, int B, int Hq, int Hkv, int L,
+                                      int Lcap, int D, int w_pretrained, int w0, float rope_theta,
+                                      int out_dtype, jl_stream_t stream) {
+  if (check_common(B, Hq, Hkv, L, D) != JL_OK) return check_common(B, Hq, Hkv, L, D);
+  if (decode_ws_bytes(B, Hq, Hkv, L, D) > kNoAllocScratchBytes) return JL_ERR_WORKSPACE;
+  void *scratch = nullptr;
+  const int st = noalloc_scratch(&scratch);
+  if (st != JL_OK) return st;
+  return jetlong_decode(q, k_cache, v_cache, out, lse, B, Hq, Hkv, L, Lcap, D, w_pretrained, w0,
+                        rope_theta, out_dtype, scratch, kNoAllocScratchBytes, stream);
+}

@@ -47,6 +47,8 @@ SIGNATURES = {
     "jetlong_decode_workspace_size": (_SZ, [_I, _I, _I, _I, _I]),
     "jetlong_decode": (_I, [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _I, _I, _F, _I,
                             _VP, _SZ, _VP]),
+    "jetlong_decode_noalloc": (_I, [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _I, _I, _F,
+                                    _I, _VP]),
     "jetlong_rope_cache": (_I, [_VP, _VP, _I, _I, _I, _I, _I, _I, _F, _VP]),
     "jetlong_device_status": (_I, [_VP]),
 }
@@ -233,6 +235,27 @@ def jetlong_decode(q, k_cache, v_cache, L: int, w_pretrained: int, w0: int, rope
                               Hkv, int(L), Lcap, D, int(w_pretrained), int(w0), float(rope_theta),
                               od, _ptr(workspace), workspace.numel(), _stream_ptr(stream))
     _check("jetlong_decode", st)
+    return out, lse
+
+
+def jetlong_decode_noalloc(q, k_cache, v_cache, L: int, w_pretrained: int, w0: int,
+                           rope_theta: float, out, lse=None, *, stream=None):
+    """jetlong_decode for callers that cannot allocate device memory: the
+    library keeps the split partials in its own fixed 4 MiB device buffer.
+    ``out`` (and ``lse``, if given) are caller-provided; nothing is allocated."""
+    B, Hq, D = q.shape
+    Lcap, Hkv = k_cache.shape[1], k_cache.shape[2]
+    _require(q, "q", (B, Hq, D), torch.bfloat16)
+    _require(k_cache, "k_cache", (B, Lcap, Hkv, D), torch.bfloat16)
+    _require(v_cache, "v_cache", (B, Lcap, Hkv, D), torch.bfloat16)
+    _require(out, "out", (B, Hq, D), out.dtype)
+    if lse is not None:
+        _require(lse, "lse", (B, Hq), torch.float32)
+    st = lib().jetlong_decode_noalloc(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(out), _ptr(lse),
+                                      B, Hq, Hkv, int(L), Lcap, D, int(w_pretrained), int(w0),
+                                      float(rope_theta), _out_dtype(out.dtype),
+                                      _stream_ptr(stream))
+    _check("jetlong_decode_noalloc", st)
     return out, lse
 
 
