@@ -319,7 +319,12 @@ def run_native(args):
 
     for _ in range(max(3, args.warmup)):
         dstep()
-    n_dec = args.decode_steps
+    # 256-step loops, repeated so that the timed region lasts long enough for
+    # the clock sampler (one sample per 200 ms); the mean over all steps is
+    # reported.
+    n_loop = args.decode_steps
+    n_rep = max(1, args.decode_reps)
+    n_dec = n_loop * n_rep
     with ClockSampler(local) as dclocks:
         barrier()
         torch.cuda.synchronize(dev)
@@ -400,6 +405,7 @@ def run_native(args):
                          "traffic": None},
             "breakdown_ms": {"rotate": rot_ms, "attend": attn_ms},
             "decode": {"workload": DECODE_WORKLOAD, "us_per_token": us_tok, "steps": n_dec,
+                       "loop": f"{n_rep} x {n_loop} steps",
                        "achieved_gbs": dec_gbs, "peak_gbs": peaks["hbm_gbs"],
                        "frac": dec_gbs / peaks["hbm_gbs"],
                        "nominal_frac": dec_gbs / NOMINAL["hbm_gbs"],
@@ -424,6 +430,7 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
     ap.add_argument("--decode-steps", type=int, default=256)
+    ap.add_argument("--decode-reps", type=int, default=8)
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--reference-seconds", type=float, default=120.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")

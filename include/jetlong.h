@@ -187,10 +187,10 @@ JL_API int jetlong_decode(const void *q, const void *k_cache, const void *v_cach
  * counterpart; this is a property of the library, not of the method.)
  *
  * Same arguments, layouts and results as jetlong_decode.  The split partials
- * live in a fixed 4 MiB buffer inside the library's device image, which every
+ * live in a fixed 8 MiB buffer inside the library's device image, which every
  * GPU that loads the library holds until the process exits; the call
  * allocates nothing.  Sizes whose workspace
- * (jetlong_decode_workspace_size(B, Hq, Hkv, L, D)) exceeds 4 MiB are
+ * (jetlong_decode_workspace_size(B, Hq, Hkv, L, D)) exceeds 8 MiB are
  * rejected with JL_ERR_WORKSPACE before anything is launched.
  *   - The first call on each device looks up the buffer's device address on
  *     the host (once per device, with that device current); make that first

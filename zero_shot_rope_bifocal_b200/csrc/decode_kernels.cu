@@ -6,7 +6,9 @@
 // Split-KV: CTA (s, c, b) streams key chunk s of KV heads [8c, 8c + 8) of
 // batch b through a three-stage shared-memory ring filled by bulk async copies
 // (cp.async.bulk + mbarrier transaction counts): each stage holds P tokens of
-// K and V for the CTA's heads, which are contiguous in the cache.  Warp w owns
+// K and V for the CTA's heads, which are contiguous in the cache.  Two CTAs
+// share an SM, so 16 warps hide each other's shuffle and shared-memory
+// latencies.  Warp w owns
 // KV head 8c + w and its Hq/Hkv query heads; lane l holds channel pairs
 // (i, i + D/2) for i in {2l, 2l+1} (D = 128) or {l} (D = 64), so the
 // correction rotation of a pair is lane-local.
@@ -36,19 +38,19 @@ namespace {
 constexpr int kDecWarps = 8;  // = KV heads per CTA
 constexpr int kDecThreads = kDecWarps * 32;
 constexpr int kStages = 3;
-constexpr int kMaxGrp = 8;
+constexpr int kCtasPerSm = 2;
 constexpr float kLog2e = 1.4426950408889634f;
 
 template <int D>
 struct DecCfg {
-  static constexpr int P = D == 128 ? 16 : 32;     // tokens per stage
+  static constexpr int P = D == 128 ? 8 : 16;      // tokens per stage
   static constexpr int EPL = D / 32;               // channels per lane
   static constexpr int HEAD_BYTES = D * 2;         // one head's K (or V) row
-  static constexpr int STAGE_HALF = P * kDecWarps * HEAD_BYTES;  // K (or V) of a stage
+  static constexpr int STAGE_HALF = P * kDecWarps * HEAD_BYTES;  // K (or V) of a stage: 16 KB
   static constexpr int STAGE = 2 * STAGE_HALF;
   static constexpr int CS = kStages * STAGE;                     // cos/sin table [P][D/2]
   static constexpr int BAR = CS + P * (D / 2) * 8;
-  static constexpr int BYTES = BAR + 8 * kStages + 16;
+  static constexpr int BYTES = BAR + 8 * kStages + 16;  // about 100 KB: two CTAs per SM
 };
 
 // Channel held by slot e of lane l: slots [0, EPL/2) are the first members of
@@ -83,50 +85,76 @@ __device__ __forceinline__ void bulk_copy(uint32_t dst, const void *src, uint32_
       : "memory");
 }
 
-// Sum 32 per-lane values across the warp so that lane l ends with the total of
-// value l (reduce-scatter by halving).  With `half_only` the values 16..31 are
-// absent: lanes l and l + 16 both end with the total of value l & 15.
-template <bool kHalfOnly>
+// Sum NV per-lane values (v[0..NV)) across the warp.  Halving steps whose
+// offset is at least NV add whole arrays; the remaining steps scatter, so that
+// lane l ends with the warp total of value (l % NV).
+template <int NV>
 __device__ __forceinline__ float reduce_scatter(float (&v)[32], int lane) {
-  if constexpr (kHalfOnly) {
 #pragma unroll
-    for (int k = 0; k < 16; ++k) v[k] += __shfl_xor_sync(0xffffffffu, v[k], 16);
-  } else {
-    const bool up = lane & 16;
+  for (int o = 16; o >= 1; o >>= 1) {
+    if (o >= NV) {
 #pragma unroll
-    for (int k = 0; k < 16; ++k) {
-      const float send = up ? v[k] : v[k + 16];
-      const float keep = up ? v[k + 16] : v[k];
-      v[k] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
-    }
-  }
+      for (int k = 0; k < NV; ++k) v[k] += __shfl_xor_sync(0xffffffffu, v[k], o);
+    } else {
+      const bool up = lane & o;
 #pragma unroll
-  for (int o = 8; o >= 1; o >>= 1) {
-    const bool up = lane & o;
-#pragma unroll
-    for (int k = 0; k < o; ++k) {
-      const float send = up ? v[k] : v[k + o];
-      const float keep = up ? v[k + o] : v[k];
-      v[k] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+      for (int k = 0; k < o; ++k) {
+        const float send = up ? v[k] : v[k + o];
+        const float keep = up ? v[k + o] : v[k];
+        v[k] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+      }
     }
   }
   return v[0];
 }
 
+// Partial dot products of one cached key (the lane's channels) with the
+// group's queries; remote keys are first turned by the correction rotation.
+template <int D, int GRP, bool REMOTE>
+__device__ __forceinline__ void token_partials(float (&part)[32], int slot0,
+                                               const __nv_bfloat16 *krow, const float2 *cs_row,
+                                               int lane, const float (&q)[GRP][D / 32]) {
+  constexpr int EPL = D / 32;
+  float kv[EPL];
+  load_row<D>(krow, lane, kv);
+  if constexpr (REMOTE) {
+    float2 cs[EPL / 2];
+    if constexpr (D == 128) {
+      const float4 c4 = *reinterpret_cast<const float4 *>(cs_row + 2 * lane);
+      cs[0] = make_float2(c4.x, c4.y);
+      cs[1] = make_float2(c4.z, c4.w);
+    } else {
+      cs[0] = cs_row[lane];
+    }
+#pragma unroll
+    for (int e = 0; e < EPL / 2; ++e) {
+      const float x = kv[e], y = kv[e + EPL / 2];
+      kv[e] = x * cs[e].x - y * cs[e].y;
+      kv[e + EPL / 2] = x * cs[e].y + y * cs[e].x;
+    }
+  }
+#pragma unroll
+  for (int h = 0; h < GRP; ++h) {
+    float d = q[h][0] * kv[0];
+#pragma unroll
+    for (int e = 1; e < EPL; ++e) d = fmaf(q[h][e], kv[e], d);
+    part[slot0 + h] = d;
+  }
+}
+
 template <int D, int GRP>
-__global__ void __launch_bounds__(kDecThreads, 1)
+__global__ void __launch_bounds__(kDecThreads, kCtasPerSm)
 decode_split_kernel(DecodeArgs a) {
   using C = DecCfg<D>;
   constexpr int P = C::P, EPL = C::EPL, HALF = D / 2;
   constexpr int NB = (32 / GRP) < P ? (32 / GRP) : P;  // tokens per score batch
-  constexpr int NV = NB * GRP;                         // values per batch: 16 or 32
-  static_assert(NV == 16 || NV == 32, "batch must fill 16 or 32 lanes");
+  constexpr int NV = NB * GRP;                         // values per batch: 8, 16 or 32
+  static_assert(NV == 8 || NV == 16 || NV == 32, "batch must fill 8, 16 or 32 values");
   static_assert(P % NB == 0, "batches tile a stage");
 
   extern __shared__ __align__(128) uint8_t dsm[];
   const uint32_t sb = smem_u32(dsm);
   float2 *cs_tab = reinterpret_cast<float2 *>(dsm + C::CS);  // [P][D/2] (cos, sin)
-  volatile uint32_t *abort = reinterpret_cast<volatile uint32_t *>(dsm + C::BAR + 8 * kStages);
 
   const int s = blockIdx.x, chunk_id = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -145,7 +173,6 @@ decode_split_kernel(DecodeArgs a) {
 
   if (tid == 0) {
     for (int i = 0; i < kStages; ++i) mbar_init(sb + C::BAR + 8 * i, 1);
-    *abort = 0u;
     fence_mbar_init();
   }
   __syncthreads();
@@ -177,15 +204,13 @@ decode_split_kernel(DecodeArgs a) {
   const double theta = static_cast<double>(a.theta);
   const float qscale = kLog2e / sqrtf(static_cast<float>(D));
   float qt[GRP][EPL], qr[GRP][EPL];
-  double freq[EPL / 2];
-#pragma unroll
-  for (int e = 0; e < EPL / 2; ++e) freq[e] = rope_freq(chan<D>(lane, e), D, theta);
   {
     float ct[EPL / 2], st[EPL / 2], cr[EPL / 2], sr[EPL / 2];
 #pragma unroll
     for (int e = 0; e < EPL / 2; ++e) {
-      rope_cos_sin(p, freq[e], ct[e], st[e]);
-      rope_cos_sin(remap(p, G), freq[e], cr[e], sr[e]);
+      const double fr = rope_freq(chan<D>(lane, e), D, theta);
+      rope_cos_sin(p, fr, ct[e], st[e]);
+      rope_cos_sin(remap(p, G), fr, cr[e], sr[e]);
     }
 #pragma unroll
     for (int h = 0; h < GRP; ++h) {
@@ -201,8 +226,6 @@ decode_split_kernel(DecodeArgs a) {
       }
     }
   }
-  // Channel e of the lane: e < EPL/2 are the first members of the pairs,
-  // e >= EPL/2 their partners (+D/2).
 
   float acc[GRP][EPL];
 #pragma unroll
@@ -243,44 +266,43 @@ decode_split_kernel(DecodeArgs a) {
       const uint8_t *kst = dsm + slot * C::STAGE + warp * C::HEAD_BYTES;
       const uint8_t *vst = kst + C::STAGE_HALF;
 #pragma unroll 1
-      for (int tb = 0; tb < P; tb += NB) {
-        if (tb >= n) break;
-        // partial scores of NB tokens x GRP heads
+      for (int tb = 0; tb < n; tb += NB) {
+        // partial scores of NB tokens x GRP heads; the query variant is
+        // chosen per batch (all remote / all local), per token only on the
+        // batch that straddles the window edge
         float part[32];
 #pragma unroll
         for (int k = 0; k < 32; ++k) part[k] = 0.f;
+        const int nb = min(NB, n - tb);
+        const int jb = jt + tb;
+        const bool all_remote = p - (jb + nb - 1) > w0eff;
+        const bool all_local = p - jb <= w0eff;
+        auto krow = [&](int pb) {
+          return reinterpret_cast<const __nv_bfloat16 *>(kst + (tb + pb) * row_bytes);
+        };
+        if (all_remote) {
 #pragma unroll
-        for (int pb = 0; pb < NB; ++pb) {
-          const int tt = tb + pb;
-          if (tt < n) {
-            const int j = jt + tt;
-            const __nv_bfloat16 *krow =
-                reinterpret_cast<const __nv_bfloat16 *>(kst + tt * row_bytes);
-            float kv[EPL];
-            load_row<D>(krow, lane, kv);
-            const bool remote = p - j > w0eff;
-            if (remote) {
+          for (int pb = 0; pb < NB; ++pb)
+            if (pb < nb)
+              token_partials<D, GRP, true>(part, pb * GRP, krow(pb), cs_tab + (tb + pb) * HALF, lane, qr);
+        } else if (all_local) {
 #pragma unroll
-              for (int e = 0; e < EPL / 2; ++e) {
-                const float2 cs = cs_tab[tt * HALF + chan<D>(lane, e)];
-                const float x = kv[e], y = kv[e + EPL / 2];
-                kv[e] = x * cs.x - y * cs.y;
-                kv[e + EPL / 2] = x * cs.y + y * cs.x;
-              }
+          for (int pb = 0; pb < NB; ++pb)
+            if (pb < nb)
+              token_partials<D, GRP, false>(part, pb * GRP, krow(pb), cs_tab, lane, qt);
+        } else {
+#pragma unroll
+          for (int pb = 0; pb < NB; ++pb)
+            if (pb < nb) {
+              if (p - (jb + pb) > w0eff)
+                token_partials<D, GRP, true>(part, pb * GRP, krow(pb), cs_tab + (tb + pb) * HALF, lane, qr);
+              else
+                token_partials<D, GRP, false>(part, pb * GRP, krow(pb), cs_tab, lane, qt);
             }
-#pragma unroll
-            for (int h = 0; h < GRP; ++h) {
-              float d = 0.f;
-#pragma unroll
-              for (int e = 0; e < EPL; ++e) d = fmaf(remote ? qr[h][e] : qt[h][e], kv[e], d);
-              part[pb * GRP + h] = d;
-            }
-          }
         }
-        const float sc = reduce_scatter<NV == 16>(part, lane);
+        const float sc = reduce_scatter<NV>(part, lane);
         const int my_pb = (lane % NV) / GRP;
-        const bool valid = tb + my_pb < n;
-        const float sv = valid ? sc : -INFINITY;
+        const float sv = my_pb < nb ? sc : -INFINITY;
         // online softmax for head (lane % GRP) over the batch
         float bm = sv;
 #pragma unroll
@@ -301,12 +323,9 @@ decode_split_kernel(DecodeArgs a) {
         }
 #pragma unroll
         for (int pb = 0; pb < NB; ++pb) {
-          const int tt = tb + pb;
-          if (tt < n) {
-            const __nv_bfloat16 *vrow =
-                reinterpret_cast<const __nv_bfloat16 *>(vst + tt * row_bytes);
+          if (pb < nb) {
             float vv[EPL];
-            load_row<D>(vrow, lane, vv);
+            load_row<D>(reinterpret_cast<const __nv_bfloat16 *>(vst + (tb + pb) * row_bytes), lane, vv);
 #pragma unroll
             for (int h = 0; h < GRP; ++h) {
               const float pr = __shfl_sync(0xffffffffu, pm, pb * GRP + h);
@@ -418,17 +437,17 @@ cudaError_t launch_decode_d(const DecodeArgs &a, cudaStream_t stream) {
 }  // namespace
 
 void decode_plan(int B, int Hkv, int L, int *n_split, int *chunk) {
-  // One CTA per SM (each holds a 3-stage ring) over the 148 SMs of a B200;
-  // chunks are whole stages of 16 tokens.  The split count is non-decreasing
-  // in L, so workspace sized for the largest L of a generation loop covers
-  // every step.
+  // Two CTAs per SM (each holds a 3-stage ring of about 100 KB) over the 148
+  // SMs of a B200; chunks are whole stages (8 or 16 tokens).  The split count
+  // is non-decreasing in L, so workspace sized for the largest L of a
+  // generation loop covers every step.
   const int units = B * ((Hkv + kDecWarps - 1) / kDecWarps);
-  int ns = (148 + units - 1) / units;
+  int ns = (kCtasPerSm * 148 + units - 1) / units;
   const int max_ns = (L + 15) / 16;
   if (ns > max_ns) ns = max_ns;
   if (ns < 1) ns = 1;
   int ch = (L + ns - 1) / ns;
-  ch = (ch + 31) / 32 * 32;  // a whole number of stages for both head dims
+  ch = (ch + 15) / 16 * 16;  // a whole number of stages for both head dims
   *chunk = ch;
   *n_split = (L + ch - 1) / ch;
 }

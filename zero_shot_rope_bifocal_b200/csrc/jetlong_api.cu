@@ -336,7 +336,7 @@ int jetlong_device_status(jl_stream_t stream) {
 namespace jl {
 namespace {
 
-constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;  // 4 MiB
+constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;  // 8 MiB
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 

@@ -93,6 +93,28 @@ struct Params {
 
 __device__ __forceinline__ float u2f(uint32_t u) { return __uint_as_float(u); }
 
+// 2^x on the FMA pipe for a pair of arguments (x <= 2^22), used for a share
+// of the softmax exponentials so that the special-function unit is not the
+// bottleneck.  x = n + f with n = round(x), f in [-1/2, 1/2]; 2^f is a cubic
+// whose coefficients come from exp2_poly_fit.py (relative error 7.5e-5,
+// below the FP16 rounding of P); 2^n is added to the exponent field.
+// Arguments are clamped at -125, so -inf gives 2^-125 (zero once in FP16).
+__device__ __forceinline__ float2 exp2_fma2(float2 x) {
+  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23: x + kRound rounds x to an integer
+  x.x = fmaxf(x.x, -125.0f);
+  x.y = fmaxf(x.y, -125.0f);
+  const float2 t = fadd2(x, make_float2(kRound, kRound));      // n in the low mantissa bits
+  const float2 n = fadd2(t, make_float2(-kRound, -kRound));    // n as a float
+  const float2 f = ffma2(n, make_float2(-1.f, -1.f), x);       // x - n
+  float2 p = ffma2(make_float2(0.0551716648f, 0.0551716648f), f,
+                   make_float2(0.242611125f, 0.242611125f));
+  p = ffma2(p, f, make_float2(0.693260968f, 0.693260968f));
+  p = ffma2(p, f, make_float2(0.999928057f, 0.999928057f));
+  // bits(t) << 23 == n << 23 (the bits of kRound shift out); add to p's exponent
+  return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
+                     __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
+}
+
 __device__ __forceinline__ void set_regs_softmax() {
   asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftmaxRegs));
 }
@@ -380,10 +402,18 @@ bifocal_prefill_kernel(const __grid_constant__ CUtensorMap tm_qt,
           if (!valid) x[c] = -INFINITY;
         }
       }
-      float tmax = -INFINITY;
+      // row max: a tree of three-input maxima (raw scores; the scale is positive)
+      float mx[4] = {x[0], x[1], x[2], x[3]};
 #pragma unroll
-      for (int c = 0; c < BN; ++c) tmax = fmaxf(tmax, x[c]);
-      tmax *= prm.scale_log2;  // raw scores; the scale is positive
+      for (int c = 4; c < BN; c += 8) {
+        mx[0] = fmax3(mx[0], x[c], x[c + 1]);
+        mx[1] = fmax3(mx[1], x[c + 2], x[c + 3]);
+        if (c + 4 < BN) {
+          mx[2] = fmax3(mx[2], x[c + 4], x[c + 5]);
+          mx[3] = fmax3(mx[3], x[c + 6], x[c + 7]);
+        }
+      }
+      const float tmax = fmaxf(fmax3(mx[0], mx[1], mx[2]), mx[3]) * prm.scale_log2;
       const bool grow =
           tmax > m_used + kRescaleThreshold || (m_used == -INFINITY && tmax > -INFINITY);
       float alpha = 1.f;
@@ -407,16 +437,31 @@ bifocal_prefill_kernel(const __grid_constant__ CUtensorMap tm_qt,
           tmem_st32(tO(s) + lane_base + c * 32, rr);
         }
       }
-      float lsum = 0.f;
+      // p = 2^(s * scale - m): masked entries are -inf and give 0 (or 2^-125
+      // on the FMA path, which rounds to 0 in FP16); a row with nothing valid
+      // yet has all entries -inf.  One column pair in four takes the FMA-pipe
+      // exponential, the rest the special-function unit.
       const float neg_m = m_used == -INFINITY ? 0.f : -m_used;
+      const float2 sc2 = make_float2(prm.scale_log2, prm.scale_log2);
+      const float2 nm2 = make_float2(neg_m, neg_m);
+      float2 acc2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                        make_float2(0.f, 0.f)};
 #pragma unroll
-      for (int c = 0; c < BN; ++c) {
-        // masked entries are -inf and give 0; a row with nothing valid yet
-        // has all entries -inf
-        x[c] = exp2f(fmaf(x[c], prm.scale_log2, neg_m));
-        lsum += x[c];
+      for (int c = 0; c < BN; c += 2) {
+        float2 v = ffma2(make_float2(x[c], x[c + 1]), sc2, nm2);
+        if ((c & 7) == 0) {
+          v = exp2_fma2(v);
+        } else {
+          v.x = ex2_sfu(v.x);
+          v.y = ex2_sfu(v.y);
+        }
+        x[c] = v.x;
+        x[c + 1] = v.y;
+        acc2[(c >> 1) & 3] = fadd2(acc2[(c >> 1) & 3], v);
       }
-      l_sum += lsum;
+      const float2 a01 = fadd2(acc2[0], acc2[1]), a23 = fadd2(acc2[2], acc2[3]);
+      const float2 a = fadd2(a01, a23);
+      l_sum += a.x + a.y;
       __syncwarp();
 #pragma unroll
       for (int c = 0; c < BN / 64; ++c) {

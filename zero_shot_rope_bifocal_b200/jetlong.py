@@ -241,7 +241,7 @@ def jetlong_decode(q, k_cache, v_cache, L: int, w_pretrained: int, w0: int, rope
 def jetlong_decode_noalloc(q, k_cache, v_cache, L: int, w_pretrained: int, w0: int,
                            rope_theta: float, out, lse=None, *, stream=None):
     """jetlong_decode for callers that cannot allocate device memory: the
-    library keeps the split partials in its own fixed 4 MiB device buffer.
+    library keeps the split partials in its own fixed 8 MiB device buffer.
     ``out`` (and ``lse``, if given) are caller-provided; nothing is allocated."""
     B, Hq, D = q.shape
     Lcap, Hkv = k_cache.shape[1], k_cache.shape[2]
