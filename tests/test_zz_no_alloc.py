@@ -45,8 +45,8 @@ def test_noalloc_decode_matches_decode_on_two_calls_in_a_row():
 
 
 def test_noalloc_rejects_sizes_beyond_its_buffer():
-    # 64 query heads over 8 KV heads need ~8.1 MiB of partials: above the 8 MiB buffer
-    w = Workload("big", 1, 64, 8, 128, 4096, 32768, 4096, 1e6, 78, False, kind="decode")
+    # a batch of 512 decodes at once needs ~8.5 MB of partials: above the 8 MiB buffer
+    w = Workload("big", 512, 32, 8, 128, 16, 32768, 4096, 1e6, 78, False, kind="decode")
     assert jl.jetlong_decode_workspace_size(w.B, w.Hq, w.Hkv, w.L, w.D) > (8 << 20)
     q = torch.zeros((w.B, w.Hq, w.D), dtype=torch.bfloat16, device="cuda")
     kc = torch.zeros((w.B, w.L, w.Hkv, w.D), dtype=torch.bfloat16, device="cuda")

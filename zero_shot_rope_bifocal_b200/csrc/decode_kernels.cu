@@ -3,27 +3,35 @@
 // correction rotation"; score rule of §3; schedule of §3.1 with L = tokens in
 // the cache including the new one, query at p = L - 1).
 //
-// Split-KV: CTA (s, c, b) streams key chunk s of KV heads [8c, 8c + 8) of
-// batch b through a three-stage shared-memory ring filled by bulk async copies
-// (cp.async.bulk + mbarrier transaction counts): each stage holds P tokens of
-// K and V for the CTA's heads, which are contiguous in the cache.  Two CTAs
-// share an SM, so 16 warps hide each other's shuffle and shared-memory
-// latencies.  Warp w owns
-// KV head 8c + w and its Hq/Hkv query heads; lane l holds channel pairs
-// (i, i + D/2) for i in {2l, 2l+1} (D = 128) or {l} (D = 64), so the
-// correction rotation of a pair is lane-local.
-//
 // Per token j: keys with p - j <= w0 are scored as cached against
-// RoPE(x_q, p); older keys are first rotated by Delta j = f(j) - j (the
-// correction rotation, so the cache is never rewritten) and scored against
-// RoPE(x_q, f(p)).  cos/sin of Delta j * theta_i are evaluated once per token
-// per CTA (double-precision angle, reduced, then the hardware sine/cosine on
-// [-pi, pi]) and shared by all heads.  The partial dot products of a batch of
-// tokens x query heads (32 values per lane) are summed across the warp by a
-// reduce-scatter that leaves one (token, head) score per lane; an online
-// softmax per head then weights V.  Each CTA writes its unnormalised partial
-// output with its running max and sum; a second kernel merges the partials by
-// log-sum-exp, one warp per head.
+// RoPE(x_q, p); older keys are first turned by the correction rotation
+// R(Delta j), Delta j = f(j) - j (so the cache is never rewritten), and scored
+// against RoPE(x_q, f(p)).
+//
+// Split-KV: CTA (s, c, b) streams key chunk s of KV heads [8c, 8c + 8) of
+// batch b (two CTAs per SM).  Warp 0 fills a three-stage shared-memory ring
+// with bulk async copies (cp.async.bulk, one per token and tensor, into rows
+// padded by 16 bytes; completion on the stage's "full" mbarrier).  For each stage the
+// CTA also builds a table of cos/sin(Delta j * theta_i) for its tokens, shared
+// by all heads; every warp writes some of its rows once it is two stages
+// behind.  The phase Delta j * theta_i / (2 pi) is formed exactly modulo one
+// turn in 64-bit fixed point (theta_i / (2 pi) held as a 64-bit binary
+// fraction), so the hardware sine/cosine only ever sees [-pi, pi).
+// Eight warps, one per KV head, run each stage on the tensor cores
+// (mma.sync m16n8k16):
+//   * S = Q K^T: the A operand holds the group's query heads (rows), FP16,
+//     pre-scaled by log2(e)/sqrt(D); K arrives through ldmatrix as B
+//     fragments, turned (remote tokens) and converted to FP16 in registers;
+//   * an online softmax per head over the stage's tokens (fp32 statistics,
+//     lazy rescaling);
+//   * O^T += V^T P^T: V through ldmatrix.trans, P taken straight from the S
+//     accumulator fragment (BF16), O^T accumulated in fp32 registers;
+// each warp then releases the stage on its "empty" mbarrier, and warp 0
+// refills the slot once all have; no CTA-wide barrier runs in the loop, so
+// warps may drift a stage apart.  Each CTA writes its unnormalised partial
+// output with its
+// running max and sum; a second kernel (launched as a programmatic dependent
+// of the first) merges the partials by log-sum-exp, one CTA per head.
 //
 // Traffic: K and V once (2 * L * Hkv * D * 2 bytes per token of output);
 // everything else is O(Hq * D * n_split).
@@ -35,47 +43,35 @@
 namespace jl {
 namespace {
 
-constexpr int kDecWarps = 8;  // = KV heads per CTA
+constexpr int kDecWarps = 8;  // warps = KV heads per CTA
 constexpr int kDecThreads = kDecWarps * 32;
 constexpr int kStages = 3;
 constexpr int kCtasPerSm = 2;
 constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
 template <int D>
 struct DecCfg {
-  static constexpr int P = D == 128 ? 8 : 16;      // tokens per stage
-  static constexpr int EPL = D / 32;               // channels per lane
-  static constexpr int HEAD_BYTES = D * 2;         // one head's K (or V) row
-  static constexpr int STAGE_HALF = P * kDecWarps * HEAD_BYTES;  // K (or V) of a stage: 16 KB
-  static constexpr int STAGE = 2 * STAGE_HALF;
-  static constexpr int CS = kStages * STAGE;                     // cos/sin table [P][D/2]
-  static constexpr int BAR = CS + P * (D / 2) * 8;
-  static constexpr int BYTES = BAR + 8 * kStages + 16;  // about 100 KB: two CTAs per SM
+  static constexpr int P = D == 128 ? 8 : 16;   // tokens per stage
+  static constexpr int NBLK = P / 8;            // 8-token score blocks per stage
+  static constexpr int KB = D / 16;             // 16-channel k-blocks
+  static constexpr int ROW = kDecWarps * D * 2 + 16;  // padded token row (all CTA heads)
+  static constexpr int HALF_STAGE = P * ROW;          // K (or V) of a stage
+  static constexpr int STAGE = 2 * HALF_STAGE;
+  // cos/sin row of one token: (cos, sin) per frequency, padded so two rows
+  // read in one 128 B wavefront use different banks (D = 128; at D = 64 the
+  // full padding would not leave room for two CTAs per SM).
+  static constexpr int CS_ROW = (D / 2) * 8 + (D == 128 ? 64 : 16);
+  static constexpr int CS_TAB = P * CS_ROW;           // one stage's correction table
+  static constexpr int CS = kStages * STAGE;          // kStages tables (one per slot)
+  static constexpr int OMEGA = CS + kStages * CS_TAB;  // theta_i / (2 pi), 0.64 fixed point
+  static constexpr int QCS = OMEGA + (D / 2) * 8;      // (cos, sin) at p and f(p), [2][D/2]
+  static constexpr int BAR = QCS + 2 * (D / 2) * 8;    // full, empty, tready [kStages] each
+  static constexpr int ABORT = BAR + 24 * kStages + 8;
+  static constexpr int BYTES = ABORT + 16;  // about 112 KB (D = 128): two CTAs per SM
 };
-
-// Channel held by slot e of lane l: slots [0, EPL/2) are the first members of
-// the lane's channel pairs, slots [EPL/2, EPL) their partners (+ D/2).
-template <int D>
-__device__ __forceinline__ int chan(int l, int e) {
-  if constexpr (D == 128) return (e & 1) + 2 * l + (e >> 1) * 64;  // 2l, 2l+1, 64+2l, 65+2l
-  else return l + e * 32;                                          // l, 32+l
-}
-
-// The lane's EPL channels of one BF16 head row in shared memory, as fp32.
-template <int D>
-__device__ __forceinline__ void load_row(const __nv_bfloat16 *row, int lane, float (&x)[D / 32]) {
-  if constexpr (D == 128) {
-    const __nv_bfloat162 lo = *reinterpret_cast<const __nv_bfloat162 *>(row + 2 * lane);
-    const __nv_bfloat162 hi = *reinterpret_cast<const __nv_bfloat162 *>(row + 64 + 2 * lane);
-    x[0] = __low2float(lo);
-    x[1] = __high2float(lo);
-    x[2] = __low2float(hi);
-    x[3] = __high2float(hi);
-  } else {
-    x[0] = bf2f(row[lane]);
-    x[1] = bf2f(row[lane + 32]);
-  }
-}
+static_assert(kCtasPerSm * (DecCfg<128>::BYTES + 1024) <= 233472, "two CTAs per SM");
+static_assert(kCtasPerSm * (DecCfg<64>::BYTES + 1024) <= 233472, "two CTAs per SM");
 
 __device__ __forceinline__ void bulk_copy(uint32_t dst, const void *src, uint32_t bytes,
                                           uint32_t bar) {
@@ -85,60 +81,134 @@ __device__ __forceinline__ void bulk_copy(uint32_t dst, const void *src, uint32_
       : "memory");
 }
 
-// Sum NV per-lane values (v[0..NV)) across the warp.  Halving steps whose
-// offset is at least NV add whole arrays; the remaining steps scatter, so that
-// lane l ends with the warp total of value (l % NV).
-template <int NV>
-__device__ __forceinline__ float reduce_scatter(float (&v)[32], int lane) {
-#pragma unroll
-  for (int o = 16; o >= 1; o >>= 1) {
-    if (o >= NV) {
-#pragma unroll
-      for (int k = 0; k < NV; ++k) v[k] += __shfl_xor_sync(0xffffffffu, v[k], o);
-    } else {
-      const bool up = lane & o;
-#pragma unroll
-      for (int k = 0; k < o; ++k) {
-        const float send = up ? v[k] : v[k + o];
-        const float keep = up ? v[k + o] : v[k];
-        v[k] = keep + __shfl_xor_sync(0xffffffffu, send, o);
-      }
-    }
-  }
-  return v[0];
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t (&r)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
 }
 
-// Partial dot products of one cached key (the lane's channels) with the
-// group's queries; remote keys are first turned by the correction rotation.
-template <int D, int GRP, bool REMOTE>
-__device__ __forceinline__ void token_partials(float (&part)[32], int slot0,
-                                               const __nv_bfloat16 *krow, const float2 *cs_row,
-                                               int lane, const float (&q)[GRP][D / 32]) {
-  constexpr int EPL = D / 32;
-  float kv[EPL];
-  load_row<D>(krow, lane, kv);
-  if constexpr (REMOTE) {
-    float2 cs[EPL / 2];
-    if constexpr (D == 128) {
-      const float4 c4 = *reinterpret_cast<const float4 *>(cs_row + 2 * lane);
-      cs[0] = make_float2(c4.x, c4.y);
-      cs[1] = make_float2(c4.z, c4.w);
-    } else {
-      cs[0] = cs_row[lane];
-    }
+// D(16x8, f32) += A(16x16) * B(16x8) with FP16 or BF16 operands (register fragments).
+__device__ __forceinline__ void mma_f16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                        uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+      "{%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ void mma_bf16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                         uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+      "{%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Pack (lo, hi) as f16x2 / bf16x2 (lo in the low half = lower index).
+__device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+__device__ __forceinline__ float bf_lo(uint32_t u) { return __uint_as_float(u << 16); }
+__device__ __forceinline__ float bf_hi(uint32_t u) { return __uint_as_float(u & 0xffff0000u); }
+
+// S (16 x 8, rows = the group's heads, columns = 8 tokens) += Q K^T over the
+// k-blocks [kb0, kb0 + 2) and their RoPE partners [kb0 + KB/2, kb0 + KB/2 + 2).
+// K is read with ldmatrix as FP16-converted B fragments; remote tokens are
+// first turned by the correction rotation (channel c pairs with c + D/2).
+template <int D, bool REMOTE>
+__device__ __forceinline__ void qk_pair(float (&sc)[4], const uint32_t (&q)[D / 16][2],
+                                        uint32_t krow_addr, const uint8_t *cs_row, int kb0,
+                                        int tq, int mat) {
+  constexpr int HK = D / 32;  // k-block offset of the RoPE partners
+  uint32_t lo[4], hi[4];      // k-blocks kb0, kb0 + 1 and their partners
+  ldsm_x4(krow_addr + (16 * kb0 + 8 * (mat & 1) + 16 * (mat >> 1)) * 2, lo);
+  ldsm_x4(krow_addr + (16 * (kb0 + HK) + 8 * (mat & 1) + 16 * (mat >> 1)) * 2, hi);
 #pragma unroll
-    for (int e = 0; e < EPL / 2; ++e) {
-      const float x = kv[e], y = kv[e + EPL / 2];
-      kv[e] = x * cs[e].x - y * cs[e].y;
-      kv[e + EPL / 2] = x * cs[e].y + y * cs[e].x;
+  for (int r = 0; r < 4; ++r) {
+    const float x0 = bf_lo(lo[r]), x1 = bf_hi(lo[r]);
+    const float y0 = bf_lo(hi[r]), y1 = bf_hi(hi[r]);
+    if constexpr (REMOTE) {
+      // lo[r]: channels c, c + 1 with c = 16 (kb0 + r / 2) + 8 (r % 2) + 2 tq
+      const int c = 16 * (kb0 + (r >> 1)) + 8 * (r & 1) + 2 * tq;
+      const float4 cs = *reinterpret_cast<const float4 *>(cs_row + c * 8);
+      lo[r] = pack_f16(x0 * cs.x - y0 * cs.y, x1 * cs.z - y1 * cs.w);
+      hi[r] = pack_f16(x0 * cs.y + y0 * cs.x, x1 * cs.w + y1 * cs.z);
+    } else {
+      lo[r] = pack_f16(x0, x1);
+      hi[r] = pack_f16(y0, y1);
     }
   }
+  mma_f16(sc, q[kb0][0], 0u, q[kb0][1], 0u, lo[0], lo[1]);
+  mma_f16(sc, q[kb0 + 1][0], 0u, q[kb0 + 1][1], 0u, lo[2], lo[3]);
+  mma_f16(sc, q[kb0 + HK][0], 0u, q[kb0 + HK][1], 0u, hi[0], hi[1]);
+  mma_f16(sc, q[kb0 + HK + 1][0], 0u, q[kb0 + HK + 1][1], 0u, hi[2], hi[3]);
+}
+
+template <int D, bool REMOTE>
+__device__ __forceinline__ void qk_block(float (&sc)[4], const uint32_t (&q)[D / 16][2],
+                                         uint32_t krow_addr, const uint8_t *cs_row, int tq,
+                                         int mat) {
+  // Two independent accumulator chains (k-block pairs alternate), summed at
+  // the end, so consecutive MMAs do not wait on each other.
+  float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
-  for (int h = 0; h < GRP; ++h) {
-    float d = q[h][0] * kv[0];
+  for (int kb0 = 0; kb0 < D / 32; kb0 += 2)
+    qk_pair<D, REMOTE>(acc[(kb0 >> 1) & 1], q, krow_addr, cs_row, kb0, tq, mat);
 #pragma unroll
-    for (int e = 1; e < EPL; ++e) d = fmaf(q[h][e], kv[e], d);
-    part[slot0 + h] = d;
+  for (int e = 0; e < 4; ++e) sc[e] += acc[0][e] + acc[1][e];
+}
+
+// Rows of the correction table of one stage: (cos, sin) of Delta j * theta_i
+// for token row tt (j = jt + tt) and frequency i < D/2, Delta j = f(j) - j.
+// The phase in turns is Delta j * omega_i modulo 1, with omega_i =
+// theta_i / (2 pi) as a 64-bit binary fraction: the 64-bit product wraps
+// exactly, its top 32 bits are the signed phase in units of 2^-32 turn, and
+// the angle handed to the sine/cosine lies in [-pi, pi).  Warp w writes rows
+// w, w + nw, ... of the stage.
+template <int D>
+__device__ __forceinline__ void correction_rows(uint8_t *tab, int jt, int n, int G, int warp,
+                                                int nw, int lane, const uint64_t *omega) {
+  using C = DecCfg<D>;
+  constexpr float kTurnToRad = 1.4629180792671596e-09f;  // 2 pi / 2^32
+  for (int tt = warp; tt < n; tt += nw) {
+    const int j = jt + tt;
+    const uint64_t delta = static_cast<uint64_t>(static_cast<int64_t>(remap(j, G) - j));
+#pragma unroll
+    for (int i = lane; i < D / 2; i += 32) {
+      const int32_t ph = static_cast<int32_t>((delta * omega[i]) >> 32);
+      float c, sn;
+      __sincosf(static_cast<float>(ph) * kTurnToRad, &sn, &c);
+      *reinterpret_cast<float2 *>(tab + tt * C::CS_ROW + i * 8) = make_float2(c, sn);
+    }
+  }
+}
+
+// Bounded mbarrier wait that also gives up once another warp raised `abort`.
+__device__ __forceinline__ bool dec_wait(uint32_t bar, uint32_t parity, volatile uint32_t *abort) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 63u) == 0u) {
+      if (*abort) return false;
+      if (global_timer_ns() - t0 > kWaitLimitNs) {
+        *abort = 1u;
+        return false;
+      }
+    }
   }
 }
 
@@ -146,265 +216,362 @@ template <int D, int GRP>
 __global__ void __launch_bounds__(kDecThreads, kCtasPerSm)
 decode_split_kernel(DecodeArgs a) {
   using C = DecCfg<D>;
-  constexpr int P = C::P, EPL = C::EPL, HALF = D / 2;
-  constexpr int NB = (32 / GRP) < P ? (32 / GRP) : P;  // tokens per score batch
-  constexpr int NV = NB * GRP;                         // values per batch: 8, 16 or 32
-  static_assert(NV == 8 || NV == 16 || NV == 32, "batch must fill 8, 16 or 32 values");
-  static_assert(P % NB == 0, "batches tile a stage");
+  constexpr int P = C::P, NBLK = C::NBLK, KB = C::KB, HALF = D / 2, MB = D / 16;
 
   extern __shared__ __align__(128) uint8_t dsm[];
   const uint32_t sb = smem_u32(dsm);
-  float2 *cs_tab = reinterpret_cast<float2 *>(dsm + C::CS);  // [P][D/2] (cos, sin)
+  volatile uint32_t *abort = reinterpret_cast<volatile uint32_t *>(dsm + C::ABORT);
+  auto full = [&](int slot) { return sb + C::BAR + 8u * static_cast<uint32_t>(slot); };
+  auto empty = [&](int slot) { return sb + C::BAR + 8u * static_cast<uint32_t>(kStages + slot); };
+  auto tready = [&](int slot) { return sb + C::BAR + 8u * static_cast<uint32_t>(2 * kStages + slot); };
 
   const int s = blockIdx.x, chunk_id = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g0 = chunk_id * kDecWarps;
-  const int nh = min(kDecWarps, a.Hkv - g0);  // KV heads of this CTA
-  const int g = g0 + warp;
-  const bool wactive = warp < nh;
+  const int nh = min(kDecWarps, a.Hkv - g0);  // KV heads of this CTA = working warps
   const int p = a.L - 1;
   const int G = a.G;
   const int w0eff = (G == 1) ? INT_MAX : a.w0;
   const int j_begin = s * a.chunk;
   const int j_end = min(a.L, j_begin + a.chunk);
   const int n_stage = (j_end - j_begin + P - 1) / P;
-  const uint32_t row_bytes = static_cast<uint32_t>(nh) * C::HEAD_BYTES;  // one token, CTA heads
-  const size_t cache_row = static_cast<size_t>(a.Hkv) * D;               // elements per token
+  const uint32_t head_bytes = static_cast<uint32_t>(nh) * D * 2;  // one token, CTA heads
+  const size_t cache_row = static_cast<size_t>(a.Hkv) * D;        // elements per token
 
-  if (tid == 0) {
-    for (int i = 0; i < kStages; ++i) mbar_init(sb + C::BAR + 8 * i, 1);
-    fence_mbar_init();
-  }
-  __syncthreads();
-
-  auto issue = [&](int t) {
-    const int slot = t % kStages;
-    const int jt = j_begin + t * P;
-    const int n = min(P, j_end - jt);
-    const uint32_t bar = sb + C::BAR + 8 * slot;
-    const uint32_t kdst = sb + slot * C::STAGE, vdst = kdst + C::STAGE_HALF;
-    mbar_arrive_expect_tx(bar, 2u * n * row_bytes);
-    const __nv_bfloat16 *ks = a.k_cache + (static_cast<size_t>(b) * a.Lcap + jt) * cache_row + g0 * D;
-    const __nv_bfloat16 *vs = a.v_cache + (static_cast<size_t>(b) * a.Lcap + jt) * cache_row + g0 * D;
-    if (nh == a.Hkv) {  // the CTA's rows of consecutive tokens are contiguous
-      bulk_copy(kdst, ks, n * row_bytes, bar);
-      bulk_copy(vdst, vs, n * row_bytes, bar);
-    } else {
-      for (int t2 = 0; t2 < n; ++t2) {
-        bulk_copy(kdst + t2 * row_bytes, ks + t2 * cache_row, row_bytes, bar);
-        bulk_copy(vdst + t2 * row_bytes, vs + t2 * cache_row, row_bytes, bar);
-      }
+  // RoPE frequencies as turns per position and the query's cos/sin at p and
+  // f(p), once per CTA.
+  uint64_t *omega = reinterpret_cast<uint64_t *>(dsm + C::OMEGA);
+  float2 *qcs = reinterpret_cast<float2 *>(dsm + C::QCS);
+  int n_issued = 0;  // warp 0: stages whose copies are posted
+  // One bulk copy per token and tensor into rows padded by 16 B (bank-conflict
+  // free ldmatrix), posted by warp 0: lane 0 adds the byte count, lanes
+  // [0, 2P) each issue one copy.  Slots past the chunk end repeat its last
+  // token, so every row the tensor core reads holds finite data; those tokens
+  // are masked.
+  auto issue = [&](int u) {  // warp 0, all lanes
+    ++n_issued;
+    const int slot = u % kStages;
+    const int ju = j_begin + u * P;
+    if (lane == 0) mbar_arrive_expect_tx(full(slot), 2u * P * head_bytes);
+    __syncwarp();
+    if (lane < 2 * P) {
+      const int t2 = lane >> 1;
+      const int j = min(ju + t2, j_end - 1);
+      const size_t off = (static_cast<size_t>(b) * a.Lcap + j) * cache_row + static_cast<size_t>(g0) * D;
+      const uint32_t dst = sb + slot * C::STAGE + (lane & 1) * C::HALF_STAGE + t2 * C::ROW;
+      bulk_copy(dst, ((lane & 1) ? a.v_cache : a.k_cache) + off, head_bytes, full(slot));
     }
   };
-  if (tid == 0)
-    for (int t = 0; t < kStages && t < n_stage; ++t) issue(t);
-
-  // Queries of this warp's heads at the true position p and the remote
-  // position f(p), for the lane's channels, pre-scaled by log2(e)/sqrt(D).
-  const double theta = static_cast<double>(a.theta);
-  const float qscale = kLog2e / sqrtf(static_cast<float>(D));
-  float qt[GRP][EPL], qr[GRP][EPL];
-  {
-    float ct[EPL / 2], st[EPL / 2], cr[EPL / 2], sr[EPL / 2];
-#pragma unroll
-    for (int e = 0; e < EPL / 2; ++e) {
-      const double fr = rope_freq(chan<D>(lane, e), D, theta);
-      rope_cos_sin(p, fr, ct[e], st[e]);
-      rope_cos_sin(remap(p, G), fr, cr[e], sr[e]);
+  // This warp's rows of the correction table of stage u (table u % kStages),
+  // then its arrival on that table's barrier; the table's previous user,
+  // stage u - kStages, must be done in every warp first.
+  auto table = [&](int u) -> bool {
+    if (u >= kStages) {
+      const bool got = dec_wait(empty(u % kStages), static_cast<uint32_t>(u / kStages - 1) & 1u, abort);
+      if (!__all_sync(0xffffffffu, got)) return false;
     }
-#pragma unroll
-    for (int h = 0; h < GRP; ++h) {
-      const int hq = (wactive ? g : g0) * GRP + h;
-      const __nv_bfloat16 *qrow = a.q + (static_cast<size_t>(b) * a.Hq + hq) * D;
-#pragma unroll
-      for (int e = 0; e < EPL / 2; ++e) {
-        const float x = bf2f(qrow[chan<D>(lane, e)]), y = bf2f(qrow[chan<D>(lane, e) + HALF]);
-        qt[h][e] = (x * ct[e] - y * st[e]) * qscale;
-        qt[h][e + EPL / 2] = (x * st[e] + y * ct[e]) * qscale;
-        qr[h][e] = (x * cr[e] - y * sr[e]) * qscale;
-        qr[h][e + EPL / 2] = (x * sr[e] + y * cr[e]) * qscale;
+    const int ju = j_begin + u * P;
+    if (p - ju > w0eff)
+      correction_rows<D>(dsm + C::CS + (u % kStages) * C::CS_TAB, ju, min(P, j_end - ju), G, warp, nh,
+                         lane, omega);
+    __syncwarp();
+    if (lane == 0) mbar_arrive(tready(u % kStages));
+    return true;
+  };
+  if (warp == 0) {
+    if (lane == 0) {
+      for (int i = 0; i < kStages; ++i) {
+        mbar_init(full(i), 1);    // copies posted, completes when their bytes land
+        mbar_init(empty(i), nh);  // one arrival per working warp
       }
+      for (int i = 0; i < kStages; ++i) mbar_init(tready(i), nh);  // table rows written
+      *abort = 0u;
+      fence_mbar_init();
     }
+    __syncwarp();
+    // The first copies go out before the RoPE tables are computed.
+    for (int u = 0; u < kStages && u < n_stage; ++u) issue(u);
+  }
+  for (int i = tid; i < HALF; i += kDecThreads)
+    omega[i] = __double2ull_rn(rope_freq(i, D, static_cast<double>(a.theta)) *
+                               (0.15915494309189533577 * 18446744073709551616.0));
+  for (int idx = tid; idx < 2 * HALF; idx += kDecThreads) {
+    const int i = idx < HALF ? idx : idx - HALF;
+    float c, sn;
+    rope_cos_sin(idx < HALF ? p : remap(p, G), rope_freq(i, D, static_cast<double>(a.theta)), c, sn);
+    qcs[idx] = make_float2(c, sn);
+  }
+  __syncthreads();
+  if (warp >= nh) return;  // no KV head for this warp; nothing below waits for it
+  bool ok = table(0);
+  if (ok && n_stage > 1) ok = table(1);
+
+  // Query fragments (A operand, rows = the group's heads, FP16, pre-scaled by
+  // log2(e)/sqrt(D)) at the true position p and the remote position f(p).
+  // Row gq holds query head gq of the group; rows >= GRP (and 8..15) are zero.
+  const int gq = lane >> 2, tq = lane & 3;     // mma fragment coordinates
+  const int mat = lane >> 3, mrow = lane & 7;  // ldmatrix: matrix and row this lane addresses
+  const int g = g0 + warp;
+  const float qscale = kLog2e / sqrtf(static_cast<float>(D));
+  uint32_t qt[KB][2], qr[KB][2];
+  {
+    const bool qrow_ok = gq < GRP;
+    const __nv_bfloat16 *qrow = a.q + (static_cast<size_t>(b) * a.Hq + g * GRP + (qrow_ok ? gq : 0)) * D;
+#pragma unroll
+    for (int kb = 0; kb < KB / 2; ++kb)
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        float vt[2][2], vr[2][2];  // [first / partner][channel c0, c0 + 1]
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int c = 16 * kb + 2 * tq + 8 * h + e;  // first member, < D/2
+          const float x = qrow_ok ? bf2f(qrow[c]) : 0.f;
+          const float y = qrow_ok ? bf2f(qrow[c + HALF]) : 0.f;
+          const float2 ct = qcs[c], cr = qcs[HALF + c];
+          vt[0][e] = (x * ct.x - y * ct.y) * qscale;
+          vt[1][e] = (x * ct.y + y * ct.x) * qscale;
+          vr[0][e] = (x * cr.x - y * cr.y) * qscale;
+          vr[1][e] = (x * cr.y + y * cr.x) * qscale;
+        }
+        qt[kb][h] = pack_f16(vt[0][0], vt[0][1]);
+        qt[kb + KB / 2][h] = pack_f16(vt[1][0], vt[1][1]);
+        qr[kb][h] = pack_f16(vr[0][0], vr[0][1]);
+        qr[kb + KB / 2][h] = pack_f16(vr[1][0], vr[1][1]);
+      }
   }
 
-  float acc[GRP][EPL];
+  // O^T accumulators: m-block mb holds (channel 16mb + gq, heads 2tq, 2tq+1)
+  // in o[mb][0..1] and channel 16mb + gq + 8 in o[mb][2..3].
+  float o[MB][4];
 #pragma unroll
-  for (int h = 0; h < GRP; ++h)
+  for (int mb = 0; mb < MB; ++mb)
 #pragma unroll
-    for (int e = 0; e < EPL; ++e) acc[h][e] = 0.f;
-  float m_mine = -INFINITY, l_mine = 0.f;  // state of head (lane % GRP)
+    for (int e = 0; e < 4; ++e) o[mb][e] = 0.f;
+  float m_run = -INFINITY;  // running max (base 2) of head gq, same in its 4 lanes
+  float l_part = 0.f;       // this lane's share of head gq's running sum
+  const uint32_t warp_col = static_cast<uint32_t>(warp) * D * 2;
 
-  bool ok = true;
-  int t_fail = 0;
-  for (int t = 0; t < n_stage; ++t) {
-    const int slot = t % kStages;
+  int slot = 0;
+  uint32_t phase = 0;
+  for (int t = 0; t < n_stage && ok; ++t) {
     const int jt = j_begin + t * P;
     const int n = min(P, j_end - jt);
-    // cos/sin of the correction angles of this stage's remote tokens
-    if (p - jt > w0eff) {
-      for (int idx = tid; idx < n * HALF; idx += kDecThreads) {
-        const int tt = idx / HALF, i = idx - tt * HALF;
-        const int j = jt + tt;
-        float c = 1.f, sn = 0.f;
-        if (p - j > w0eff) {
-          const double ang = static_cast<double>(remap(j, G) - j) *
-                             rope_freq(i, D, theta);  // Delta j * theta_i
-          const double r = ang - rint(ang * 0.15915494309189533577) * 6.283185307179586232;
-          __sincosf(static_cast<float>(r), &sn, &c);
-        }
-        cs_tab[tt * HALF + i] = make_float2(c, sn);
-      }
-    }
-    const uint32_t bar = sb + C::BAR + 8 * slot;
-    ok = mbar_wait_bounded(bar, static_cast<uint32_t>(t / kStages) & 1u, kWaitLimitNs);
-    if (__syncthreads_or(!ok)) {
+    ok = dec_wait(full(slot), phase, abort) && dec_wait(tready(slot), phase, abort);
+    if (!__all_sync(0xffffffffu, ok)) {
       ok = false;
-      t_fail = t;
       break;
     }
-    if (wactive) {
-      const uint8_t *kst = dsm + slot * C::STAGE + warp * C::HEAD_BYTES;
-      const uint8_t *vst = kst + C::STAGE_HALF;
-#pragma unroll 1
-      for (int tb = 0; tb < n; tb += NB) {
-        // partial scores of NB tokens x GRP heads; the query variant is
-        // chosen per batch (all remote / all local), per token only on the
-        // batch that straddles the window edge
-        float part[32];
+    {
+      const uint32_t kst = sb + slot * C::STAGE + warp_col;
+      const uint32_t vst = kst + C::HALF_STAGE;
+      const uint8_t *tab = dsm + C::CS + slot * C::CS_TAB;
+      uint32_t pfrag[NBLK];  // P^T fragments (BF16), one per 8-token block
 #pragma unroll
-        for (int k = 0; k < 32; ++k) part[k] = 0.f;
-        const int nb = min(NB, n - tb);
+      for (int nb = 0; nb < NBLK; ++nb) {
+        const int tb = nb * 8;
+        const uint32_t krow = kst + (tb + mrow) * C::ROW;
+        const uint8_t *cs_row = tab + (tb + gq) * C::CS_ROW;  // this lane's token gq
         const int jb = jt + tb;
-        const bool all_remote = p - (jb + nb - 1) > w0eff;
+        const int nb_valid = min(8, n - tb);
+        const bool all_remote = p - (jb + 7) > w0eff;
         const bool all_local = p - jb <= w0eff;
-        auto krow = [&](int pb) {
-          return reinterpret_cast<const __nv_bfloat16 *>(kst + (tb + pb) * row_bytes);
-        };
+        float sc[4] = {0.f, 0.f, 0.f, 0.f};
         if (all_remote) {
-#pragma unroll
-          for (int pb = 0; pb < NB; ++pb)
-            if (pb < nb)
-              token_partials<D, GRP, true>(part, pb * GRP, krow(pb), cs_tab + (tb + pb) * HALF, lane, qr);
+          qk_block<D, true>(sc, qr, krow, cs_row, tq, mat);
         } else if (all_local) {
-#pragma unroll
-          for (int pb = 0; pb < NB; ++pb)
-            if (pb < nb)
-              token_partials<D, GRP, false>(part, pb * GRP, krow(pb), cs_tab, lane, qt);
-        } else {
-#pragma unroll
-          for (int pb = 0; pb < NB; ++pb)
-            if (pb < nb) {
-              if (p - (jb + pb) > w0eff)
-                token_partials<D, GRP, true>(part, pb * GRP, krow(pb), cs_tab + (tb + pb) * HALF, lane, qr);
-              else
-                token_partials<D, GRP, false>(part, pb * GRP, krow(pb), cs_tab, lane, qt);
-            }
+          qk_block<D, false>(sc, qt, krow, cs_row, tq, mat);
+        } else {  // the block on the window edge: both variants, picked per token
+          float sl[4] = {0.f, 0.f, 0.f, 0.f};
+          qk_block<D, true>(sc, qr, krow, cs_row, tq, mat);
+          qk_block<D, false>(sl, qt, krow, cs_row, tq, mat);
+          if (p - (jb + 2 * tq) <= w0eff) sc[0] = sl[0];
+          if (p - (jb + 2 * tq + 1) <= w0eff) sc[1] = sl[1];
         }
-        const float sc = reduce_scatter<NV>(part, lane);
-        const int my_pb = (lane % NV) / GRP;
-        const float sv = my_pb < nb ? sc : -INFINITY;
-        // online softmax for head (lane % GRP) over the batch
-        float bm = sv;
-#pragma unroll
-        for (int o = GRP; o < NV; o <<= 1) bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, o));
-        const float m_new = fmaxf(m_mine, bm);  // finite: the batch holds a valid token
-        const float alpha_mine = exp2f(m_mine - m_new);
-        const float pm = exp2f(sv - m_new);
-        float ps = pm;
-#pragma unroll
-        for (int o = GRP; o < NV; o <<= 1) ps += __shfl_xor_sync(0xffffffffu, ps, o);
-        l_mine = l_mine * alpha_mine + ps;
-        m_mine = m_new;
-#pragma unroll
-        for (int h = 0; h < GRP; ++h) {
-          const float al = __shfl_sync(0xffffffffu, alpha_mine, h);
-#pragma unroll
-          for (int e = 0; e < EPL; ++e) acc[h][e] *= al;
+        // scores of head gq for tokens tb + 2tq, tb + 2tq + 1
+        const float s0 = 2 * tq < nb_valid ? sc[0] : -INFINITY;
+        const float s1 = 2 * tq + 1 < nb_valid ? sc[1] : -INFINITY;
+        float bm = fmaxf(s0, s1);
+        bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 1));
+        bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 2));
+        // lazy online softmax: the reference max moves only when it grows by
+        // more than 2^8 (O and l share it, so the result is exact)
+        float alpha = 1.f;
+        if (bm > m_run + kRescaleThreshold || (m_run == -INFINITY && bm > -INFINITY)) {
+          if (m_run != -INFINITY) alpha = exp2f(m_run - bm);
+          m_run = bm;
         }
+        if (__any_sync(0xffffffffu, alpha != 1.f)) {
+          // O^T columns are heads 2tq, 2tq+1; their factors live in lanes 4*head
+          const float a0 = __shfl_sync(0xffffffffu, alpha, (2 * tq) * 4);
+          const float a1 = __shfl_sync(0xffffffffu, alpha, (2 * tq + 1) * 4);
 #pragma unroll
-        for (int pb = 0; pb < NB; ++pb) {
-          if (pb < nb) {
-            float vv[EPL];
-            load_row<D>(reinterpret_cast<const __nv_bfloat16 *>(vst + (tb + pb) * row_bytes), lane, vv);
-#pragma unroll
-            for (int h = 0; h < GRP; ++h) {
-              const float pr = __shfl_sync(0xffffffffu, pm, pb * GRP + h);
-#pragma unroll
-              for (int e = 0; e < EPL; ++e) acc[h][e] = fmaf(pr, vv[e], acc[h][e]);
-            }
+          for (int mb = 0; mb < MB; ++mb) {
+            o[mb][0] *= a0;
+            o[mb][1] *= a1;
+            o[mb][2] *= a0;
+            o[mb][3] *= a1;
           }
+          l_part *= alpha;
+        }
+        const float neg_m = m_run == -INFINITY ? 0.f : -m_run;
+        const float p0 = ex2_sfu(s0 + neg_m), p1 = ex2_sfu(s1 + neg_m);
+        l_part += p0 + p1;
+        pfrag[nb] = pack_bf16(p0, p1);
+      }
+      // O^T += V^T P^T over this stage's tokens (k = 16 tokens; with 8-token
+      // stages the upper half of P is zero and V's rows are reused)
+      const uint32_t pb0 = pfrag[0], pb1 = NBLK > 1 ? pfrag[NBLK - 1] : 0u;
+#pragma unroll
+      for (int mb = 0; mb < MB; mb += 2) {
+        uint32_t lo[4];
+        ldsm_x4_t(vst + mrow * C::ROW + (16 * mb + 8 * (mat & 1) + 16 * (mat >> 1)) * 2, lo);
+        if constexpr (NBLK > 1) {
+          uint32_t hi[4];
+          ldsm_x4_t(vst + (8 + mrow) * C::ROW + (16 * mb + 8 * (mat & 1) + 16 * (mat >> 1)) * 2, hi);
+          mma_bf16(o[mb], lo[0], lo[1], hi[0], hi[1], pb0, pb1);
+          mma_bf16(o[mb + 1], lo[2], lo[3], hi[2], hi[3], pb0, pb1);
+        } else {
+          mma_bf16(o[mb], lo[0], lo[1], lo[0], lo[1], pb0, pb1);
+          mma_bf16(o[mb + 1], lo[2], lo[3], lo[2], lo[3], pb0, pb1);
         }
       }
     }
-    __syncthreads();  // stage slot and cos/sin table free again
-    if (tid == 0 && t + kStages < n_stage) issue(t + kStages);
+    __syncwarp();
+    if (lane == 0) mbar_arrive(empty(slot));
+    // This warp's rows of the table two stages ahead.
+    if (t + 2 < n_stage) ok = table(t + 2);
+    // Warp 0 refills this slot once every warp has released it.
+    if (warp == 0 && ok && t + kStages < n_stage) {
+      ok = __all_sync(0xffffffffu, dec_wait(empty(slot), phase, abort));
+      if (ok) issue(t + kStages);
+    }
+    if (++slot == kStages) {
+      slot = 0;
+      phase ^= 1u;
+    }
   }
-  if (!ok) {
-    // Stages t_fail .. t_fail + kStages - 1 may still be in flight: let them
-    // land (bounded) before the CTA exits, then report.
-    if (tid == 0) {
-      for (int u = t_fail; u < n_stage && u < t_fail + kStages; ++u)
-        mbar_wait_bounded(sb + C::BAR + 8 * (u % kStages), static_cast<uint32_t>(u / kStages) & 1u,
-                          kWaitLimitNs);
+  if (!ok || *abort) {
+    // This warp stops.  Warp 0 first lets the copies it posted land
+    // (bounded), so none writes into shared memory after the CTA exits: only
+    // the last kStages stages it issued can be in flight, since a slot is
+    // refilled only after every warp consumed its previous stage.
+    if (lane == 0) {
+      *abort = 1u;
       atomicOr(a.dev_error, kDevTimeout);
     }
+    if (warp == 0 && lane == 0)
+      for (int u = max(0, n_issued - kStages); u < n_issued; ++u)
+        mbar_wait_bounded(full(u % kStages), static_cast<uint32_t>(u / kStages) & 1u, 2000000ull);
     return;
   }
-  if (!wactive) return;
-  // Partial record: [D] unnormalised output, then the running max (base 2) and sum.
+  // Row sums: the four lanes of head gq hold its shares.
+  float l_run = l_part + __shfl_xor_sync(0xffffffffu, l_part, 1);
+  l_run += __shfl_xor_sync(0xffffffffu, l_run, 2);
+  // Partial record per query head: [D] unnormalised output, then the running
+  // max (base 2) and sum.
+  const size_t rec_stride = static_cast<size_t>(a.n_split) * (D + 2);
+  float *rec0 = a.partial + ((static_cast<size_t>(b) * a.Hq + g * GRP) * a.n_split + s) * (D + 2);
 #pragma unroll
-  for (int h = 0; h < GRP; ++h) {
-    float *rec = a.partial +
-                 ((static_cast<size_t>(b) * a.Hq + g * GRP + h) * a.n_split + s) * (D + 2);
+  for (int e = 0; e < 2; ++e) {
+    const int h = 2 * tq + e;  // O^T column = query head of the group
+    if (h < GRP) {
+      float *rec = rec0 + h * rec_stride;
 #pragma unroll
-    for (int e = 0; e < EPL; ++e) rec[chan<D>(lane, e)] = acc[h][e];
+      for (int mb = 0; mb < MB; ++mb) {
+        rec[16 * mb + gq] = o[mb][e];
+        rec[16 * mb + gq + 8] = o[mb][2 + e];
+      }
+    }
   }
-  if (lane < GRP) {
-    float *rec = a.partial +
-                 ((static_cast<size_t>(b) * a.Hq + g * GRP + lane) * a.n_split + s) * (D + 2);
-    rec[D] = m_mine;
-    rec[D + 1] = l_mine;
+  if (tq == 0 && gq < GRP) {
+    float *rec = rec0 + gq * rec_stride;
+    rec[D] = m_run;
+    rec[D + 1] = l_run;
   }
 }
 
-// Merge the split partials of one (b, head): one warp per head.
+// Merge the split partials of one (b, head), one CTA of 8 warps per head:
+// block-wide max of the split maxima, the weights 2^(m_s - M) kept in shared
+// memory, then each warp accumulates every 8th split (lanes over channel
+// pairs) and the 8 warp sums are added.  Launched as a programmatic dependent
+// of the split kernel: the wait below returns once that grid has finished and
+// its partials are visible.
+constexpr int kCombineThreads = 256;
+constexpr int kMaxSplit = kCtasPerSm * 148;  // decode_plan never exceeds this
+
 template <int D>
-__global__ void __launch_bounds__(128)
+__global__ void __launch_bounds__(kCombineThreads)
 decode_combine_kernel(DecodeArgs a) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int bh = blockIdx.x * 4 + warp;
-  if (bh >= a.B * a.Hq) return;
-  const float *rec = a.partial + static_cast<size_t>(bh) * a.n_split * (D + 2);
-  float M = -INFINITY;
-  for (int s = lane; s < a.n_split; s += 32) M = fmaxf(M, rec[s * (D + 2) + D]);
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  constexpr int NW = kCombineThreads / 32;
+  constexpr int PAIRS = D / 64;  // float2 channel pairs per lane
+  __shared__ float wsh[kMaxSplit];
+  __shared__ float red[NW][D];
+  __shared__ float part[NW];
+  const int bh = blockIdx.x;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int ns = a.n_split;
+  const float *rec = a.partial + static_cast<size_t>(bh) * ns * (D + 2);
+
+  float m = -INFINITY;
+  for (int s = tid; s < ns; s += kCombineThreads) m = fmaxf(m, rec[s * (D + 2) + D]);
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-  float lsum = 0.f;
-  for (int s = lane; s < a.n_split; s += 32) {
-    const float m = rec[s * (D + 2) + D];
-    lsum += rec[s * (D + 2) + D + 1] * exp2f(m - M);
-  }
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if (lane == 0) part[warp] = m;
+  __syncthreads();
+  float M = part[0];
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) lsum += __shfl_xor_sync(0xffffffffu, lsum, o);
-  constexpr int PER = D / 32;
-  float o_acc[PER];
-#pragma unroll
-  for (int e = 0; e < PER; ++e) o_acc[e] = 0.f;
-  for (int s = 0; s < a.n_split; ++s) {
+  for (int w = 1; w < NW; ++w) M = fmaxf(M, part[w]);
+  __syncthreads();  // part[] is reused below
+
+  float l = 0.f;
+  for (int s = tid; s < ns; s += kCombineThreads) {
     const float w = exp2f(rec[s * (D + 2) + D] - M);
-#pragma unroll
-    for (int e = 0; e < PER; ++e) o_acc[e] = fmaf(w, rec[s * (D + 2) + lane + 32 * e], o_acc[e]);
+    wsh[s] = w;
+    l = fmaf(rec[s * (D + 2) + D + 1], w, l);
   }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
+  if (lane == 0) part[warp] = l;
+  __syncthreads();
+  float lsum = 0.f;
+#pragma unroll
+  for (int w = 0; w < NW; ++w) lsum += part[w];
+
+  float2 acc[PAIRS];
+#pragma unroll
+  for (int e = 0; e < PAIRS; ++e) acc[e] = make_float2(0.f, 0.f);
+  if (lane < D / 2) {  // D = 64: lanes 0..31 hold one pair each
+#pragma unroll 4
+    for (int s = warp; s < ns; s += NW) {
+      const float w = wsh[s];
+      const float2 *r2 = reinterpret_cast<const float2 *>(rec + static_cast<size_t>(s) * (D + 2));
+#pragma unroll
+      for (int e = 0; e < PAIRS; ++e) {
+        const float2 v = r2[lane + 32 * e];
+        acc[e].x = fmaf(w, v.x, acc[e].x);
+        acc[e].y = fmaf(w, v.y, acc[e].y);
+      }
+    }
+#pragma unroll
+    for (int e = 0; e < PAIRS; ++e) {
+      red[warp][2 * (lane + 32 * e)] = acc[e].x;
+      red[warp][2 * (lane + 32 * e) + 1] = acc[e].y;
+    }
+  }
+  __syncthreads();
   const float inv = 1.f / lsum;
+  for (int c = tid; c < D; c += kCombineThreads) {
+    float o = 0.f;
 #pragma unroll
-  for (int e = 0; e < PER; ++e) {
-    const size_t idx = static_cast<size_t>(bh) * D + lane + 32 * e;
+    for (int w = 0; w < NW; ++w) o += red[w][c];
+    const size_t idx = static_cast<size_t>(bh) * D + c;
     if (a.out_f32)
-      reinterpret_cast<float *>(a.out)[idx] = o_acc[e] * inv;
+      reinterpret_cast<float *>(a.out)[idx] = o * inv;
     else
-      reinterpret_cast<__nv_bfloat16 *>(a.out)[idx] = __float2bfloat16_rn(o_acc[e] * inv);
+      reinterpret_cast<__nv_bfloat16 *>(a.out)[idx] = __float2bfloat16_rn(o * inv);
   }
-  if (lane == 0 && a.lse) a.lse[bh] = (M + log2f(lsum)) * 0.69314718055994531f;
+  if (tid == 0 && a.lse) a.lse[bh] = (M + log2f(lsum)) * 0.69314718055994531f;
 }
 
 template <int D, int GRP>
@@ -429,9 +596,18 @@ cudaError_t launch_decode_d(const DecodeArgs &a, cudaStream_t stream) {
     default: return cudaErrorInvalidValue;
   }
   if (e != cudaSuccess) return e;
-  const int nbh = a.B * a.Hq;
-  decode_combine_kernel<D><<<(nbh + 3) / 4, 128, 0, stream>>>(a);
-  return cudaGetLastError();
+  if (a.n_split > kMaxSplit) return cudaErrorInvalidValue;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(a.B * a.Hq));
+  cfg.blockDim = dim3(kCombineThreads);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, decode_combine_kernel<D>, a);
 }
 
 }  // namespace

@@ -25,6 +25,7 @@ def main(argv=None) -> int:
     ap.add_argument("--workload", default=None)
     ap.add_argument("--L", type=int, default=None)
     ap.add_argument("--w0", type=int, default=None)
+    ap.add_argument("--w-pretrained", type=int, default=None)
     ap.add_argument("--reps", type=int, default=3)
     args = ap.parse_args(argv)
     name = args.workload or ("qwen3_8b_64k" if args.case == "prefill" else "decode_8b_32k")
@@ -33,6 +34,8 @@ def main(argv=None) -> int:
         w = w.with_(L=args.L)
     if args.w0 is not None:
         w = w.with_(w0=args.w0)
+    if args.w_pretrained is not None:
+        w = w.with_(w_pretrained=args.w_pretrained)
     dev = torch.device("cuda", 0)
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if args.case == "prefill":
@@ -65,7 +68,8 @@ def main(argv=None) -> int:
     ev1.record()
     torch.cuda.synchronize()
     st = jl.jetlong_device_status()
-    print(f"{args.case} {name} L={w.L}: {ev0.elapsed_time(ev1) / args.reps:.3f} ms/rep, "
+    print(f"{args.case} {name} L={w.L} w_pretrained={w.w_pretrained} w0={w.w0}: "
+          f"{ev0.elapsed_time(ev1) / args.reps:.3f} ms/rep, "
           f"status {st}")
     return 0 if st == jl.JL_OK else 1
 
