@@ -11,6 +11,11 @@ kernel (jetlong_prefill_attend), with inputs resident in HBM.  The headline
 After the prefill steps, 256 decode steps on a 131072-token true-position
 cache (Qwen3-8B shapes) are timed the same way and reported as microseconds
 per token and achieved HBM bandwidth over the K+V bytes a step must read.
+Both are also timed as a matched control -- the same kernels with the
+bifocal rule off (w_pretrained = L, so G = 1: plain causal RoPE attention at
+true positions) -- and the ratio is reported as the routing cost.  The
+prefill is also timed in its unfused three-pass form (jetlong_prefill_three_pass)
+to report what fusion saves.
 
 Every input is synthetic and seeded (zero_shot_rope_bifocal_b200.synth);
 each is larger than the 126 MB L2 (q alone is 1 GiB), so no flush is needed
@@ -297,6 +302,55 @@ def run_native(args):
     if jl.jetlong_device_status() != jl.JL_OK:
         raise RuntimeError("device status not OK after timing")
     t_max = reduce_max(t_ms, world, dev)
+
+    # ---- matched control: the same kernels with the bifocal rule off
+    # (w_pretrained = L, so G = 1: plain causal RoPE at true positions), on the
+    # same inputs; it prices the routing (remote visits, edge tiles, rotation).
+    def ctl_step(ev_mid=None, ev_end=None):
+        jl.jetlong_prefill_rotate(x.q, x.k, x.v, L, w.theta, ws, stream=stream)
+        if ev_mid is not None:
+            ev_mid.record(stream)
+        jl.jetlong_prefill_attend(out, lse, Hkv, L, w.w0, ws, stream=stream)
+        if ev_end is not None:
+            ev_end.record(stream)
+
+    ctl_step()
+    n_ctl = max(1, min(args.steps, 3))
+    barrier()
+    torch.cuda.synchronize(dev)
+    ev0.record(stream)
+    for s in range(n_ctl):
+        ctl_step(mids[s], ends[s])
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    ctl_step_ms = reduce_max(ev0.elapsed_time(ev1), world, dev) / n_ctl
+    ctl_attn_ms = sum(mids[s].elapsed_time(ends[s]) for s in range(n_ctl)) / n_ctl
+    if jl.jetlong_device_status() != jl.JL_OK:
+        raise RuntimeError("device status not OK after the control prefill")
+
+    # ---- the unfused three-pass form (A + B - C merge) on the same inputs:
+    # what fusing the passes into one kernel saves
+    ws3 = torch.empty(jl.jetlong_prefill_three_pass_workspace_size(B, Hq, Hkv, L, D),
+                      dtype=torch.uint8, device=dev)
+
+    def three_step():
+        jl.jetlong_prefill_three_pass(x.q, x.k, x.v, w.w_pretrained, w.w0, w.theta, out=out,
+                                      lse=lse, workspace=ws3, stream=stream)
+
+    three_step()
+    barrier()
+    torch.cuda.synchronize(dev)
+    ev0.record(stream)
+    for _ in range(n_ctl):
+        three_step()
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    three_ms = reduce_max(ev0.elapsed_time(ev1), world, dev) / n_ctl
+    del ws3
+    if jl.jetlong_device_status() != jl.JL_OK:
+        raise RuntimeError("device status not OK after the three-pass prefill")
     flops_rank = prefill_flops(B, Hq, L, D) * args.steps
     flops_all = reduce_sum(flops_rank, world, dev)
     value = flops_all / (t_max * 1e-3) / 1e12
@@ -339,6 +393,25 @@ def run_native(args):
         raise RuntimeError("device status not OK after decode timing")
     us_tok = 1e3 * dec_ms / n_dec
     dec_gbs = decode_bytes(wd.B, wd.Hkv, wd.L, wd.D) / (us_tok * 1e-6) / 1e9
+
+    # matched control decode (G = 1: every key local, no correction rotation)
+    def dstep_ctl():
+        jl.jetlong_decode(dq, kc, d.v, wd.L, wd.L, wd.w0, wd.theta, out=dout, lse=dlse,
+                          workspace=dws, stream=stream)
+
+    for _ in range(3):
+        dstep_ctl()
+    barrier()
+    torch.cuda.synchronize(dev)
+    ev0.record(stream)
+    for _ in range(n_loop):
+        dstep_ctl()
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    ctl_us_tok = 1e3 * reduce_max(ev0.elapsed_time(ev1), world, dev) / n_loop
+    if jl.jetlong_device_status() != jl.JL_OK:
+        raise RuntimeError("device status not OK after the control decode")
 
     # ---- end to end through the public API from pinned host buffers
     hq = x.q.cpu().pin_memory()
@@ -411,9 +484,24 @@ def run_native(args):
                        "nominal_frac": dec_gbs / NOMINAL["hbm_gbs"],
                        "bytes_per_token": decode_bytes(wd.B, wd.Hkv, wd.L, wd.D),
                        "clocks": dclocks.summary()},
+            "control": {
+                "what": "same kernels, bifocal rule off (w_pretrained = L, G = 1): plain causal "
+                        "RoPE attention at true positions, same inputs",
+                "prefill_attend_ms": ctl_attn_ms,
+                "prefill_attend_tflops": prefill_flops(B, Hq, L, D) / (ctl_attn_ms * 1e-3) / 1e12,
+                "prefill_step_ms": ctl_step_ms,
+                "routing_cost_prefill": attn_ms / ctl_attn_ms - 1.0,
+                "decode_us_per_token": ctl_us_tok,
+                "routing_cost_decode": us_tok / ctl_us_tok - 1.0},
+            "three_pass": {
+                "what": "unfused inclusion-exclusion form: rotate + passes A (remote, causal), "
+                        "B (true, band), C (remote, band) + merge kernel, same inputs",
+                "ms_per_step": three_ms,
+                "tflops": prefill_flops(B, Hq, L, D) / (three_ms * 1e-3) / 1e12,
+                "fused_speedup": three_ms / (t_max / args.steps)},
             "e2e": {"value": e2e_val, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
-            "gpu_launches": 2 * args.steps + 2 * n_dec,
+            "gpu_launches": 2 * args.steps + 2 * n_dec,  # timed regions: 2 per prefill step, 2 per decode
             "clocks": clocks.summary(),
             "cpu_baseline": cpu,
         }

@@ -152,6 +152,33 @@ JL_API int jetlong_prefill_attend(void *out, float *lse, int B, int Hq, int Hkv,
                                   size_t workspace_bytes, jl_stream_t stream);
 
 /*
+ * The unfused three-pass form of the same result (Jet-Long paper, §3.3
+ * "Inclusion-exclusion merge"), kept as a cross-check of the fused kernel
+ * and to measure what fusion saves.  Three attention passes over the
+ * operands of jetlong_prefill_rotate:
+ *   A: remote positions f(i), f(j) on every causal pair j <= i;
+ *   B: true positions i, j on the band 0 <= i - j <= w0;
+ *   C: remote positions on the same band;
+ * each writing an fp32 output and lse into the workspace, then
+ *   out = (W_A O_A + W_B O_B - W_C O_C) / (W_A + W_B - W_C),  W_X = exp(lse_X),
+ *   lse = log(W_A + W_B - W_C).
+ * The band passes use w0 even when G = 1 (then B and C coincide and cancel).
+ * Arguments and layouts as for jetlong_prefill (no cache output);
+ * workspace: at least jetlong_prefill_three_pass_workspace_size(...) bytes,
+ * 256-byte aligned (the prefill operands plus 3 fp32 outputs and 3 lse rows).
+ * Precision: the subtraction loses accuracy where the band holds most of a
+ * row's softmax mass under remote positions; the fused path has no
+ * subtraction.  Returns JL_OK or an error code (nothing launched on error).
+ */
+JL_API size_t jetlong_prefill_three_pass_workspace_size(int B, int Hq, int Hkv, int L, int D);
+
+JL_API int jetlong_prefill_three_pass(const void *q, const void *k, const void *v, void *out,
+                                      float *lse, int B, int Hq, int Hkv, int L, int D,
+                                      int w_pretrained, int w0, float rope_theta, int out_dtype,
+                                      void *workspace, size_t workspace_bytes,
+                                      jl_stream_t stream);
+
+/*
  * Bytes of workspace jetlong_decode needs for a cache of L tokens (host only).
  * Non-decreasing in L: sizing it for the largest L a generation loop will reach
  * covers every earlier step.  Returns 0 if a size is invalid.

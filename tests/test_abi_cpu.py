@@ -108,6 +108,39 @@ def test_prefill_rejects_bad_arguments(lib, kw, status):
     assert prefill_call(lib, **kw) == status
 
 
+def three_pass_call(lib, **kw):
+    a = dict(q=P, k=P, v=P, out=P, lse=None, B=1, Hq=2, Hkv=1, L=512, D=64, wp=128, w0=32,
+             theta=1e4, od=0, ws=P, wsb=1 << 40, stream=None)
+    a.update(kw)
+    return lib.jetlong_prefill_three_pass(a["q"], a["k"], a["v"], a["out"], a["lse"], a["B"],
+                                          a["Hq"], a["Hkv"], a["L"], a["D"], a["wp"], a["w0"],
+                                          a["theta"], a["od"], a["ws"], a["wsb"], a["stream"])
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(v=None), jl.JL_ERR_NULL),
+    (dict(Hq=3, Hkv=2), jl.JL_ERR_SHAPE),
+    (dict(D=32), jl.JL_ERR_UNSUPPORTED),
+    (dict(w0=-1), jl.JL_ERR_SHAPE),
+    (dict(od=7), jl.JL_ERR_UNSUPPORTED),
+    (dict(out=ctypes.c_void_p(264)), jl.JL_ERR_ALIGN),
+    (dict(ws=None), jl.JL_ERR_WORKSPACE),
+])
+def test_three_pass_rejects_bad_arguments(lib, kw, status):
+    assert three_pass_call(lib, **kw) == status
+
+
+def test_three_pass_needs_room_for_the_pass_outputs(lib):
+    # Enough for the fused prefill's operands but not for the three fp32 pass
+    # outputs and lse rows.
+    B, Hq, Hkv, L, D = 1, 2, 1, 512, 64
+    fused = jl.jetlong_prefill_workspace_size(B, Hq, Hkv, L, D)
+    three = jl.jetlong_prefill_three_pass_workspace_size(B, Hq, Hkv, L, D)
+    assert three >= fused + 3 * B * L * Hq * D * 4 + 3 * B * Hq * L * 4
+    assert three_pass_call(lib, wsb=fused) == jl.JL_ERR_WORKSPACE
+    assert three_pass_call(lib, wsb=three - 1) == jl.JL_ERR_WORKSPACE
+
+
 def decode_call(lib, **kw):
     a = dict(q=P, kc=P, vc=P, out=P, lse=None, B=1, Hq=32, Hkv=8, L=1000, Lcap=1000, D=128,
              wp=32768, w0=4096, theta=1e6, od=0, ws=P, wsb=1 << 40, stream=None)

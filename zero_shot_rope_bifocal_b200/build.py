@@ -22,7 +22,8 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libjetlong.so")
-SOURCES = ["jetlong_api.cu", "rope_kernels.cu", "decode_kernels.cu", "prefill_sm100.cu"]
+SOURCES = ["jetlong_api.cu", "rope_kernels.cu", "decode_kernels.cu", "prefill_sm100.cu",
+           "three_pass.cu"]
 HEADERS = ["jl_common.cuh", "sm100_ptx.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 CFLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden"]

@@ -86,6 +86,14 @@ size_t prefill_ws_bytes(int B, int Hq, int Hkv, int L, int D) {
   return 2 * align_up(q) + 3 * align_up(k);  // q_true, q_remote, k_true, k_remote, v
 }
 
+// Three-pass workspace: the prefill operands, then O_A, O_B, O_C (fp32
+// [B, L, Hq, D]) and lse_A, lse_B, lse_C (fp32 [B, Hq, L]).
+size_t three_pass_ws_bytes(int B, int Hq, int Hkv, int L, int D) {
+  const size_t o = align_up(static_cast<size_t>(B) * L * Hq * D * sizeof(float));
+  const size_t l = align_up(static_cast<size_t>(B) * Hq * L * sizeof(float));
+  return prefill_ws_bytes(B, Hq, Hkv, L, D) + 3 * o + 3 * l;
+}
+
 size_t decode_ws_bytes(int B, int Hq, int Hkv, int L, int D) {
   int ns = 0, ch = 0;
   decode_plan(B, Hkv, L, &ns, &ch);
@@ -140,7 +148,8 @@ enum PrefillStage : int { kStageRotate = 1, kStageAttend = 2, kStageBoth = 3 };
 int prepare_prefill(int stage, const void *q, const void *k, const void *v, void *out, float *lse,
                     int B, int Hq, int Hkv, int L, int D, int w_pretrained, int w0,
                     float rope_theta, int out_dtype, void *k_cache_out, int k_cache_capacity,
-                    void *workspace, size_t workspace_bytes, PrefillArgs *a) {
+                    void *workspace, size_t workspace_bytes, PrefillArgs *a,
+                    bool three_pass = false) {
   const bool rot = stage & kStageRotate, att = stage & kStageAttend;
   if (rot && (!q || !k || !v)) return JL_ERR_NULL;
   if (att && !out) return JL_ERR_NULL;
@@ -153,7 +162,8 @@ int prepare_prefill(int stage, const void *q, const void *k, const void *v, void
               (k_cache_out && !aligned16(k_cache_out))))
     return JL_ERR_ALIGN;
   if (att && (!aligned16(out) || (lse && !aligned16(lse)))) return JL_ERR_ALIGN;
-  const size_t need = prefill_ws_bytes(B, Hq, Hkv, L, D);
+  const size_t need = three_pass ? three_pass_ws_bytes(B, Hq, Hkv, L, D)
+                                 : prefill_ws_bytes(B, Hq, Hkv, L, D);
   if (!workspace || workspace_bytes < need) return JL_ERR_WORKSPACE;
   if (reinterpret_cast<uintptr_t>(workspace) % kAlign) return JL_ERR_ALIGN;
 
@@ -231,6 +241,45 @@ int jetlong_prefill_attend(void *out, float *lse, int B, int Hq, int Hkv, int L,
                                  const_cast<void *>(workspace), workspace_bytes, &a);
   if (st != JL_OK) return st;
   if (launch_prefill_attention(a, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return JL_ERR_CUDA;
+  return JL_OK;
+}
+
+size_t jetlong_prefill_three_pass_workspace_size(int B, int Hq, int Hkv, int L, int D) {
+  if (check_common(B, Hq, Hkv, L, D) != JL_OK) return 0;
+  return three_pass_ws_bytes(B, Hq, Hkv, L, D);
+}
+
+int jetlong_prefill_three_pass(const void *q, const void *k, const void *v, void *out, float *lse,
+                               int B, int Hq, int Hkv, int L, int D, int w_pretrained, int w0,
+                               float rope_theta, int out_dtype, void *workspace,
+                               size_t workspace_bytes, jl_stream_t stream) {
+  PrefillArgs a;
+  const int st = prepare_prefill(kStageBoth, q, k, v, out, lse, B, Hq, Hkv, L, D, w_pretrained,
+                                 w0, rope_theta, out_dtype, nullptr, 0, workspace, workspace_bytes,
+                                 &a, /*three_pass=*/true);
+  if (st != JL_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t *ws = static_cast<uint8_t *>(workspace) + prefill_ws_bytes(B, Hq, Hkv, L, D);
+  const size_t ob = align_up(static_cast<size_t>(B) * L * Hq * D * sizeof(float));
+  const size_t lb = align_up(static_cast<size_t>(B) * Hq * L * sizeof(float));
+  float *o_pass[3], *l_pass[3];
+  for (int i = 0; i < 3; ++i) {
+    o_pass[i] = reinterpret_cast<float *>(ws + i * ob);
+    l_pass[i] = reinterpret_cast<float *>(ws + 3 * ob + i * lb);
+  }
+  if (launch_rope_qk(a, s) != cudaSuccess) return JL_ERR_CUDA;
+  const PrefillPass passes[3] = {kPassRemoteCausal, kPassLocalBand, kPassRemoteBand};
+  for (int i = 0; i < 3; ++i) {
+    PrefillArgs p = a;
+    p.pass = passes[i];
+    p.out = o_pass[i];
+    p.lse = l_pass[i];
+    p.out_f32 = 1;
+    if (launch_prefill_attention(p, s) != cudaSuccess) return JL_ERR_CUDA;
+  }
+  if (launch_three_pass_merge(o_pass[0], o_pass[1], o_pass[2], l_pass[0], l_pass[1], l_pass[2],
+                              out, lse, out_dtype == JL_F32, B, Hq, L, D, s) != cudaSuccess)
     return JL_ERR_CUDA;
   return JL_OK;
 }

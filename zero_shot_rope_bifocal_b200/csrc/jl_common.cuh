@@ -55,6 +55,15 @@ __device__ __forceinline__ void rope_cos_sin(long long pos, double freq, float &
 __device__ __forceinline__ float bf2f(__nv_bfloat16 x) { return __bfloat162float(x); }
 
 // ---------------------------------------------------------------- launchers
+// What one prefill attention launch computes: the fused bifocal rule (§3), or
+// one pass of the three-pass inclusion-exclusion merge (§3.3).
+enum PrefillPass : int {
+  kPassFused = 0,
+  kPassRemoteCausal = 1,  // A: remote positions, every causal pair
+  kPassLocalBand = 2,     // B: true positions, 0 <= i - j <= w0
+  kPassRemoteBand = 3,    // C: remote positions, 0 <= i - j <= w0
+};
+
 struct PrefillArgs {
   // caller buffers
   const __nv_bfloat16 *q, *k, *v;
@@ -69,6 +78,7 @@ struct PrefillArgs {
   // sizes and method parameters
   int B, Hq, Hkv, L, D, w_pretrained, w0, G;
   float theta;
+  int pass;  // PrefillPass
   unsigned int *dev_error;
 };
 
@@ -77,6 +87,13 @@ cudaError_t launch_rope_qk(const PrefillArgs &a, cudaStream_t stream);
 
 // The attention kernel proper (tcgen05 / TMEM / TMA).
 cudaError_t launch_prefill_attention(const PrefillArgs &a, cudaStream_t stream);
+
+// out = (W_A O_A + W_B O_B - W_C O_C) / (W_A + W_B - W_C), W_X = exp(lse_X),
+// over the three passes' fp32 outputs [B, L, Hq, D] and lse [B, Hq, L].
+cudaError_t launch_three_pass_merge(const float *o_a, const float *o_b, const float *o_c,
+                                    const float *l_a, const float *l_b, const float *l_c,
+                                    void *out, float *lse, int out_f32, int B, int Hq, int L,
+                                    int D, cudaStream_t stream);
 
 struct DecodeArgs {
   const __nv_bfloat16 *q, *k_cache, *v_cache;

@@ -84,6 +84,7 @@ struct Layout {
 
 struct Params {
   int B, Hq, Hkv, L, G, w0eff, n_qt, grp, npair;
+  int pass;  // PrefillPass: the fused rule or one pass of the three-pass merge
   float scale_log2;
   void *out;
   float *lse;
@@ -166,14 +167,34 @@ bifocal_prefill_kernel(const __grid_constant__ CUtensorMap tm_qt,
   const int p1 = min(p0 + BM, prm.L) - 1;
   const int w0 = prm.w0eff;
 
-  // Visit plan: remote visits of key tiles [0, n_rem), then local visits of
-  // key tiles [kl0, n_kt).  Every causal pair of the tile is kept by exactly
-  // one visit.
+  // Visit plan: remote visits of key tiles [kr0, kr0 + n_rem), then local
+  // visits of key tiles [kl0, n_kt).  A remote visit keeps the pairs with
+  // dlo <= i - j <= dhi, a local visit those with 0 <= i - j <= w0.  Fused
+  // rule: remote tiles [0, n_rem) with i - j > w0, so every causal pair of
+  // the tile is kept by exactly one visit.  The passes of the three-pass
+  // merge (§3.3) reuse the same machinery: A = remote positions on every
+  // causal pair, B = true positions on the band 0 <= i - j <= w0, C = remote
+  // positions on the band.
   const int n_kt = p1 / BN + 1;
-  int n_rem = 0, kl0 = 0;
-  if (prm.G > 1) {
-    n_rem = (p1 - w0 > 0) ? ((p1 - w0 - 1) / BN + 1) : 0;
+  int n_rem = 0, kl0 = 0, kr0 = 0;
+  int dlo = w0 == INT_MAX ? INT_MAX : w0 + 1, dhi = INT_MAX;
+  if (prm.pass == kPassFused) {
+    if (prm.G > 1) {
+      n_rem = (p1 - w0 > 0) ? ((p1 - w0 - 1) / BN + 1) : 0;
+      kl0 = max(0, p0 - w0) / BN;
+    }
+  } else if (prm.pass == kPassRemoteCausal) {
+    n_rem = n_kt;
+    kl0 = n_kt;
+    dlo = 0;
+  } else if (prm.pass == kPassLocalBand) {
     kl0 = max(0, p0 - w0) / BN;
+  } else {  // kPassRemoteBand
+    kr0 = max(0, p0 - w0) / BN;
+    n_rem = n_kt - kr0;
+    kl0 = n_kt;
+    dlo = 0;
+    dhi = w0;
   }
   const int nv = n_rem + (n_kt - kl0);
   const bool switch_q = n_rem > 0 && n_rem < nv;
@@ -235,7 +256,7 @@ bifocal_prefill_kernel(const __grid_constant__ CUtensorMap tm_qt,
       uint32_t issued[NS] = {0, 0, 0, 0};  // uses issued per slot
       for (int j = 0; j < nv && ok; ++j) {
         const bool remote = j < n_rem;
-        const int kt = remote ? j : kl0 + (j - n_rem);
+        const int kt = remote ? kr0 + j : kl0 + (j - n_rem);
         for (int part = 0; part < 2 && ok; ++part, ++r) {
           const int slot = r % NS;
           const uint32_t use = static_cast<uint32_t>(r / NS);
@@ -371,7 +392,7 @@ bifocal_prefill_kernel(const __grid_constant__ CUtensorMap tm_qt,
     bool ok = active;
     for (int j = 0; j < nv && ok; ++j) {
       const bool remote = j < n_rem;
-      const int kt = remote ? j : kl0 + (j - n_rem);
+      const int kt = remote ? kr0 + j : kl0 + (j - n_rem);
       ok = wait_or_abort(bar(LY::kSFull + s), static_cast<uint32_t>(j) & 1u, abort);
       if (__any_sync(0xffffffffu, !ok)) {
         ok = false;
@@ -391,14 +412,14 @@ bifocal_prefill_kernel(const __grid_constant__ CUtensorMap tm_qt,
       const int k0 = kt * BN;
       bool whole;
       if (remote)
-        whole = row_ok && (row - (k0 + BN - 1) > w0);
+        whole = row_ok && (row - (k0 + BN - 1) >= dlo) && (row - k0 <= dhi);
       else
         whole = row_ok && (k0 + BN - 1 <= row) && (row - k0 <= w0);
       if (!whole) {
 #pragma unroll
         for (int c = 0; c < BN; ++c) {
           const int d = row - (k0 + c);
-          const bool valid = row_ok && d >= 0 && (remote ? (d > w0) : (d <= w0));
+          const bool valid = row_ok && d >= 0 && (remote ? (d >= dlo && d <= dhi) : (d <= w0));
           if (!valid) x[c] = -INFINITY;
         }
       }
@@ -574,7 +595,10 @@ cudaError_t launch_d(const PrefillArgs &a, cudaStream_t stream) {
   prm.Hkv = a.Hkv;
   prm.L = a.L;
   prm.G = a.G;
-  prm.w0eff = a.G == 1 ? INT_MAX : a.w0;
+  // The fused rule with G = 1 is plain causal attention; a pass of the
+  // three-pass merge keeps its band whatever G is.
+  prm.w0eff = (a.G == 1 && a.pass == kPassFused) ? INT_MAX : a.w0;
+  prm.pass = a.pass;
   prm.n_qt = (a.L + BM - 1) / BM;
   prm.grp = a.Hq / a.Hkv;
   prm.npair = (prm.grp + 1) / 2;

@@ -44,6 +44,9 @@ SIGNATURES = {
     "jetlong_prefill_rotate": (_I, [_VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _F, _VP, _I, _VP, _SZ,
                                     _VP]),
     "jetlong_prefill_attend": (_I, [_VP, _VP, _I, _I, _I, _I, _I, _I, _I, _I, _VP, _SZ, _VP]),
+    "jetlong_prefill_three_pass_workspace_size": (_SZ, [_I, _I, _I, _I, _I]),
+    "jetlong_prefill_three_pass": (_I, [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _I, _F,
+                                        _I, _VP, _SZ, _VP]),
     "jetlong_decode_workspace_size": (_SZ, [_I, _I, _I, _I, _I]),
     "jetlong_decode": (_I, [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _I, _I, _F, _I,
                             _VP, _SZ, _VP]),
@@ -135,6 +138,10 @@ def jetlong_prefill_workspace_size(B, Hq, Hkv, L, D) -> int:
     return int(lib().jetlong_prefill_workspace_size(B, Hq, Hkv, L, D))
 
 
+def jetlong_prefill_three_pass_workspace_size(B, Hq, Hkv, L, D) -> int:
+    return int(lib().jetlong_prefill_three_pass_workspace_size(B, Hq, Hkv, L, D))
+
+
 def jetlong_decode_workspace_size(B, Hq, Hkv, L, D) -> int:
     return int(lib().jetlong_decode_workspace_size(B, Hq, Hkv, L, D))
 
@@ -207,6 +214,37 @@ def jetlong_prefill_attend(out, lse, Hkv: int, w_pretrained: int, w0: int, works
                                       int(w_pretrained), int(w0), _out_dtype(out.dtype),
                                       _ptr(workspace), workspace.numel(), _stream_ptr(stream))
     _check("jetlong_prefill_attend", st)
+
+
+def jetlong_prefill_three_pass(q, k, v, w_pretrained: int, w0: int, rope_theta: float, *,
+                               out=None, lse=None, out_dtype=torch.bfloat16, want_lse: bool = True,
+                               workspace=None, stream=None):
+    """The unfused three-pass (inclusion-exclusion) form of jetlong_prefill.
+    Returns (out, lse or None)."""
+    if q.dim() != 4 or k.dim() != 4:
+        raise ValueError("q, k, v must be [B, L, H, D]")
+    B, L, Hq, D = q.shape
+    Hkv = k.shape[2]
+    _require(q, "q", (B, L, Hq, D), torch.bfloat16)
+    _require(k, "k", (B, L, Hkv, D), torch.bfloat16)
+    _require(v, "v", (B, L, Hkv, D), torch.bfloat16)
+    od = _out_dtype(out_dtype if out is None else out.dtype)
+    if out is None:
+        out = torch.empty((B, L, Hq, D), dtype=torch.bfloat16 if od == JL_BF16 else torch.float32,
+                          device=q.device)
+    _require(out, "out", (B, L, Hq, D), out.dtype)
+    if lse is None and want_lse:
+        lse = torch.empty((B, Hq, L), dtype=torch.float32, device=q.device)
+    if lse is not None:
+        _require(lse, "lse", (B, Hq, L), torch.float32)
+    if workspace is None:
+        workspace = _ws(jetlong_prefill_three_pass_workspace_size(B, Hq, Hkv, L, D), q.device)
+    st = lib().jetlong_prefill_three_pass(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq,
+                                          Hkv, L, D, int(w_pretrained), int(w0),
+                                          float(rope_theta), od, _ptr(workspace),
+                                          workspace.numel(), _stream_ptr(stream))
+    _check("jetlong_prefill_three_pass", st)
+    return out, lse
 
 
 def jetlong_decode(q, k_cache, v_cache, L: int, w_pretrained: int, w0: int, rope_theta: float, *,

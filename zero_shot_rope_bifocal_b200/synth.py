@@ -112,6 +112,24 @@ def decode_inputs(w: Workload, Lcap: int | None = None, device="cpu") -> DecodeI
     return DecodeInputs(q.to(torch.bfloat16), k.to(torch.bfloat16), v.to(torch.bfloat16))
 
 
+@dataclass
+class GenerationInputs:
+    q: torch.Tensor      # [n_steps, B, Hq, D] bf16, the query of each step (pre-RoPE)
+    k_raw: torch.Tensor  # [B, L0 + n_steps, Hkv, D] bf16, pre-RoPE keys of every slot
+    v: torch.Tensor      # [B, L0 + n_steps, Hkv, D] bf16
+
+
+def generation_inputs(w: Workload, L0: int, n_steps: int, device="cpu") -> GenerationInputs:
+    """A cache prefix of ``L0`` tokens plus ``n_steps`` generated tokens: their
+    raw keys and values, and one query per step.  Draw order: K, V, queries."""
+    g = _gen(w.seed, device)
+    cap = L0 + n_steps
+    k = torch.randn((w.B, cap, w.Hkv, w.D), generator=g, device=device, dtype=torch.float32)
+    v = torch.randn((w.B, cap, w.Hkv, w.D), generator=g, device=device, dtype=torch.float32)
+    q = torch.randn((n_steps, w.B, w.Hq, w.D), generator=g, device=device, dtype=torch.float32)
+    return GenerationInputs(q.to(torch.bfloat16), k.to(torch.bfloat16), v.to(torch.bfloat16))
+
+
 def sample_rows(L: int, w0: int, w_pretrained: int, n: int, seed: int) -> list[int]:
     """Query rows to check on a large workload: the edges of the local window,
     the native-window and group boundaries, the last rows, then seeded random
