@@ -53,9 +53,14 @@ def test_generation_loop_across_group_transition():
         assert_lse(f64(lse), lse_ref, f"step L={L}")
         groups.append(jl.jetlong_group_size(L, w.w_pretrained))
     assert groups == [3, 3, 3, 3, 4, 4, 4, 4]  # L = 98301..98308
-    # the appended rows are the true-position RoPE of each key, to BF16 rounding
+    # The appended rows are the true-position RoPE of each key.  Both sides
+    # round a rotation to BF16 (the GPU's fp32 one, the oracle's fp64 one), so
+    # a value near a rounding boundary may land one BF16 ulp (2^-7 relative)
+    # apart; with rotations that agree to ~1e-7 that happens for ~1e-4 of
+    # the entries at most.
     got, ref = f64(kc), ref_cache64
-    assert np.all(np.abs(got - ref) <= 2.0 ** -8 * np.abs(ref) + 1e-6)
+    assert np.all(np.abs(got - ref) <= 2.0 ** -7 * np.abs(ref) + 1e-6)
+    assert np.mean(got != ref) < 1e-3
 
 
 @pytest.mark.parametrize("L", [262144, 524288, 1048576])

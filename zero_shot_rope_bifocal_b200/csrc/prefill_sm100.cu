@@ -26,19 +26,24 @@
 //
 // CTA = two 128-row query tiles of the same 128 positions, for two query
 // heads of one KV group (GQA packing: each K/V tile staged in shared memory
-// serves 256 query rows).  Warp-specialised, 12 warps:
-//   * warps 0-3 / 4-7: softmax for query tile 0 / 1 (one thread per row =
-//     one TMEM lane); they also rescale their O rows when needed and run the
-//     epilogue;
-//   * warp 8: TMA producer (queries once per variant, K and V tiles through a
-//     four-slot ring);
-//   * warp 9: tcgen05.mma issuer, in the order
+// serves 256 query rows).  Warp-specialised, 20 warps:
+//   * warps 0-3 / 4-7: softmax for query tile 0 / 1, score columns [0, 64);
+//     warps 8-11 / 12-15: the same rows, columns [64, 128).  Two threads (one
+//     per column half) own each row of a tile (a TMEM lane); they trade their
+//     half-row maxima through shared memory and one mbarrier per warp pair,
+//     rescale their halves of the O row when needed and run the epilogue;
+//   * warp 16: TMA producer (queries once per variant, K and V tiles through
+//     a four-slot ring);
+//   * warp 17: tcgen05.mma issuer, in the order
 //       S0(j+1) = Q0 K(j+1)^T after O0 += P0(j) V(j), and likewise for tile 1,
 //     so the tensor core works on one tile while the other tile's softmax
 //     runs;
-//   * warps 10-11 hold no role.
-// TMEM (512 columns): S0 | S1 | O0 | O1; P of each tile overwrites the first
-// 64 columns of its S as packed FP16 once the S row is in registers.
+//   * warps 18-19 hold no role.
+// Two threads per row keep 32 scores live at a time, so the softmax fits the
+// 96 registers per thread that 20 warps leave, without spills.
+// TMEM (512 columns): S0 | S1 | O0 | O1; each half of a row writes its P
+// (packed FP16) over the first 32 columns of its own 64-column half of S
+// once those scores are in registers.
 // Each wait is bounded in time (jl::kWaitLimitNs) and also gives up when
 // another role has given up; the CTA then records a device error, drains its
 // MMAs and in-flight copies, frees TMEM and exits.
@@ -53,12 +58,18 @@ namespace {
 constexpr int BM = 128;  // query rows per tile (= TMEM lanes)
 constexpr int BN = 128;  // keys per tile
 constexpr int NS = 4;    // K/V ring slots (one K or V tile each)
-constexpr int kWarps = 12;
+constexpr int kSoftmaxWarps = 16;  // 4 warpgroups: (tile, column half)
+constexpr int kWarps = 20;
 constexpr int kThreads = kWarps * 32;
-constexpr int kProducerWarp = 8;
-constexpr int kMmaWarp = 9;
-constexpr int kSoftmaxRegs = 200;
-constexpr int kOtherRegs = 96;
+constexpr int kProducerWarp = 16;
+constexpr int kMmaWarp = 17;
+constexpr int HBN = BN / 2;  // score columns per softmax thread
+// Registers: 20 warps put 5 on each of the 4 SM sub-partitions, whose
+// register files hold 16,384 each, so every thread gets 96 and the softmax
+// is written to fit (32 scores live at a time).  No setmaxnreg: an increase
+// can only be served from what other warps release with a decrease, and the
+// four non-softmax warps could not release enough to lift the 16 softmax
+// warps to a useful size.
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 constexpr uint32_t kF16 = 0;               // operand format code of kind::f16
 
@@ -72,8 +83,12 @@ struct Layout {
   // barrier indices (8 bytes each)
   static constexpr int kQFull = 0, kQEmpty = 2, kKvFull = 4, kKvEmpty = 4 + NS,
                        kSFull = 4 + 2 * NS, kPFull = 6 + 2 * NS, kOFull = 8 + 2 * NS,
-                       kDrain = 10 + 2 * NS, kNumBars = 11 + 2 * NS;
-  static constexpr int TMEM_SLOT = BAR + 8 * kNumBars;
+                       kDrain = 10 + 2 * NS, kPair = 11 + 2 * NS,  // 8 pair barriers
+                       kNumBars = 19 + 2 * NS;
+  // half-row maxima (and, at the end, half-row sums) traded by the two
+  // threads of a row: [parity][tile][half][row] floats
+  static constexpr int XCHG = BAR + 8 * kNumBars;
+  static constexpr int TMEM_SLOT = XCHG + 2 * 2 * 2 * BM * 4;
   static constexpr int ABORT = TMEM_SLOT + 4;
   static constexpr int SKIP = TMEM_SLOT + 8;
   static constexpr int BYTES = TMEM_SLOT + 16;
@@ -114,13 +129,6 @@ __device__ __forceinline__ float2 exp2_fma2(float2 x) {
   // bits(t) << 23 == n << 23 (the bits of kRound shift out); add to p's exponent
   return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(t.x) << 23)),
                      __int_as_float(__float_as_int(p.y) + (__float_as_int(t.y) << 23)));
-}
-
-__device__ __forceinline__ void set_regs_softmax() {
-  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftmaxRegs));
-}
-__device__ __forceinline__ void set_regs_other() {
-  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kOtherRegs));
 }
 
 // Bounded wait that also gives up once another role has raised `abort`.
@@ -210,9 +218,12 @@ bifocal_prefill_kernel(const __grid_constant__ CUtensorMap tm_qt,
 
   if (tid == 0) {
     // P-ready barriers take one arrival from every softmax thread of the
-    // tile; all others one arrival (plus transaction bytes for TMA).
+    // tile (two per row), pair barriers one from each thread of a warp pair;
+    // all others one arrival (plus transaction bytes for TMA).
     for (int i = 0; i < LY::kNumBars; ++i)
-      mbar_init(bar(i), (i == LY::kPFull || i == LY::kPFull + 1) ? BM : 1);
+      mbar_init(bar(i), (i == LY::kPFull || i == LY::kPFull + 1) ? 2 * BM
+                        : (i >= LY::kPair && i < LY::kPair + 8)   ? 64
+                                                                  : 1);
     fence_mbar_init();
   }
   if (warp == kProducerWarp && lane == 0) {
@@ -239,8 +250,7 @@ bifocal_prefill_kernel(const __grid_constant__ CUtensorMap tm_qt,
   constexpr uint32_t IDESC_PV = idesc_f16kind_f32(BM, D, kF16, false, true);
   constexpr int NBOX = D / 64;
 
-  if (warp >= 8) {
-    set_regs_other();
+  if (warp >= kSoftmaxWarps) {
     if (warp == kProducerWarp && lane == 0) {
       // ---------------------------------------------------------- producer
       auto load_q = [&](int s, bool remote) {
@@ -300,9 +310,10 @@ bifocal_prefill_kernel(const __grid_constant__ CUtensorMap tm_qt,
       auto pv = [&](int s, uint32_t vslot, bool acc) {
         const uint32_t vb = sb + LY::RING + vslot * LY::TILE;
 #pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk)
-          mma_f16kind_ts(tO(s), tS(s) + kk * 8, smem_desc_sw128(vb + kk * 16 * 128, LY::BOX, 1024),
-                         IDESC_PV, (acc || kk > 0) ? 1u : 0u);
+        for (int kk = 0; kk < BN / 16; ++kk)  // P of keys [16kk, 16kk+16): half kk/4's columns
+          mma_f16kind_ts(tO(s), tS(s) + (kk >> 2) * HBN + (kk & 3) * 8,
+                         smem_desc_sw128(vb + kk * 16 * 128, LY::BOX, 1024), IDESC_PV,
+                         (acc || kk > 0) ? 1u : 0u);
       };
       bool ok = wait_or_abort(bar(LY::kQFull + 0), 0u, abort);
       if (ok && has1) ok = wait_or_abort(bar(LY::kQFull + 1), 0u, abort);
@@ -379,18 +390,24 @@ bifocal_prefill_kernel(const __grid_constant__ CUtensorMap tm_qt,
     }
   } else {
     // ------------------------------------------------------------ softmax
-    set_regs_softmax();
-    const int s = warp >> 2;             // query tile of this warpgroup
+    const int s = (warp >> 2) & 1;       // query tile of this warpgroup
+    const int half = warp >> 3;          // score columns [half * 64, half * 64 + 64)
     const int wq = warp & 3;             // TMEM lane quarter
     const int rloc = tid & (BM - 1);     // row inside the tile
     const int row = p0 + rloc;
     const bool active = s == 0 || has1;
     const bool row_ok = active && row < prm.L;
     const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
-    float m_used = -INFINITY;  // reference max of this row (base 2)
-    float l_sum = 0.f;
+    const uint32_t pair_bar = bar(LY::kPair + s * 4 + wq);  // this warp and its other half
+    float *xchg = reinterpret_cast<float *>(smem + LY::XCHG);
+    // slot of (parity, tile, half, row) in the exchange buffer
+    auto xslot = [&](int par, int h) { return ((par * 2 + s) * 2 + h) * BM + rloc; };
+    const int c0 = half * HBN;           // first score column of this thread
+    float m_used = -INFINITY;  // reference max of this row (base 2), same in both halves
+    float l_sum = 0.f;         // this half's share of the row sum
     bool ok = active;
-    for (int j = 0; j < nv && ok; ++j) {
+    int j = 0;
+    for (; j < nv && ok; ++j) {
       const bool remote = j < n_rem;
       const int kt = remote ? kr0 + j : kl0 + (j - n_rem);
       ok = wait_or_abort(bar(LY::kSFull + s), static_cast<uint32_t>(j) & 1u, abort);
@@ -399,42 +416,56 @@ bifocal_prefill_kernel(const __grid_constant__ CUtensorMap tm_qt,
         break;
       }
       tc_fence_after();
-      float x[BN];
-      {
-        uint32_t(&xr)[BN] = reinterpret_cast<uint32_t(&)[BN]>(x);
-#pragma unroll
-        for (int c = 0; c < BN / 32; ++c)
-          tmem_ld32(tS(s) + lane_base + c * 32, reinterpret_cast<uint32_t(&)[32]>(xr[c * 32]));
-        tmem_wait_ld();
-#pragma unroll
-        for (int c = 0; c < BN / 32; ++c) reg_fence(reinterpret_cast<uint32_t(&)[32]>(xr[c * 32]));
-      }
-      const int k0 = kt * BN;
+      const int k0 = kt * BN + c0;  // key of this thread's first score column
       bool whole;
       if (remote)
-        whole = row_ok && (row - (k0 + BN - 1) >= dlo) && (row - k0 <= dhi);
+        whole = row_ok && (row - (k0 + HBN - 1) >= dlo) && (row - k0 <= dhi);
       else
-        whole = row_ok && (k0 + BN - 1 <= row) && (row - k0 <= w0);
-      if (!whole) {
+        whole = row_ok && (k0 + HBN - 1 <= row) && (row - k0 <= w0);
+      // This thread's scores, 32 columns at a time, with the mask applied
+      // (raw scores; the scale is positive and applied later).
+      auto load_chunk = [&](int cc, float (&x)[32]) {
+        uint32_t(&xr)[32] = reinterpret_cast<uint32_t(&)[32]>(x);
+        tmem_ld32(tS(s) + lane_base + c0 + cc * 32, xr);
+        tmem_wait_ld();
+        reg_fence(xr);
+        if (!whole) {
 #pragma unroll
-        for (int c = 0; c < BN; ++c) {
-          const int d = row - (k0 + c);
-          const bool valid = row_ok && d >= 0 && (remote ? (d >= dlo && d <= dhi) : (d <= w0));
-          if (!valid) x[c] = -INFINITY;
+          for (int c = 0; c < 32; ++c) {
+            const int d = row - (k0 + cc * 32 + c);
+            const bool valid = row_ok && d >= 0 && (remote ? (d >= dlo && d <= dhi) : (d <= w0));
+            if (!valid) x[c] = -INFINITY;
+          }
         }
-      }
-      // row max: a tree of three-input maxima (raw scores; the scale is positive)
-      float mx[4] = {x[0], x[1], x[2], x[3]};
+      };
+      // pass 1: the half-row max (a tree of three-input maxima per chunk),
+      // then the other half's through shared memory
+      float hmax = -INFINITY;
+#pragma unroll 1
+      for (int cc = 0; cc < HBN / 32; ++cc) {
+        float x[32];
+        load_chunk(cc, x);
+        float mx[4] = {x[0], x[1], x[2], x[3]};
 #pragma unroll
-      for (int c = 4; c < BN; c += 8) {
-        mx[0] = fmax3(mx[0], x[c], x[c + 1]);
-        mx[1] = fmax3(mx[1], x[c + 2], x[c + 3]);
-        if (c + 4 < BN) {
-          mx[2] = fmax3(mx[2], x[c + 4], x[c + 5]);
-          mx[3] = fmax3(mx[3], x[c + 6], x[c + 7]);
+        for (int c = 4; c < 32; c += 8) {
+          mx[0] = fmax3(mx[0], x[c], x[c + 1]);
+          mx[1] = fmax3(mx[1], x[c + 2], x[c + 3]);
+          if (c + 4 < 32) {
+            mx[2] = fmax3(mx[2], x[c + 4], x[c + 5]);
+            mx[3] = fmax3(mx[3], x[c + 6], x[c + 7]);
+          }
         }
+        hmax = fmax3(hmax, fmax3(mx[0], mx[1], mx[2]), mx[3]);
       }
-      const float tmax = fmaxf(fmax3(mx[0], mx[1], mx[2]), mx[3]) * prm.scale_log2;
+      xchg[xslot(j & 1, half)] = hmax;
+      mbar_arrive(pair_bar);
+      ok = wait_or_abort(pair_bar, static_cast<uint32_t>(j) & 1u, abort);
+      if (__any_sync(0xffffffffu, !ok)) {
+        ok = false;
+        break;
+      }
+      const float tmax = fmaxf(hmax, xchg[xslot(j & 1, half ^ 1)]) * prm.scale_log2;
+      // both halves see the same tmax and m_used, so they take the same step
       const bool grow =
           tmax > m_used + kRescaleThreshold || (m_used == -INFINITY && tmax > -INFINITY);
       float alpha = 1.f;
@@ -443,73 +474,82 @@ bifocal_prefill_kernel(const __grid_constant__ CUtensorMap tm_qt,
         m_used = tmax;
       }
       l_sum *= alpha;
-      // O of this tile holds visits 0..j-1 (all complete: S(j) was issued
-      // after P(j-1) V(j-1)); rows whose max was -inf hold 0 there.
-      if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
-        __syncwarp();
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t rr[32];
-          tmem_ld32(tO(s) + lane_base + c * 32, rr);
-          tmem_wait_ld();
-          reg_fence(rr);
-#pragma unroll
-          for (int e = 0; e < 32; ++e) rr[e] = __float_as_uint(u2f(rr[e]) * alpha);
-          tmem_st32(tO(s) + lane_base + c * 32, rr);
-        }
-      }
-      // p = 2^(s * scale - m): masked entries are -inf and give 0 (or 2^-125
+      // pass 2: p = 2^(s * scale - m) per chunk, written back as packed FP16
+      // P over the first half of this thread's own columns (chunk cc lands on
+      // columns already read).  Masked entries are -inf and give 0 (or 2^-125
       // on the FMA path, which rounds to 0 in FP16); a row with nothing valid
-      // yet has all entries -inf.  One column pair in four takes the FMA-pipe
+      // yet has all entries -inf.  One column pair in eight takes the FMA-pipe
       // exponential, the rest the special-function unit.
       const float neg_m = m_used == -INFINITY ? 0.f : -m_used;
       const float2 sc2 = make_float2(prm.scale_log2, prm.scale_log2);
       const float2 nm2 = make_float2(neg_m, neg_m);
-      float2 acc2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
-                        make_float2(0.f, 0.f)};
+      float2 acc2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+#pragma unroll 1
+      for (int cc = 0; cc < HBN / 32; ++cc) {
+        float x[32];
+        load_chunk(cc, x);
+        uint32_t pr[16];
 #pragma unroll
-      for (int c = 0; c < BN; c += 2) {
-        float2 v = ffma2(make_float2(x[c], x[c + 1]), sc2, nm2);
-        if ((c & 7) == 0) {
-          v = exp2_fma2(v);
-        } else {
-          v.x = ex2_sfu(v.x);
-          v.y = ex2_sfu(v.y);
+        for (int c = 0; c < 32; c += 2) {
+          float2 v = ffma2(make_float2(x[c], x[c + 1]), sc2, nm2);
+          if ((c & 15) == 0) {
+            v = exp2_fma2(v);
+          } else {
+            v.x = ex2_sfu(v.x);
+            v.y = ex2_sfu(v.y);
+          }
+          acc2[(c >> 1) & 1] = fadd2(acc2[(c >> 1) & 1], v);
+          const __half2 h2 = __floats2half2_rn(v.x, v.y);
+          pr[c >> 1] = *reinterpret_cast<const uint32_t *>(&h2);
         }
-        x[c] = v.x;
-        x[c + 1] = v.y;
-        acc2[(c >> 1) & 3] = fadd2(acc2[(c >> 1) & 3], v);
+        __syncwarp();
+        tmem_st16(tS(s) + lane_base + c0 + cc * 16, pr);
+        tmem_wait_st();
       }
-      const float2 a01 = fadd2(acc2[0], acc2[1]), a23 = fadd2(acc2[2], acc2[3]);
-      const float2 a = fadd2(a01, a23);
+      const float2 a = fadd2(acc2[0], acc2[1]);
       l_sum += a.x + a.y;
-      __syncwarp();
+      // O of this tile holds visits 0..j-1 (all complete: S(j) was issued
+      // after P(j-1) V(j-1)); rows whose max was -inf hold 0 there.  Each
+      // half rescales its half of the O row before PV(j) may start.
+      if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+        __syncwarp();
+#pragma unroll 1
+        for (int c = 0; c < D / 64; ++c) {  // one 32-column chunk at a time (registers)
+          uint32_t rr[32];
+          const uint32_t col = tO(s) + lane_base + half * (D / 2) + c * 32;
+          tmem_ld32(col, rr);
+          tmem_wait_ld();
+          reg_fence(rr);
 #pragma unroll
-      for (int c = 0; c < BN / 64; ++c) {
-        uint32_t rr[32];
-#pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const __half2 h2 = __floats2half2_rn(x[c * 64 + 2 * e], x[c * 64 + 2 * e + 1]);
-          rr[e] = *reinterpret_cast<const uint32_t *>(&h2);
+          for (int e = 0; e < 32; ++e) rr[e] = __float_as_uint(u2f(rr[e]) * alpha);
+          tmem_st32(col, rr);
+          tmem_wait_st();
         }
-        tmem_st32(tS(s) + lane_base + c * 32, rr);
       }
-      tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bar(LY::kPFull + s));
     }
-    // ---- epilogue
+    // ---- epilogue: the row sum is the two halves' sums
     if (ok) ok = wait_or_abort(bar(LY::kOFull + s), 0u, abort);
     if (__all_sync(0xffffffffu, ok) && active) {
+      xchg[xslot(j & 1, half)] = l_sum;
+      mbar_arrive(pair_bar);
+      ok = wait_or_abort(pair_bar, static_cast<uint32_t>(j) & 1u, abort);
+    } else {
+      ok = false;
+    }
+    if (__all_sync(0xffffffffu, ok)) {
+      const float l_row = l_sum + xchg[xslot(j & 1, half ^ 1)];
       tc_fence_after();
-      const float inv_l = row_ok ? 1.f / l_sum : 0.f;
+      const float inv_l = row_ok ? 1.f / l_row : 0.f;
       const int head = head0 + s;
-      const size_t obase = ((static_cast<size_t>(b) * prm.L + row) * prm.Hq + head) * D;
-#pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
+      const int ch0 = half * (D / 2);  // first output channel of this thread
+      const size_t obase = ((static_cast<size_t>(b) * prm.L + row) * prm.Hq + head) * D + ch0;
+#pragma unroll 1
+      for (int c = 0; c < D / 64; ++c) {
         uint32_t rr[32];
         __syncwarp();
-        tmem_ld32(tO(s) + lane_base + c * 32, rr);  // whole warp, valid row or not
+        tmem_ld32(tO(s) + lane_base + ch0 + c * 32, rr);  // whole warp, valid row or not
         tmem_wait_ld();
         reg_fence(rr);
         if (!row_ok) continue;
@@ -534,9 +574,9 @@ bifocal_prefill_kernel(const __grid_constant__ CUtensorMap tm_qt,
           }
         }
       }
-      if (row_ok && prm.lse)
+      if (row_ok && half == 0 && prm.lse)
         prm.lse[(static_cast<size_t>(b) * prm.Hq + head) * prm.L + row] =
-            (m_used + log2f(l_sum)) * 0.69314718055994531f;
+            (m_used + log2f(l_row)) * 0.69314718055994531f;
     }
   }
 
