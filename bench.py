@@ -100,33 +100,51 @@ def reduce_sum(x: float, world: int, device=None) -> float:
 
 # ---------------------------------------------------------------- clocks
 class ClockSampler:
-    """Samples SM clocks and throttle reasons with nvidia-smi while running."""
+    """Samples SM clocks and throttle reasons with nvidia-smi (every 100 ms).
+
+    The sampler starts on entry and waits for its first sample, so that the
+    timed region that follows is covered; ``window(t0, t1)`` (times from
+    ``now()``) restricts the summary to the samples taken inside it.
+    """
 
     QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    PERIOD_S = 0.1
 
     def __init__(self, gpu_index: int):
         self.gpu = gpu_index
         self.proc = None
-        self.lines = []
+        self.lines = []  # (arrival time, csv line)
         self.thread = None
+        self.t0 = None
+        self.t1 = None
+
+    @staticmethod
+    def now() -> float:
+        return time.monotonic()
 
     def __enter__(self):
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.QUERY}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", str(int(self.PERIOD_S * 1000))],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.thread = threading.Thread(target=self._read, daemon=True)
             self.thread.start()
+            deadline = time.monotonic() + 5.0
+            while not self.lines and time.monotonic() < deadline and self.proc.poll() is None:
+                time.sleep(0.02)
         except (OSError, FileNotFoundError):
             self.proc = None
         return self
 
     def _read(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            self.lines.append((time.monotonic(), line.strip()))
+
+    def window(self, t0: float, t1: float) -> None:
+        self.t0, self.t1 = t0, t1
 
     def __exit__(self, *exc):
         if self.proc is not None:
@@ -139,11 +157,17 @@ class ClockSampler:
                 self.thread.join(timeout=2)
 
     def summary(self):
-        if not self.lines:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        lines = self.lines
+        if self.t0 is not None:
+            # a sample reports the state when it was taken, shortly before it
+            # arrives: keep those that arrived inside the window or within one
+            # period after it
+            lines = [(t, ln) for t, ln in lines if self.t0 <= t <= self.t1 + self.PERIOD_S]
+        if not lines:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
         sm, smax, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
+        for _, ln in lines:
             f = [x.strip() for x in ln.split(",")]
             if len(f) < 9:
                 continue
@@ -290,11 +314,13 @@ def run_native(args):
     with ClockSampler(local) as clocks:
         barrier()
         torch.cuda.synchronize(dev)
+        tw0 = clocks.now()
         ev0.record(stream)
         for s in range(args.steps):
             step(mids[s], ends[s])
         ev1.record(stream)
         torch.cuda.synchronize(dev)
+        clocks.window(tw0, clocks.now())
         barrier()
     t_ms = ev0.elapsed_time(ev1)
     attn_ms = sum(mids[s].elapsed_time(ends[s]) for s in range(args.steps)) / args.steps
@@ -382,11 +408,13 @@ def run_native(args):
     with ClockSampler(local) as dclocks:
         barrier()
         torch.cuda.synchronize(dev)
+        tw0 = dclocks.now()
         ev0.record(stream)
         for _ in range(n_dec):
             dstep()
         ev1.record(stream)
         torch.cuda.synchronize(dev)
+        dclocks.window(tw0, dclocks.now())
         barrier()
     dec_ms = reduce_max(ev0.elapsed_time(ev1), world, dev)
     if jl.jetlong_device_status() != jl.JL_OK:
@@ -463,7 +491,9 @@ def run_native(args):
             "metric": "bifocal-attn prefill TFLOP/s @128K (Qwen3-8B layer); decode us/token",
             "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": t_max / args.steps, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "scaling": "weak", "vs_baseline": None, "dtype": "f16",
+            "precision": "BF16 inputs and outputs; FP16 tensor-core operands (rotated Q/K, V, "
+                         "P) with FP32 accumulation; FP32 softmax statistics",
             "data": "synthetic (seeded N(0,1) Q/K/V, K per-channel LogNormal(0,0.5) scale)",
             "config": {"workload": PREFILL_WORKLOAD, "B": B, "Hq": Hq, "Hkv": Hkv, "D": D, "L": L,
                        "w_pretrained": w.w_pretrained, "w0": w.w0, "rope_theta": w.theta,

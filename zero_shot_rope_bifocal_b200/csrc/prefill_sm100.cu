@@ -297,22 +297,23 @@ bifocal_prefill_kernel(const __grid_constant__ CUtensorMap tm_qt,
     } else if (warp == kMmaWarp && lane == 0) {
       // ---------------------------------------------------------- MMA issuer
       auto qk = [&](int s, uint32_t kslot) {
-        const uint32_t qa = sb + LY::Q0 + s * LY::TILE;
-        const uint32_t kb = sb + LY::RING + kslot * LY::TILE;
+        // descriptors of k-step 0; step kk moves the start address by off(kk)
+        // (the address field holds addr >> 4 in its low bits)
+        const uint64_t dq = smem_desc_sw128(sb + LY::Q0 + s * LY::TILE, 16, 1024);
+        const uint64_t dk = smem_desc_sw128(sb + LY::RING + kslot * LY::TILE, 16, 1024);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * LY::BOX + (kk & 3) * 32;
-          mma_f16kind_ss(tS(s), smem_desc_sw128(qa + off, 16, 1024), smem_desc_sw128(kb + off, 16, 1024),
-                         IDESC_QK, kk > 0 ? 1u : 0u);
+          const uint64_t off = static_cast<uint64_t>(((kk >> 2) * LY::BOX + (kk & 3) * 32) >> 4);
+          mma_f16kind_ss(tS(s), dq + off, dk + off, IDESC_QK, kk > 0 ? 1u : 0u);
         }
         mma_commit(bar(LY::kSFull + s));
       };
       auto pv = [&](int s, uint32_t vslot, bool acc) {
-        const uint32_t vb = sb + LY::RING + vslot * LY::TILE;
+        const uint64_t dv = smem_desc_sw128(sb + LY::RING + vslot * LY::TILE, LY::BOX, 1024);
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk)  // P of keys [16kk, 16kk+16): half kk/4's columns
           mma_f16kind_ts(tO(s), tS(s) + (kk >> 2) * HBN + (kk & 3) * 8,
-                         smem_desc_sw128(vb + kk * 16 * 128, LY::BOX, 1024), IDESC_PV,
+                         dv + static_cast<uint64_t>((kk * 16 * 128) >> 4), IDESC_PV,
                          (acc || kk > 0) ? 1u : 0u);
       };
       bool ok = wait_or_abort(bar(LY::kQFull + 0), 0u, abort);
