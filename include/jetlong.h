@@ -252,6 +252,20 @@ JL_API int jetlong_rope_cache(const void *k, void *k_cache, int B, int n, int Hk
  */
 JL_API int jetlong_device_status(jl_stream_t stream);
 
+/*
+ * Diagnostic for the failure path above (no counterpart in the paper).
+ * Launches one thread that waits on a shared-memory mbarrier no one ever
+ * arrives at, with the same bounded wait the attention kernels use, here
+ * limited to limit_ms milliseconds (1 <= limit_ms <= 2000).  The wait gives
+ * up and records JL_ERR_DEVICE_TIMEOUT exactly as an expired wait in a real
+ * kernel does; the next jetlong_device_status() returns it and clears it.
+ * Nothing faults or hangs, and the context stays usable.  Note that a
+ * prefill launched while the report is set ends at once without computing
+ * (it honours the earlier failure), so read the status first.
+ * Returns JL_OK if launched, JL_ERR_SHAPE for a limit out of range.
+ */
+JL_API int jetlong_check_device_timeout(int limit_ms, jl_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

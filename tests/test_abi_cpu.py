@@ -141,6 +141,11 @@ def test_three_pass_needs_room_for_the_pass_outputs(lib):
     assert three_pass_call(lib, wsb=three - 1) == jl.JL_ERR_WORKSPACE
 
 
+@pytest.mark.parametrize("limit_ms", [0, -1, 2001])
+def test_timeout_check_rejects_limits_out_of_range(lib, limit_ms):
+    assert lib.jetlong_check_device_timeout(limit_ms, None) == jl.JL_ERR_SHAPE
+
+
 def decode_call(lib, **kw):
     a = dict(q=P, kc=P, vc=P, out=P, lse=None, B=1, Hq=32, Hkv=8, L=1000, Lcap=1000, D=128,
              wp=32768, w0=4096, theta=1e6, od=0, ws=P, wsb=1 << 40, stream=None)

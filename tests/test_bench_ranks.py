@@ -48,6 +48,38 @@ def test_two_rank_reductions():
         assert f == want_f
 
 
+def _failing_worker(rank, world, port, q):
+    import datetime
+
+    import torch.distributed as dist
+    os.environ.update(RANK=str(rank), WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank,
+                            world_size=world, timeout=datetime.timedelta(seconds=5))
+    if rank == 1:
+        os._exit(3)  # this rank dies before the timing reduction
+    try:
+        bench.reduce_max(1.0, world)
+        q.put("completed")
+    except Exception as e:  # noqa: BLE001 - any error is the expected outcome
+        q.put(f"error: {type(e).__name__}")
+
+
+def test_a_dead_rank_ends_the_others_reduction_with_an_error():
+    # The survivor's collective fails (peer gone or the short process-group
+    # timeout), so the job ends instead of waiting forever.
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_failing_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+    assert procs[1].exitcode == 3
+    assert procs[0].exitcode is not None, "surviving rank hung"
+    assert q.get(timeout=10).startswith("error")
+
+
 def test_single_rank_is_identity():
     assert bench.reduce_max(3.5, 1) == 3.5
     assert bench.reduce_sum(7.0, 1) == 7.0

@@ -8,6 +8,7 @@
 
 #include "../../include/jetlong.h"
 #include "jl_common.cuh"
+#include "sm100_ptx.cuh"
 
 namespace jl {
 
@@ -20,6 +21,16 @@ namespace {
 constexpr size_t kAlign = 256;
 
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+// One thread waits on an mbarrier that never completes, bounded by limit_ns,
+// and records the timeout the way the attention kernels do.
+__global__ void wait_timeout_check_kernel(unsigned int *dev_error, unsigned long long limit_ns) {
+  __shared__ __align__(8) unsigned long long barrier_word;
+  const uint32_t bar = smem_u32(&barrier_word);
+  mbar_init(bar, 1);
+  fence_mbar_init();
+  if (!mbar_wait_bounded(bar, 0u, limit_ns)) atomicOr(dev_error, kDevTimeout);
+}
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -350,6 +361,16 @@ int jetlong_rope_cache(const void *k, void *k_cache, int B, int n, int Hkv, int 
                         reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
     return JL_ERR_CUDA;
   return JL_OK;
+}
+
+int jetlong_check_device_timeout(int limit_ms, jl_stream_t stream) {
+  if (limit_ms < 1 || limit_ms > 2000) return JL_ERR_SHAPE;
+  DeviceState *dev = nullptr;
+  const int st = current_device(&dev);
+  if (st != JL_OK) return st;
+  wait_timeout_check_kernel<<<1, 1, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      dev->err, static_cast<unsigned long long>(limit_ms) * 1000000ull);
+  return cudaGetLastError() == cudaSuccess ? JL_OK : JL_ERR_CUDA;
 }
 
 int jetlong_device_status(jl_stream_t stream) {

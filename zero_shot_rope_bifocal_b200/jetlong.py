@@ -54,6 +54,7 @@ SIGNATURES = {
                                     _I, _VP]),
     "jetlong_rope_cache": (_I, [_VP, _VP, _I, _I, _I, _I, _I, _I, _F, _VP]),
     "jetlong_device_status": (_I, [_VP]),
+    "jetlong_check_device_timeout": (_I, [_I, _VP]),
 }
 
 _lib = None
@@ -307,6 +308,13 @@ def jetlong_rope_cache(k, k_cache, pos0: int, rope_theta: float, *, stream=None)
                                   float(rope_theta), _stream_ptr(stream))
     _check("jetlong_rope_cache", st)
     return k_cache
+
+
+def jetlong_check_device_timeout(limit_ms: int = 50, *, stream=None) -> None:
+    """Launch the bounded-wait timeout check (a wait that nothing completes);
+    the next jetlong_device_status() returns JL_ERR_DEVICE_TIMEOUT."""
+    _check("jetlong_check_device_timeout",
+           lib().jetlong_check_device_timeout(int(limit_ms), _stream_ptr(stream)))
 
 
 def jetlong_device_status(stream=None) -> int:
