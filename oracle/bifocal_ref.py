@@ -52,6 +52,7 @@ __all__ = [
     "prefill_rows",
     "prefill_literal",
     "decode",
+    "prefill_chunk",
     "merge_three_pass",
 ]
 
@@ -304,6 +305,60 @@ def decode(q, k_cache, v_cache, L: int, w_pretrained: int, w0: int, theta: float
             tot = e.sum(axis=0)
             lse[b, heads] = m + np.log(tot)
             o[b, heads, :] = (e / tot).T @ vv
+    return o, lse
+
+
+# --------------------------------------------------------------------------
+# Chunked prefill on the true-position cache (§3.1 schedule, §3.2 cache)
+# --------------------------------------------------------------------------
+def prefill_chunk(q, k_cache, v_cache, P0: int, w_pretrained: int, w0: int, theta: float):
+    """A chunk of n new tokens at positions P0 .. P0+n-1 appended to a prompt.
+
+    q: [B, n, Hq, D] pre-RoPE queries of the chunk.  k_cache / v_cache:
+    [B, >=P0+n, Hkv, D], rows [0, P0+n) valid, keys at true positions (the
+    chunk's own keys already appended, §3.2).  One G for the call, from the
+    length after the chunk, L = P0 + n (§3.1: G follows the current sequence
+    length; one G per prefill call).  Query i sits at p = P0 + i and sees keys
+    j <= p, scored like a decode step with that G:
+
+      local  (p - j <= w0): s = RoPE(x_q, p) . k_cache[j]
+      remote (p - j >  w0): s = RoPE(x_q, f(p)) . R(f(j) - j) k_cache[j]
+
+    scaled by 1/sqrt(D).  Returns (o [B, n, Hq, D], lse [B, Hq, n]), float64.
+    With P0 = 0 and n = L this is the whole-prompt prefill.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    kc = np.asarray(k_cache)
+    vc = np.asarray(v_cache)
+    B, n, Hq, D = q.shape
+    Hkv = kc.shape[2]
+    L = P0 + n
+    if kc.shape[1] < L or vc.shape[:3] != kc.shape[:3]:
+        raise ValueError("cache shorter than P0 + n")
+    grp = Hq // Hkv
+    G = group_size(L, w_pretrained)
+    scale = 1.0 / math.sqrt(D)
+    o = np.zeros((B, n, Hq, D))
+    lse = np.zeros((B, Hq, n))
+    jpos_all = np.arange(L, dtype=np.int64)
+    for b in range(B):
+        for g in range(Hkv):
+            c_all = kc[b, :L, g, :].astype(np.float64)
+            v_all = vc[b, :L, g, :].astype(np.float64)
+            c_corr_all = correction_rotate(c_all, jpos_all, G, theta)
+            heads = np.arange(g * grp, (g + 1) * grp)
+            for i in range(n):
+                p = P0 + i
+                c, cc, vv = c_all[: p + 1], c_corr_all[: p + 1], v_all[: p + 1]
+                local = (p - jpos_all[: p + 1]) <= w0
+                q_true = rope(q[b, i, heads], np.int64(p), theta)
+                q_remote = rope(q[b, i, heads], remap(np.int64(p), G), theta)
+                s = np.where(local[:, None], c @ q_true.T, cc @ q_remote.T) * scale
+                m = s.max(axis=0)
+                e = np.exp(s - m)
+                tot = e.sum(axis=0)
+                lse[b, heads, i] = m + np.log(tot)
+                o[b, i, heads, :] = (e / tot).T @ vv
     return o, lse
 
 

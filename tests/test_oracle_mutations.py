@@ -34,10 +34,11 @@ def mutated(func_name, old, new):
 
 
 def some_pin_fails(tests):
+    # a pin that fails an assertion, or that the mutant makes raise, caught it
     for t in tests:
         try:
             t()
-        except AssertionError:
+        except Exception:  # noqa: BLE001
             return True
     return False
 
@@ -56,6 +57,12 @@ PREFILL_PINS = [
 def decode_pins():
     return [lambda L=L: pins.test_decode_equals_last_prefill_row(L) for L in (129, 300, 512)] + [
         pins.test_decode_group_transition_page_boundary]
+
+
+def chunk_pins():
+    return [pins.test_chunk_of_the_whole_prompt_is_the_prefill,
+            lambda: pins.test_chunk_tail_rows_are_the_prefill_rows(300),
+            pins.test_one_token_chunk_is_a_decode_step]
 
 
 MUTANTS = [
@@ -96,6 +103,12 @@ MUTANTS = [
     ("decode", "q_remote = rope(q[b, heads], remap(np.int64(p), G), theta)",
      "q_remote = rope(q[b, heads], np.int64(p), theta)", decode_pins()),
     ("rope_cache", "+ int(pos0)", "+ int(pos0) + 1", [pins.test_rope_cache_offset] + decode_pins()),
+    # chunked prefill
+    ("prefill_chunk", "G = group_size(L, w_pretrained)", "G = group_size(P0 + 1, w_pretrained)",
+     chunk_pins()),
+    ("prefill_chunk", "                p = P0 + i\n", "                p = P0 + i + 1\n", chunk_pins()),
+    ("prefill_chunk", "c, cc, vv = c_all[: p + 1], c_corr_all[: p + 1], v_all[: p + 1]",
+     "c, cc, vv = c_all[:p], c_corr_all[:p], v_all[:p]", chunk_pins()),
 ]
 
 

@@ -334,3 +334,40 @@ def test_decode_group_transition_page_boundary():
         od, ld = oracle.decode(q[:, L - 1], cache, v, L, wp, w0, theta)
         o, lse = oracle.prefill_rows(q[:, :L], k[:, :L], v[:, :L], wp, w0, theta, [L - 1])
         np.testing.assert_allclose(od, o[:, 0], atol=1e-10)
+
+
+# ---------------------------------------------------------------- chunked prefill
+def test_chunk_of_the_whole_prompt_is_the_prefill():
+    # The cache formulation (keys stored at true positions, remote scores via
+    # the correction rotation R(f(j) - j), §3.2) against the direct rule of §3
+    # on pre-RoPE keys: two independent routes to the same numbers.
+    w, q, k, v = tiny_inputs("tiny")
+    cache = oracle.rope_cache(k, 0, w.theta)
+    oc, lc = oracle.prefill_chunk(q, cache, v, 0, w.w_pretrained, w.w0, w.theta)
+    o, lse = oracle.prefill(q, k, v, w.w_pretrained, w.w0, w.theta)
+    np.testing.assert_allclose(oc, o, atol=1e-10)
+    np.testing.assert_allclose(lc, lse, atol=1e-10)
+
+
+@pytest.mark.parametrize("P0", [1, 128, 300, 511])
+def test_chunk_tail_rows_are_the_prefill_rows(P0):
+    # A chunk that ends at L uses G(L), the prefill's G, so its rows are the
+    # prefill's rows P0..L-1 (G(P0) differs from G(L) for P0 = 300: 3 vs 4).
+    w, q, k, v = tiny_inputs("tiny")
+    L = q.shape[1]
+    cache = oracle.rope_cache(k, 0, w.theta)
+    oc, lc = oracle.prefill_chunk(q[:, P0:], cache, v, P0, w.w_pretrained, w.w0, w.theta)
+    o, lse = oracle.prefill_rows(q, k, v, w.w_pretrained, w.w0, w.theta, list(range(P0, L)))
+    np.testing.assert_allclose(oc, o, atol=1e-10)
+    np.testing.assert_allclose(lc, lse, atol=1e-10)
+
+
+def test_one_token_chunk_is_a_decode_step():
+    w, q, k, v = tiny_inputs("tiny")
+    cache = oracle.rope_cache(k, 0, w.theta)
+    for L in (97, 300, 512):
+        oc, lc = oracle.prefill_chunk(q[:, L - 1:L], cache, v, L - 1, w.w_pretrained, w.w0,
+                                      w.theta)
+        od, ld = oracle.decode(q[:, L - 1], cache, v, L, w.w_pretrained, w.w0, w.theta)
+        np.testing.assert_allclose(oc[:, 0], od, atol=1e-12)
+        np.testing.assert_allclose(lc[:, :, 0], ld, atol=1e-12)
