@@ -179,6 +179,34 @@ JL_API int jetlong_prefill_three_pass(const void *q, const void *k, const void *
                                       jl_stream_t stream);
 
 /*
+ * A prefill chunk: n new tokens at positions P0 .. P0+n-1 appended to a
+ * prompt whose cache already holds them (Jet-Long paper, §3.1 and §3.2; the
+ * chunk's keys written first, e.g. with jetlong_rope_cache).  One G for the
+ * call, from the length after the chunk, L = P0 + n.  Query i sits at
+ * p = P0 + i and sees keys [0, p]: local keys (p - j <= w0) as cached,
+ * older keys turned by the correction rotation R(f(j) - j) and scored
+ * against RoPE(x_q, f(p)).  With P0 = 0 and n = L this equals jetlong_prefill
+ * on the same data.  Runs on the split-KV decode kernels (a chunk is n
+ * decode problems over one cache), so its cost grows with n * L.
+ *
+ *   q       [B, n, Hq, D] BF16 pre-RoPE queries of the chunk (read)
+ *   k_cache [B, Lcap, Hkv, D] BF16, RoPE at true positions, rows [0, P0+n)
+ *   v_cache [B, Lcap, Hkv, D] BF16 (read)
+ *   out     [B, n, Hq, D] out_dtype (written); lse [B, Hq, n] float32 (may be NULL)
+ *   P0 >= 0, n >= 1, P0 + n <= Lcap, B * n <= 65535; Hq / Hkv in {1, 2, 4, 8}.
+ *   workspace: at least jetlong_prefill_chunk_workspace_size(...) bytes,
+ *       256-byte aligned.
+ * Returns JL_OK or an error code (nothing launched on error).
+ */
+JL_API size_t jetlong_prefill_chunk_workspace_size(int B, int Hq, int Hkv, int P0, int n, int D);
+
+JL_API int jetlong_prefill_chunk(const void *q, const void *k_cache, const void *v_cache,
+                                 void *out, float *lse, int B, int Hq, int Hkv, int P0, int n,
+                                 int Lcap, int D, int w_pretrained, int w0, float rope_theta,
+                                 int out_dtype, void *workspace, size_t workspace_bytes,
+                                 jl_stream_t stream);
+
+/*
  * Bytes of workspace jetlong_decode needs for a cache of L tokens (host only).
  * Non-decreasing in L: sizing it for the largest L a generation loop will reach
  * covers every earlier step.  Returns 0 if a size is invalid.

@@ -146,6 +146,38 @@ def test_timeout_check_rejects_limits_out_of_range(lib, limit_ms):
     assert lib.jetlong_check_device_timeout(limit_ms, None) == jl.JL_ERR_SHAPE
 
 
+def chunk_call(lib, **kw):
+    a = dict(q=P, kc=P, vc=P, out=P, lse=None, B=1, Hq=32, Hkv=8, P0=1000, n=64, Lcap=1064,
+             D=128, wp=32768, w0=4096, theta=1e6, od=0, ws=P, wsb=1 << 40, stream=None)
+    a.update(kw)
+    return lib.jetlong_prefill_chunk(a["q"], a["kc"], a["vc"], a["out"], a["lse"], a["B"], a["Hq"],
+                                     a["Hkv"], a["P0"], a["n"], a["Lcap"], a["D"], a["wp"],
+                                     a["w0"], a["theta"], a["od"], a["ws"], a["wsb"], a["stream"])
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(q=None), jl.JL_ERR_NULL),
+    (dict(n=0), jl.JL_ERR_SHAPE),
+    (dict(P0=-1), jl.JL_ERR_SHAPE),
+    (dict(Lcap=1063), jl.JL_ERR_SHAPE),            # P0 + n > Lcap
+    (dict(B=2, n=40000, Lcap=41000), jl.JL_ERR_SHAPE),  # B * n > 65535
+    (dict(Hq=48), jl.JL_ERR_UNSUPPORTED),
+    (dict(D=96), jl.JL_ERR_UNSUPPORTED),
+    (dict(out=ctypes.c_void_p(260)), jl.JL_ERR_ALIGN),
+    (dict(wsb=0), jl.JL_ERR_WORKSPACE),
+])
+def test_prefill_chunk_rejects_bad_arguments(lib, kw, status):
+    assert chunk_call(lib, **kw) == status
+
+
+def test_chunk_workspace_covers_a_decode_step():
+    # a one-token chunk is a decode step: same plan, same workspace
+    for L in (1, 1000, 131072):
+        assert (jl.jetlong_prefill_chunk_workspace_size(1, 32, 8, L - 1, 1, 128) ==
+                jl.jetlong_decode_workspace_size(1, 32, 8, L, 128))
+    assert jl.jetlong_prefill_chunk_workspace_size(1, 32, 8, 0, 0, 128) == 0
+
+
 def decode_call(lib, **kw):
     a = dict(q=P, kc=P, vc=P, out=P, lse=None, B=1, Hq=32, Hkv=8, L=1000, Lcap=1000, D=128,
              wp=32768, w0=4096, theta=1e6, od=0, ws=P, wsb=1 << 40, stream=None)

@@ -15,6 +15,8 @@ from .jetlong import (  # noqa: F401
     jetlong_group_size,
     jetlong_prefill,
     jetlong_prefill_attend,
+    jetlong_prefill_chunk,
+    jetlong_prefill_chunk_workspace_size,
     jetlong_prefill_rotate,
     jetlong_prefill_three_pass,
     jetlong_prefill_three_pass_workspace_size,

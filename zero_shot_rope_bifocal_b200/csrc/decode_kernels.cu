@@ -33,6 +33,11 @@
 // running max and sum; a second kernel (launched as a programmatic dependent
 // of the first) merges the partials by log-sum-exp, one CTA per head.
 //
+// The same kernels run a prefill chunk (§3.1, §3.2): n queries at positions
+// P0 .. P0+n-1 are n problems over one cache (grid z = batch x query), each
+// over keys [0, its position], with one G for the call; splits past a
+// query's last key write empty partials, which the combine weighs by zero.
+//
 // Traffic: K and V once (2 * L * Hkv * D * 2 bytes per token of output);
 // everything else is O(Hq * D * n_split).
 #include <cmath>
@@ -225,15 +230,16 @@ decode_split_kernel(DecodeArgs a) {
   auto empty = [&](int slot) { return sb + C::BAR + 8u * static_cast<uint32_t>(kStages + slot); };
   auto tready = [&](int slot) { return sb + C::BAR + 8u * static_cast<uint32_t>(2 * kStages + slot); };
 
-  const int s = blockIdx.x, chunk_id = blockIdx.y, b = blockIdx.z;
+  const int s = blockIdx.x, chunk_id = blockIdx.y, bq = blockIdx.z;  // bq = b * nq + query
+  const int b = bq / a.nq;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g0 = chunk_id * kDecWarps;
   const int nh = min(kDecWarps, a.Hkv - g0);  // KV heads of this CTA = working warps
-  const int p = a.L - 1;
+  const int p = a.q_pos0 + (bq - b * a.nq);  // this query's position; keys [0, p]
   const int G = a.G;
   const int w0eff = (G == 1) ? INT_MAX : a.w0;
   const int j_begin = s * a.chunk;
-  const int j_end = min(a.L, j_begin + a.chunk);
+  const int j_end = min(p + 1, j_begin + a.chunk);  // may be <= j_begin: an empty split
   const int n_stage = (j_end - j_begin + P - 1) / P;
   const uint32_t head_bytes = static_cast<uint32_t>(nh) * D * 2;  // one token, CTA heads
   const size_t cache_row = static_cast<size_t>(a.Hkv) * D;        // elements per token
@@ -316,7 +322,7 @@ decode_split_kernel(DecodeArgs a) {
   uint32_t qt[KB][2], qr[KB][2];
   {
     const bool qrow_ok = gq < GRP;
-    const __nv_bfloat16 *qrow = a.q + (static_cast<size_t>(b) * a.Hq + g * GRP + (qrow_ok ? gq : 0)) * D;
+    const __nv_bfloat16 *qrow = a.q + (static_cast<size_t>(bq) * a.Hq + g * GRP + (qrow_ok ? gq : 0)) * D;
 #pragma unroll
     for (int kb = 0; kb < KB / 2; ++kb)
 #pragma unroll
@@ -470,7 +476,7 @@ decode_split_kernel(DecodeArgs a) {
   // Partial record per query head: [D] unnormalised output, then the running
   // max (base 2) and sum.
   const size_t rec_stride = static_cast<size_t>(a.n_split) * (D + 2);
-  float *rec0 = a.partial + ((static_cast<size_t>(b) * a.Hq + g * GRP) * a.n_split + s) * (D + 2);
+  float *rec0 = a.partial + ((static_cast<size_t>(bq) * a.Hq + g * GRP) * a.n_split + s) * (D + 2);
 #pragma unroll
   for (int e = 0; e < 2; ++e) {
     const int h = 2 * tq + e;  // O^T column = query head of the group
@@ -571,7 +577,11 @@ decode_combine_kernel(DecodeArgs a) {
     else
       reinterpret_cast<__nv_bfloat16 *>(a.out)[idx] = __float2bfloat16_rn(o * inv);
   }
-  if (tid == 0 && a.lse) a.lse[bh] = (M + log2f(lsum)) * 0.69314718055994531f;
+  if (tid == 0 && a.lse) {  // lse is [B, Hq, nq]
+    const int h = bh % a.Hq, bqi = bh / a.Hq;
+    const int bb = bqi / a.nq, qi = bqi - bb * a.nq;
+    a.lse[(static_cast<size_t>(bb) * a.Hq + h) * a.nq + qi] = (M + log2f(lsum)) * 0.69314718055994531f;
+  }
 }
 
 template <int D, int GRP>
@@ -581,7 +591,7 @@ cudaError_t launch_split(const DecodeArgs &a, cudaStream_t stream) {
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   const int n_chunk = (a.Hkv + kDecWarps - 1) / kDecWarps;
-  decode_split_kernel<D, GRP><<<dim3(a.n_split, n_chunk, a.B), kDecThreads, smem, stream>>>(a);
+  decode_split_kernel<D, GRP><<<dim3(a.n_split, n_chunk, a.B * a.nq), kDecThreads, smem, stream>>>(a);
   return cudaGetLastError();
 }
 
@@ -598,7 +608,7 @@ cudaError_t launch_decode_d(const DecodeArgs &a, cudaStream_t stream) {
   if (e != cudaSuccess) return e;
   if (a.n_split > kMaxSplit) return cudaErrorInvalidValue;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(a.B * a.Hq));
+  cfg.gridDim = dim3(static_cast<unsigned>(a.B * a.nq * a.Hq));
   cfg.blockDim = dim3(kCombineThreads);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = stream;

@@ -300,13 +300,26 @@ size_t jetlong_decode_workspace_size(int B, int Hq, int Hkv, int L, int D) {
   return decode_ws_bytes(B, Hq, Hkv, L, D);
 }
 
-int jetlong_decode(const void *q, const void *k_cache, const void *v_cache, void *out, float *lse,
-                   int B, int Hq, int Hkv, int L, int Lcap, int D, int w_pretrained, int w0,
-                   float rope_theta, int out_dtype, void *workspace, size_t workspace_bytes,
-                   jl_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+// Queries at positions q_pos0 .. q_pos0 + nq - 1 (per batch entry) against the
+// true-position cache, each over keys [0, its position], with one G from the
+// longest range L = q_pos0 + nq: a decode step (nq = 1) or a prefill chunk.
+int cache_attention(const void *q, const void *k_cache, const void *v_cache, void *out, float *lse,
+                    int B, int Hq, int Hkv, int nq, int q_pos0, int Lcap, int D, int w_pretrained,
+                    int w0, float rope_theta, int out_dtype, void *workspace,
+                    size_t workspace_bytes, jl_stream_t stream) {
   if (!q || !k_cache || !v_cache || !out) return JL_ERR_NULL;
+  if (nq < 1 || q_pos0 < 0) return JL_ERR_SHAPE;
+  const long long L_ll = static_cast<long long>(q_pos0) + nq;
+  if (L_ll > (1ll << 31) - 1) return JL_ERR_SHAPE;
+  const int L = static_cast<int>(L_ll);
   int st = check_common(B, Hq, Hkv, L, D);
   if (st != JL_OK) return st;
+  if (static_cast<long long>(B) * nq > 65535) return JL_ERR_SHAPE;  // grid z of the split kernel
+  if (static_cast<long long>(B) * nq * Hq * L > (1ll << 40)) return JL_ERR_SHAPE;
   if (Lcap < L) return JL_ERR_SHAPE;
   if (!decode_supports_group(Hq / Hkv)) return JL_ERR_UNSUPPORTED;
   if ((st = check_method(w_pretrained, w0, rope_theta)) != JL_OK) return st;
@@ -314,7 +327,7 @@ int jetlong_decode(const void *q, const void *k_cache, const void *v_cache, void
   if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out) ||
       (lse && !aligned16(lse)))
     return JL_ERR_ALIGN;
-  const size_t need = decode_ws_bytes(B, Hq, Hkv, L, D);
+  const size_t need = decode_ws_bytes(B * nq, Hq, Hkv, L, D);
   if (!workspace || workspace_bytes < need) return JL_ERR_WORKSPACE;
   if (reinterpret_cast<uintptr_t>(workspace) % kAlign) return JL_ERR_ALIGN;
 
@@ -339,10 +352,42 @@ int jetlong_decode(const void *q, const void *k_cache, const void *v_cache, void
   a.w0 = w0;
   a.G = group_size(L, w_pretrained);
   a.theta = rope_theta;
-  decode_plan(B, Hkv, L, &a.n_split, &a.chunk);
+  a.nq = nq;
+  a.q_pos0 = q_pos0;
+  decode_plan(B * nq, Hkv, L, &a.n_split, &a.chunk);
   a.dev_error = dev->err;
   if (launch_decode(a, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return JL_ERR_CUDA;
   return JL_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int jetlong_decode(const void *q, const void *k_cache, const void *v_cache, void *out, float *lse,
+                   int B, int Hq, int Hkv, int L, int Lcap, int D, int w_pretrained, int w0,
+                   float rope_theta, int out_dtype, void *workspace, size_t workspace_bytes,
+                   jl_stream_t stream) {
+  if (L < 1) return JL_ERR_SHAPE;
+  return cache_attention(q, k_cache, v_cache, out, lse, B, Hq, Hkv, 1, L - 1, Lcap, D,
+                         w_pretrained, w0, rope_theta, out_dtype, workspace, workspace_bytes,
+                         stream);
+}
+
+size_t jetlong_prefill_chunk_workspace_size(int B, int Hq, int Hkv, int P0, int n, int D) {
+  if (n < 1 || P0 < 0 || static_cast<long long>(P0) + n > (1ll << 31) - 1) return 0;
+  if (check_common(B, Hq, Hkv, P0 + n, D) != JL_OK) return 0;
+  if (static_cast<long long>(B) * n > 65535) return 0;
+  return decode_ws_bytes(B * n, Hq, Hkv, P0 + n, D);
+}
+
+int jetlong_prefill_chunk(const void *q, const void *k_cache, const void *v_cache, void *out,
+                          float *lse, int B, int Hq, int Hkv, int P0, int n, int Lcap, int D,
+                          int w_pretrained, int w0, float rope_theta, int out_dtype,
+                          void *workspace, size_t workspace_bytes, jl_stream_t stream) {
+  return cache_attention(q, k_cache, v_cache, out, lse, B, Hq, Hkv, n, P0, Lcap, D,
+                         w_pretrained, w0, rope_theta, out_dtype, workspace, workspace_bytes,
+                         stream);
 }
 
 int jetlong_rope_cache(const void *k, void *k_cache, int B, int n, int Hkv, int D, int pos0,

@@ -104,6 +104,11 @@ struct DecodeArgs {
   int B, Hq, Hkv, L, Lcap, D, w_pretrained, w0, G;
   float theta;
   int n_split, chunk;
+  // Queries per batch entry and the position of the first: a decode step has
+  // nq = 1 at q_pos0 = L - 1; a prefill chunk has nq = n at q_pos0 = P0, and
+  // query i sees keys [0, q_pos0 + i].  q is [B, nq, Hq, D], out likewise,
+  // lse [B, Hq, nq]; L is the longest key range, q_pos0 + nq.
+  int nq, q_pos0;
   unsigned int *dev_error;
 };
 

@@ -48,6 +48,9 @@ SIGNATURES = {
     "jetlong_prefill_three_pass": (_I, [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _I, _F,
                                         _I, _VP, _SZ, _VP]),
     "jetlong_decode_workspace_size": (_SZ, [_I, _I, _I, _I, _I]),
+    "jetlong_prefill_chunk_workspace_size": (_SZ, [_I, _I, _I, _I, _I, _I]),
+    "jetlong_prefill_chunk": (_I, [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _I, _I, _I,
+                                   _F, _I, _VP, _SZ, _VP]),
     "jetlong_decode": (_I, [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _I, _I, _F, _I,
                             _VP, _SZ, _VP]),
     "jetlong_decode_noalloc": (_I, [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _I, _I, _F,
@@ -274,6 +277,42 @@ def jetlong_decode(q, k_cache, v_cache, L: int, w_pretrained: int, w0: int, rope
                               Hkv, int(L), Lcap, D, int(w_pretrained), int(w0), float(rope_theta),
                               od, _ptr(workspace), workspace.numel(), _stream_ptr(stream))
     _check("jetlong_decode", st)
+    return out, lse
+
+
+def jetlong_prefill_chunk_workspace_size(B, Hq, Hkv, P0, n, D) -> int:
+    return int(lib().jetlong_prefill_chunk_workspace_size(B, Hq, Hkv, P0, n, D))
+
+
+def jetlong_prefill_chunk(q, k_cache, v_cache, P0: int, w_pretrained: int, w0: int,
+                          rope_theta: float, *, out=None, lse=None, out_dtype=torch.bfloat16,
+                          want_lse: bool = True, workspace=None, stream=None):
+    """Queries of a chunk at positions P0.. against a true-position cache that
+    already holds the chunk's keys; one G from P0 + n.  Returns (out, lse)."""
+    if q.dim() != 4 or k_cache.dim() != 4:
+        raise ValueError("q must be [B, n, Hq, D] and the caches [B, Lcap, Hkv, D]")
+    B, n, Hq, D = q.shape
+    Lcap, Hkv = k_cache.shape[1], k_cache.shape[2]
+    _require(q, "q", (B, n, Hq, D), torch.bfloat16)
+    _require(k_cache, "k_cache", (B, Lcap, Hkv, D), torch.bfloat16)
+    _require(v_cache, "v_cache", (B, Lcap, Hkv, D), torch.bfloat16)
+    od = _out_dtype(out_dtype if out is None else out.dtype)
+    if out is None:
+        out = torch.empty((B, n, Hq, D), dtype=torch.bfloat16 if od == JL_BF16 else torch.float32,
+                          device=q.device)
+    _require(out, "out", (B, n, Hq, D), out.dtype)
+    if lse is None and want_lse:
+        lse = torch.empty((B, Hq, n), dtype=torch.float32, device=q.device)
+    if lse is not None:
+        _require(lse, "lse", (B, Hq, n), torch.float32)
+    if workspace is None:
+        workspace = _ws(jetlong_prefill_chunk_workspace_size(B, Hq, Hkv, int(P0), n, D),
+                        q.device)
+    st = lib().jetlong_prefill_chunk(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(out), _ptr(lse),
+                                     B, Hq, Hkv, int(P0), n, Lcap, D, int(w_pretrained), int(w0),
+                                     float(rope_theta), od, _ptr(workspace), workspace.numel(),
+                                     _stream_ptr(stream))
+    _check("jetlong_prefill_chunk", st)
     return out, lse
 
 
