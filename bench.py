@@ -229,6 +229,15 @@ def threads_used() -> int:
 
 
 # ---------------------------------------------------------------- reference arm
+def workload_config(w, world: int) -> dict:
+    """The ``config`` both arms report for the headline prefill workload."""
+    return {"workload": PREFILL_WORKLOAD, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D, "L": w.L,
+            "w_pretrained": w.w_pretrained, "w0": w.w0, "rope_theta": w.theta,
+            "G": -(-w.L // w.w_pretrained) if w.L > w.w_pretrained else 1,
+            "l2": "inputs larger than L2 (q 1 GiB, k/v 256 MiB each); no flush",
+            "parallelism": f"independent layer per rank x{world}"}
+
+
 def run_reference(args):
     rank, world, _ = dist_env()
     if rank != 0:
@@ -252,8 +261,7 @@ def run_reference(args):
         "warmup": args.warmup, "ms_per_step": 1e3 * tot_t / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded N(0,1) Q/K/V, K per-channel LogNormal(0,0.5) scale)",
-        "config": {"workload": PREFILL_WORKLOAD, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D,
-                   "L": w.L, "w_pretrained": w.w_pretrained, "w0": w.w0, "rope_theta": w.theta},
+        "config": workload_config(w, world),
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads_used(),
                          "kind": "oracle",
                          "sample": f"{nrows} query rows (all 32 heads) of the 128K prefill, "
@@ -524,11 +532,7 @@ def run_native(args):
             "precision": "BF16 inputs and outputs; FP16 tensor-core operands (rotated Q/K, V, "
                          "P) with FP32 accumulation; FP32 softmax statistics",
             "data": "synthetic (seeded N(0,1) Q/K/V, K per-channel LogNormal(0,0.5) scale)",
-            "config": {"workload": PREFILL_WORKLOAD, "B": B, "Hq": Hq, "Hkv": Hkv, "D": D, "L": L,
-                       "w_pretrained": w.w_pretrained, "w0": w.w0, "rope_theta": w.theta,
-                       "G": jl.jetlong_group_size(L, w.w_pretrained),
-                       "l2": "inputs larger than L2 (q 1 GiB, k/v 256 MiB each); no flush",
-                       "parallelism": f"independent layer per rank x{world}"},
+            "config": workload_config(w, world),
             "roofline": {"bound": "tensor", "achieved": attn_tflops, "peak": peak,
                          "unit": "TFLOP/s", "frac": attn_tflops / peak,
                          "peak_source": f"{src} bf16_tflops_sustained",

@@ -89,6 +89,17 @@ JL_API const char *jetlong_status_string(int status);
 JL_API const char *jetlong_version(void);
 
 /*
+ * Forget the per-device state the library keeps on the host (the checked
+ * compute capability and the address of each device's error word); the next
+ * call on a device looks them up again.  The library holds no device
+ * allocation to free: it computes its cos/sin tables inside the kernels and
+ * its only device-side storage is static (the error word and the
+ * jetlong_decode_noalloc buffer).  Call it when no call of this library is
+ * in flight on another thread.
+ */
+JL_API void jetlong_shutdown(void);
+
+/*
  * Dynamic group size of §3.1, Eq. (2): G = max(1, ceil(L / w_pretrained)).
  * Host only, no CUDA call.  Returns G >= 1, or JL_ERR_SHAPE if L < 1 or
  * w_pretrained < 1.

@@ -66,6 +66,12 @@ def test_workspace_sizes(lib):
         prev = cur
 
 
+def test_shutdown_can_be_called_without_a_device(lib):
+    lib.jetlong_shutdown()
+    lib.jetlong_shutdown()
+    assert jl.jetlong_group_size(131072, 32768) == 4
+
+
 def test_status_strings(lib):
     for code in range(-9, 1):
         assert jl.status_string(code).startswith("JL_")

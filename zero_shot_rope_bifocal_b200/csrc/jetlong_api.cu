@@ -136,6 +136,11 @@ const char *jetlong_status_string(int s) {
 
 const char *jetlong_version(void) { return "0.1.0"; }
 
+void jetlong_shutdown(void) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  for (DeviceState &st : g_dev) st = DeviceState{};
+}
+
 int jetlong_group_size(int L, int w_pretrained) {
   if (L < 1 || w_pretrained < 1) return JL_ERR_SHAPE;
   return group_size(L, w_pretrained);

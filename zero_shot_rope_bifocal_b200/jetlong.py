@@ -37,6 +37,7 @@ _VP, _I, _F, _SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_
 SIGNATURES = {
     "jetlong_status_string": (ctypes.c_char_p, [_I]),
     "jetlong_version": (ctypes.c_char_p, []),
+    "jetlong_shutdown": (None, []),
     "jetlong_group_size": (_I, [_I, _I]),
     "jetlong_prefill_workspace_size": (_SZ, [_I, _I, _I, _I, _I]),
     "jetlong_prefill": (_I, [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _I, _F, _I,
