@@ -623,12 +623,14 @@ cudaError_t launch_decode_d(const DecodeArgs &a, cudaStream_t stream) {
 }  // namespace
 
 void decode_plan(int B, int Hkv, int L, int *n_split, int *chunk) {
-  // Two CTAs per SM (each holds a 3-stage ring of about 100 KB) over the 148
+  // Two CTAs per SM (each holds a 3-stage ring of about 108 KB) over the 148
   // SMs of a B200; chunks are whole stages (8 or 16 tokens).  The split count
-  // is non-decreasing in L, so workspace sized for the largest L of a
+  // fills at most one wave of CTAs (rounding up would start a second,
+  // nearly empty wave: 64 units x 5 splits = 320 CTAs for 296 slots).  It is
+  // non-decreasing in L, so workspace sized for the largest L of a
   // generation loop covers every step.
   const int units = B * ((Hkv + kDecWarps - 1) / kDecWarps);
-  int ns = (kCtasPerSm * 148 + units - 1) / units;
+  int ns = (kCtasPerSm * 148) / units;
   const int max_ns = (L + 15) / 16;
   if (ns > max_ns) ns = max_ns;
   if (ns < 1) ns = 1;
