@@ -126,6 +126,22 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   return r;
 }
+__device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
+  float2 d;
+  asm("{.reg .b64 ra, rb, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+__device__ __forceinline__ float2 fsub2(float2 a, float2 b) {
+  float2 d;
+  asm("{.reg .b64 ra, rb, rd;\n\tmov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "sub.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
 __device__ __forceinline__ float bf_lo(uint32_t u) { return __uint_as_float(u << 16); }
 __device__ __forceinline__ float bf_hi(uint32_t u) { return __uint_as_float(u & 0xffff0000u); }
 
@@ -148,9 +164,13 @@ __device__ __forceinline__ void qk_pair(float (&sc)[4], const uint32_t (&q)[D / 
     if constexpr (REMOTE) {
       // lo[r]: channels c, c + 1 with c = 16 (kb0 + r / 2) + 8 (r % 2) + 2 tq
       const int c = 16 * (kb0 + (r >> 1)) + 8 * (r & 1) + 2 * tq;
-      const float4 cs = *reinterpret_cast<const float4 *>(cs_row + c * 8);
-      lo[r] = pack_f16(x0 * cs.x - y0 * cs.y, x1 * cs.z - y1 * cs.w);
-      hi[r] = pack_f16(x0 * cs.y + y0 * cs.x, x1 * cs.w + y1 * cs.z);
+      const float4 cs = *reinterpret_cast<const float4 *>(cs_row + c * 8);  // cos c, c+1, sin c, c+1
+      const float2 xx = make_float2(x0, x1), yy = make_float2(y0, y1);
+      const float2 co = make_float2(cs.x, cs.y), si = make_float2(cs.z, cs.w);
+      const float2 l2 = fsub2(fmul2(xx, co), fmul2(yy, si));  // x cos - y sin
+      const float2 h2 = ffma2(yy, co, fmul2(xx, si));         // x sin + y cos
+      lo[r] = pack_f16(l2.x, l2.y);
+      hi[r] = pack_f16(h2.x, h2.y);
     } else {
       lo[r] = pack_f16(x0, x1);
       hi[r] = pack_f16(y0, y1);
@@ -176,8 +196,9 @@ __device__ __forceinline__ void qk_block(float (&sc)[4], const uint32_t (&q)[D /
   for (int e = 0; e < 4; ++e) sc[e] += acc[0][e] + acc[1][e];
 }
 
-// Rows of the correction table of one stage: (cos, sin) of Delta j * theta_i
-// for token row tt (j = jt + tt) and frequency i < D/2, Delta j = f(j) - j.
+// Rows of the correction table of one stage: cos and sin of Delta j * theta_i
+// for token row tt (j = jt + tt) and frequency i < D/2, Delta j = f(j) - j,
+// stored per channel pair (i, i+1) as (cos_i, cos_i+1, sin_i, sin_i+1).
 // The phase in turns is Delta j * omega_i modulo 1, with omega_i =
 // theta_i / (2 pi) as a 64-bit binary fraction: the 64-bit product wraps
 // exactly, its top 32 bits are the signed phase in units of 2^-32 turn, and
@@ -191,12 +212,14 @@ __device__ __forceinline__ void correction_rows(uint8_t *tab, int jt, int n, int
   for (int tt = warp; tt < n; tt += nw) {
     const int j = jt + tt;
     const uint64_t delta = static_cast<uint64_t>(static_cast<int64_t>(remap(j, G) - j));
-#pragma unroll
-    for (int i = lane; i < D / 2; i += 32) {
-      const int32_t ph = static_cast<int32_t>((delta * omega[i]) >> 32);
-      float c, sn;
-      __sincosf(static_cast<float>(ph) * kTurnToRad, &sn, &c);
-      *reinterpret_cast<float2 *>(tab + tt * C::CS_ROW + i * 8) = make_float2(c, sn);
+    if (lane < D / 4) {  // lane: channels 2 lane, 2 lane + 1
+      const int i = 2 * lane;
+      const int32_t p0 = static_cast<int32_t>((delta * omega[i]) >> 32);
+      const int32_t p1 = static_cast<int32_t>((delta * omega[i + 1]) >> 32);
+      float c0, s0, c1, s1;
+      __sincosf(static_cast<float>(p0) * kTurnToRad, &s0, &c0);
+      __sincosf(static_cast<float>(p1) * kTurnToRad, &s1, &c1);
+      *reinterpret_cast<float4 *>(tab + tt * C::CS_ROW + i * 8) = make_float4(c0, c1, s0, s1);
     }
   }
 }
@@ -217,7 +240,9 @@ __device__ __forceinline__ bool dec_wait(uint32_t bar, uint32_t parity, volatile
   }
 }
 
-template <int D, int GRP>
+// BIFOCAL = false is the G = 1 instantiation: every key is local, so it has
+// no remote query, no correction table and no rotation code.
+template <int D, int GRP, bool BIFOCAL>
 __global__ void __launch_bounds__(kDecThreads, kCtasPerSm)
 decode_split_kernel(DecodeArgs a) {
   using C = DecCfg<D>;
@@ -237,7 +262,7 @@ decode_split_kernel(DecodeArgs a) {
   const int nh = min(kDecWarps, a.Hkv - g0);  // KV heads of this CTA = working warps
   const int p = a.q_pos0 + (bq - b * a.nq);  // this query's position; keys [0, p]
   const int G = a.G;
-  const int w0eff = (G == 1) ? INT_MAX : a.w0;
+  const int w0eff = BIFOCAL ? a.w0 : INT_MAX;
   const int j_begin = s * a.chunk;
   const int j_end = min(p + 1, j_begin + a.chunk);  // may be <= j_begin: an empty split
   const int n_stage = (j_end - j_begin + P - 1) / P;
@@ -309,8 +334,11 @@ decode_split_kernel(DecodeArgs a) {
   }
   __syncthreads();
   if (warp >= nh) return;  // no KV head for this warp; nothing below waits for it
-  bool ok = table(0);
-  if (ok && n_stage > 1) ok = table(1);
+  bool ok = true;
+  if constexpr (BIFOCAL) {
+    ok = table(0);
+    if (ok && n_stage > 1) ok = table(1);
+  }
 
   // Query fragments (A operand, rows = the group's heads, FP16, pre-scaled by
   // log2(e)/sqrt(D)) at the true position p and the remote position f(p).
@@ -362,7 +390,7 @@ decode_split_kernel(DecodeArgs a) {
   for (int t = 0; t < n_stage && ok; ++t) {
     const int jt = j_begin + t * P;
     const int n = min(P, j_end - jt);
-    ok = dec_wait(full(slot), phase, abort) && dec_wait(tready(slot), phase, abort);
+    ok = dec_wait(full(slot), phase, abort) && (!BIFOCAL || dec_wait(tready(slot), phase, abort));
     if (!__all_sync(0xffffffffu, ok)) {
       ok = false;
       break;
@@ -382,7 +410,9 @@ decode_split_kernel(DecodeArgs a) {
         const bool all_remote = p - (jb + 7) > w0eff;
         const bool all_local = p - jb <= w0eff;
         float sc[4] = {0.f, 0.f, 0.f, 0.f};
-        if (all_remote) {
+        if (!BIFOCAL) {
+          qk_block<D, false>(sc, qt, krow, cs_row, tq, mat);
+        } else if (all_remote) {
           qk_block<D, true>(sc, qr, krow, cs_row, tq, mat);
         } else if (all_local) {
           qk_block<D, false>(sc, qt, krow, cs_row, tq, mat);
@@ -445,7 +475,7 @@ decode_split_kernel(DecodeArgs a) {
     __syncwarp();
     if (lane == 0) mbar_arrive(empty(slot));
     // This warp's rows of the table two stages ahead.
-    if (t + 2 < n_stage) ok = table(t + 2);
+    if (BIFOCAL && t + 2 < n_stage) ok = table(t + 2);
     // Warp 0 refills this slot once every warp has released it.
     if (warp == 0 && ok && t + kStages < n_stage) {
       ok = __all_sync(0xffffffffu, dec_wait(empty(slot), phase, abort));
@@ -584,15 +614,20 @@ decode_combine_kernel(DecodeArgs a) {
   }
 }
 
-template <int D, int GRP>
-cudaError_t launch_split(const DecodeArgs &a, cudaStream_t stream) {
+template <int D, int GRP, bool BIFOCAL>
+cudaError_t launch_split_v(const DecodeArgs &a, cudaStream_t stream) {
   const int smem = DecCfg<D>::BYTES;
-  cudaError_t e = cudaFuncSetAttribute(decode_split_kernel<D, GRP>,
+  cudaError_t e = cudaFuncSetAttribute(decode_split_kernel<D, GRP, BIFOCAL>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   const int n_chunk = (a.Hkv + kDecWarps - 1) / kDecWarps;
-  decode_split_kernel<D, GRP><<<dim3(a.n_split, n_chunk, a.B * a.nq), kDecThreads, smem, stream>>>(a);
+  decode_split_kernel<D, GRP, BIFOCAL><<<dim3(a.n_split, n_chunk, a.B * a.nq), kDecThreads, smem, stream>>>(a);
   return cudaGetLastError();
+}
+
+template <int D, int GRP>
+cudaError_t launch_split(const DecodeArgs &a, cudaStream_t stream) {
+  return a.G > 1 ? launch_split_v<D, GRP, true>(a, stream) : launch_split_v<D, GRP, false>(a, stream);
 }
 
 template <int D>
