@@ -617,8 +617,7 @@ decode_combine_kernel(DecodeArgs a) {
 template <int D, int GRP, bool BIFOCAL>
 cudaError_t launch_split_v(const DecodeArgs &a, cudaStream_t stream) {
   const int smem = DecCfg<D>::BYTES;
-  cudaError_t e = cudaFuncSetAttribute(decode_split_kernel<D, GRP, BIFOCAL>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  cudaError_t e = ensure_smem_limit<decode_split_kernel<D, GRP, BIFOCAL>>(smem);
   if (e != cudaSuccess) return e;
   const int n_chunk = (a.Hkv + kDecWarps - 1) / kDecWarps;
   decode_split_kernel<D, GRP, BIFOCAL><<<dim3(a.n_split, n_chunk, a.B * a.nq), kDecThreads, smem, stream>>>(a);

@@ -7,10 +7,28 @@
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <climits>
 #include <cstdint>
 
 namespace jl {
+
+// Sets a kernel's dynamic shared-memory limit once per device (bit `dev` of a
+// per-kernel mask), so later launches make no other CUDA call and can be
+// captured into a CUDA graph.
+template <auto Kernel>
+cudaError_t ensure_smem_limit(int bytes) {
+  static std::atomic<unsigned long long> done{0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return cudaGetLastError();
+  const unsigned long long bit = 1ull << (dev & 63);
+  if (done.load(std::memory_order_acquire) & bit) return cudaSuccess;
+  const cudaError_t e =
+      cudaFuncSetAttribute(Kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) done.fetch_or(bit, std::memory_order_acq_rel);
+  return e;
+}
+
 
 // Kernel-side error bits written to the device error word.
 enum : unsigned int {

@@ -649,8 +649,7 @@ cudaError_t launch_d(const PrefillArgs &a, cudaStream_t stream) {
   prm.out_f32 = a.out_f32;
   prm.dev_error = a.dev_error;
   const int smem = Layout<D>::ALLOC;
-  cudaError_t e = cudaFuncSetAttribute(bifocal_prefill_kernel<D>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  cudaError_t e = ensure_smem_limit<bifocal_prefill_kernel<D>>(smem);
   if (e != cudaSuccess) return e;
   const dim3 grid(prm.n_qt, a.Hkv * prm.npair, a.B);
   bifocal_prefill_kernel<D><<<grid, kThreads, smem, stream>>>(tqt, tqr, tkt, tkr, tv, prm);
