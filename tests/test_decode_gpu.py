@@ -117,3 +117,40 @@ def test_decode_after_prefill_matches_last_row():
     assert_o(f64(out_d), o_ref[:, 0], "decode after prefill")
     assert_lse(f64(lse_d), lse_ref[:, :, 0], "decode after prefill")
     assert_o(f64(out_d), f64(out_p[:, -1]), "decode vs prefill row")
+
+
+def test_decode_calls_replay_from_a_cuda_graph():
+    # After a first (eager) call has set the kernels' shared-memory limits, a
+    # call makes no CUDA API call besides its launches, so a decode loop can
+    # be captured once and replayed; the replay equals the eager calls bit
+    # for bit.
+    w = WORKLOADS["decode_8b_32k"].with_(w_pretrained=8192)  # G = 4 at 32K
+    d = decode_inputs(w)
+    cache = oracle_cache_bf16(d.k_raw, w.theta).cuda()
+    v, q = d.v.cuda(), d.q.cuda()
+    Ls = [w.L - 3, w.L - 2, w.L - 1, w.L]
+    ws = torch.empty(jl.jetlong_decode_workspace_size(w.B, w.Hq, w.Hkv, w.L, w.D),
+                     dtype=torch.uint8, device="cuda")
+    outs = [torch.empty((w.B, w.Hq, w.D), dtype=torch.float32, device="cuda") for _ in Ls]
+    lses = [torch.empty((w.B, w.Hq), dtype=torch.float32, device="cuda") for _ in Ls]
+
+    def loop(stream=None):
+        for L, o, l in zip(Ls, outs, lses):
+            jl.jetlong_decode(q, cache, v, L, w.w_pretrained, w.w0, w.theta, out=o, lse=l,
+                              workspace=ws, stream=stream)
+
+    loop()
+    eager = [(o.clone(), l.clone()) for o, l in zip(outs, lses)]
+    for o, l in zip(outs, lses):
+        o.fill_(float("nan"))
+        l.fill_(float("nan"))
+    cap = torch.cuda.Stream()
+    cap.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=cap):
+        loop(cap)
+    g.replay()
+    torch.cuda.synchronize()
+    assert jl.jetlong_device_status() == jl.JL_OK
+    for (eo, el), o, l in zip(eager, outs, lses):
+        assert torch.equal(eo, o) and torch.equal(el, l)

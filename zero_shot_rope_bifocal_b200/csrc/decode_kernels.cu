@@ -186,14 +186,12 @@ template <int D, bool REMOTE>
 __device__ __forceinline__ void qk_block(float (&sc)[4], const uint32_t (&q)[D / 16][2],
                                          uint32_t krow_addr, const uint8_t *cs_row, int tq,
                                          int mat) {
-  // Two independent accumulator chains (k-block pairs alternate), summed at
-  // the end, so consecutive MMAs do not wait on each other.
-  float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+  // one accumulator chain: the warp's other work (the other lanes' rotation
+  // math, the other warps) covers the MMA latency, and two chains measured
+  // slower (more registers live)
 #pragma unroll
   for (int kb0 = 0; kb0 < D / 32; kb0 += 2)
-    qk_pair<D, REMOTE>(acc[(kb0 >> 1) & 1], q, krow_addr, cs_row, kb0, tq, mat);
-#pragma unroll
-  for (int e = 0; e < 4; ++e) sc[e] += acc[0][e] + acc[1][e];
+    qk_pair<D, REMOTE>(sc, q, krow_addr, cs_row, kb0, tq, mat);
 }
 
 // Rows of the correction table of one stage: cos and sin of Delta j * theta_i
