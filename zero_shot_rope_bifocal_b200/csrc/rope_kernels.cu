@@ -20,8 +20,9 @@
 //
 // Cache writer (§3.2): k_cache[b, pos0 + t] = RoPE(k[b, t], pos0 + t).
 //
-// Each CTA evaluates cos/sin once per (position, frequency) into shared
-// memory and applies it to every head of that position; channel pairs are
+// Each CTA forms the frequencies once, evaluates cos/sin once per (position,
+// frequency) into shared memory and applies it to every head of that
+// position; channel pairs are
 // (i, i + D/2), processed two pairs per thread with BF16x2 loads and stores.
 #include "jl_common.cuh"
 
@@ -29,7 +30,7 @@ namespace jl {
 namespace {
 
 constexpr int kRopeThreads = 256;
-constexpr int kPosPerCta = 4;
+constexpr int kPosPerCta = 8;
 
 // Rotated pairs (a[i], a[i+D/2]) and (a[i+1], a[i+1+D/2]) of one BF16 head row,
 // in fp32: returns (r0, r1) for channels i, i+1 and (s0, s1) for i+D/2, i+1+D/2.
@@ -65,7 +66,7 @@ __device__ __forceinline__ bool store_f16(__half *dst, int i, int half, const Ro
 
 __global__ void __launch_bounds__(kRopeThreads)
 rope_qk_kernel(PrefillArgs a) {
-  extern __shared__ float2 cs_smem[];  // [2][kPosPerCta][D/2] (cos, sin)
+  extern __shared__ float2 cs_smem[];  // [2][kPosPerCta][D/2] (cos, sin), then [D/2] freq
   const int half = a.D / 2;
   const int b = blockIdx.y;
   const int p_begin = blockIdx.x * kPosPerCta;
@@ -74,7 +75,10 @@ rope_qk_kernel(PrefillArgs a) {
   float2 *cs_true = cs_smem;
   float2 *cs_remote = cs_smem + kPosPerCta * half;
 
+  double *freq = reinterpret_cast<double *>(cs_smem + 2 * kPosPerCta * half);
   const double theta = static_cast<double>(a.theta);
+  for (int i = threadIdx.x; i < half; i += blockDim.x) freq[i] = rope_freq(i, a.D, theta);
+  __syncthreads();
   for (int idx = threadIdx.x; idx < npos * half * (two ? 2 : 1); idx += blockDim.x) {
     const int var = idx / (npos * half);
     const int rem = idx - var * npos * half;
@@ -82,7 +86,7 @@ rope_qk_kernel(PrefillArgs a) {
     const int pos = p_begin + t;
     const long long ppos = var == 0 ? pos : remap(pos, a.G);
     float c, s;
-    rope_cos_sin(ppos, rope_freq(i, a.D, theta), c, s);
+    rope_cos_sin(ppos, freq[i], c, s);
     (var == 0 ? cs_true : cs_remote)[t * half + i] = make_float2(c, s);
   }
   __syncthreads();
@@ -134,16 +138,19 @@ rope_qk_kernel(PrefillArgs a) {
 __global__ void __launch_bounds__(kRopeThreads)
 rope_cache_kernel(const __nv_bfloat16 *__restrict__ k, __nv_bfloat16 *__restrict__ k_cache, int n,
                   int Hkv, int D, int pos0, int Lcap, float theta_f) {
-  extern __shared__ float2 cs_smem[];  // [kPosPerCta][D/2]
+  extern __shared__ float2 cs_smem[];  // [kPosPerCta][D/2], then [D/2] freq
   const int half = D / 2;
   const int b = blockIdx.y;
   const int t_begin = blockIdx.x * kPosPerCta;
   const int npos = min(kPosPerCta, n - t_begin);
+  double *freq = reinterpret_cast<double *>(cs_smem + kPosPerCta * half);
   const double theta = static_cast<double>(theta_f);
+  for (int i = threadIdx.x; i < half; i += blockDim.x) freq[i] = rope_freq(i, D, theta);
+  __syncthreads();
   for (int idx = threadIdx.x; idx < npos * half; idx += blockDim.x) {
     const int t = idx / half, i = idx - t * half;
     float c, s;
-    rope_cos_sin(static_cast<long long>(pos0) + t_begin + t, rope_freq(i, D, theta), c, s);
+    rope_cos_sin(static_cast<long long>(pos0) + t_begin + t, freq[i], c, s);
     cs_smem[t * half + i] = make_float2(c, s);
   }
   __syncthreads();
@@ -164,7 +171,7 @@ rope_cache_kernel(const __nv_bfloat16 *__restrict__ k, __nv_bfloat16 *__restrict
 
 cudaError_t launch_rope_qk(const PrefillArgs &a, cudaStream_t stream) {
   const dim3 grid((a.L + kPosPerCta - 1) / kPosPerCta, a.B);
-  const size_t smem = 2 * kPosPerCta * (a.D / 2) * sizeof(float2);
+  const size_t smem = 2 * kPosPerCta * (a.D / 2) * sizeof(float2) + (a.D / 2) * sizeof(double);
   rope_qk_kernel<<<grid, kRopeThreads, smem, stream>>>(a);
   return cudaGetLastError();
 }
@@ -173,7 +180,7 @@ cudaError_t launch_rope_cache(const __nv_bfloat16 *k, __nv_bfloat16 *k_cache, in
                               int Hkv, int D, int pos0, int Lcap, float theta,
                               cudaStream_t stream) {
   const dim3 grid((n + kPosPerCta - 1) / kPosPerCta, B);
-  const size_t smem = kPosPerCta * (D / 2) * sizeof(float2);
+  const size_t smem = kPosPerCta * (D / 2) * sizeof(float2) + (D / 2) * sizeof(double);
   rope_cache_kernel<<<grid, kRopeThreads, smem, stream>>>(k, k_cache, n, Hkv, D, pos0, Lcap, theta);
   return cudaGetLastError();
 }
