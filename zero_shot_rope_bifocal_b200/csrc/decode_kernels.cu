@@ -11,27 +11,30 @@
 // Split-KV: CTA (s, c, b) streams key chunk s of KV heads [8c, 8c + 8) of
 // batch b (two CTAs per SM).  Warp 0 fills a three-stage shared-memory ring
 // with bulk async copies (cp.async.bulk, one per token and tensor, into rows
-// padded by 16 bytes; completion on the stage's "full" mbarrier).  For each stage the
-// CTA also builds a table of cos/sin(Delta j * theta_i) for its tokens, shared
-// by all heads; every warp writes some of its rows once it is two stages
-// behind.  The phase Delta j * theta_i / (2 pi) is formed exactly modulo one
-// turn in 64-bit fixed point (theta_i / (2 pi) held as a 64-bit binary
-// fraction), so the hardware sine/cosine only ever sees [-pi, pi).
+// padded by 16 bytes; completion on the stage's "full" mbarrier).  For each
+// stage with remote tokens the CTA also builds a table of
+// cos/sin(Delta j * theta_i) for its tokens, shared by all heads; every warp
+// writes some of its rows once it is two stages behind.  The phase
+// Delta j * theta_i / (2 pi) is formed exactly modulo one turn in 64-bit
+// fixed point (theta_i / (2 pi) held as a 64-bit binary fraction), so the
+// hardware sine/cosine only ever sees [-pi, pi).
 // Eight warps, one per KV head, run each stage on the tensor cores
 // (mma.sync m16n8k16):
 //   * S = Q K^T: the A operand holds the group's query heads (rows), FP16,
 //     pre-scaled by log2(e)/sqrt(D); K arrives through ldmatrix as B
-//     fragments, turned (remote tokens) and converted to FP16 in registers;
+//     fragments, turned (remote tokens, packed FP32x2 arithmetic) and
+//     converted to FP16 in registers;
 //   * an online softmax per head over the stage's tokens (fp32 statistics,
 //     lazy rescaling);
 //   * O^T += V^T P^T: V through ldmatrix.trans, P taken straight from the S
-//     accumulator fragment (BF16), O^T accumulated in fp32 registers;
-// each warp then releases the stage on its "empty" mbarrier, and warp 0
+//     accumulator fragment (BF16), O^T accumulated in fp32 registers.
+// Each warp then releases the stage on its "empty" mbarrier, and warp 0
 // refills the slot once all have; no CTA-wide barrier runs in the loop, so
 // warps may drift a stage apart.  Each CTA writes its unnormalised partial
-// output with its
-// running max and sum; a second kernel (launched as a programmatic dependent
-// of the first) merges the partials by log-sum-exp, one CTA per head.
+// output with its running max and sum; a second kernel (launched as a
+// programmatic dependent of the first) merges the partials by log-sum-exp,
+// one CTA per head.  With G = 1 every key is local and a separate
+// instantiation without the remote path runs.
 //
 // The same kernels run a prefill chunk (§3.1, §3.2): n queries at positions
 // P0 .. P0+n-1 are n problems over one cache (grid z = batch x query), each
@@ -186,9 +189,8 @@ template <int D, bool REMOTE>
 __device__ __forceinline__ void qk_block(float (&sc)[4], const uint32_t (&q)[D / 16][2],
                                          uint32_t krow_addr, const uint8_t *cs_row, int tq,
                                          int mat) {
-  // one accumulator chain: the warp's other work (the other lanes' rotation
-  // math, the other warps) covers the MMA latency, and two chains measured
-  // slower (more registers live)
+  // one accumulator chain: the other warps' work covers the MMA latency, and
+  // two interleaved chains (more registers live) measured slower
 #pragma unroll
   for (int kb0 = 0; kb0 < D / 32; kb0 += 2)
     qk_pair<D, REMOTE>(sc, q, krow_addr, cs_row, kb0, tq, mat);
