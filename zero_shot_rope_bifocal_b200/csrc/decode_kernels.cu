@@ -33,7 +33,7 @@
 // warps may drift a stage apart.  Each CTA writes its unnormalised partial
 // output with its running max and sum; a second kernel (launched as a
 // programmatic dependent of the first) merges the partials by log-sum-exp,
-// one CTA per head.  With G = 1 every key is local and a separate
+// one CTA per (head, 32-channel slice).  With G = 1 every key is local and a separate
 // instantiation without the remote path runs.
 //
 // The same kernels run a prefill chunk (§3.1, §3.2): n queries at positions
@@ -526,45 +526,61 @@ decode_split_kernel(DecodeArgs a) {
   }
 }
 
-// Merge the split partials of one (b, head), one CTA of 8 warps per head:
-// block-wide max of the split maxima, the weights 2^(m_s - M) kept in shared
-// memory, then each warp accumulates every 8th split (lanes over channel
-// pairs) and the 8 warp sums are added.  Launched as a programmatic dependent
-// of the split kernel: the wait below returns once that grid has finished and
-// its partials are visible.
+// Merge the split partials of one (b, head) for one 32-channel slice, one
+// CTA of 8 warps: the block-wide max of the split maxima and the weights
+// 2^(m_s - M) (one round of loads), then warp w sums splits w, w + 8, ... for
+// channel `lane` of the slice with every load issued up front (the loop is
+// unrolled to the largest split count), and the 8 warp sums are added.
+// Launched as a programmatic dependent of the split kernel: the wait below
+// returns once that grid has finished and its partials are visible.
 constexpr int kCombineThreads = 256;
+constexpr int kCombineWarps = kCombineThreads / 32;
 constexpr int kMaxSplit = kCtasPerSm * 148;  // decode_plan never exceeds this
+constexpr int kSplitsPerWarp = (kMaxSplit + kCombineWarps - 1) / kCombineWarps;
+static_assert(kMaxSplit <= 2 * kCombineThreads, "two splits per thread in the max pass");
 
 template <int D>
 __global__ void __launch_bounds__(kCombineThreads)
 decode_combine_kernel(DecodeArgs a) {
   asm volatile("griddepcontrol.wait;" ::: "memory");
-  constexpr int NW = kCombineThreads / 32;
-  constexpr int PAIRS = D / 64;  // float2 channel pairs per lane
   __shared__ float wsh[kMaxSplit];
-  __shared__ float red[NW][D];
-  __shared__ float part[NW];
-  const int bh = blockIdx.x;
+  __shared__ float red[kCombineWarps][32];
+  __shared__ float part[kCombineWarps];
+  const int bh = blockIdx.x;     // (b * nq + query) * Hq + head
+  const int c = blockIdx.y * 32 + (threadIdx.x & 31);  // channel of this lane
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int ns = a.n_split;
   const float *rec = a.partial + static_cast<size_t>(bh) * ns * (D + 2);
 
-  float m = -INFINITY;
-  for (int s = tid; s < ns; s += kCombineThreads) m = fmaxf(m, rec[s * (D + 2) + D]);
+  // the split maxima and sums, two splits per thread at most
+  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+  if (tid < ns) {
+    m0 = rec[tid * (D + 2) + D];
+    l0 = rec[tid * (D + 2) + D + 1];
+  }
+  if (tid + kCombineThreads < ns) {
+    m1 = rec[(tid + kCombineThreads) * (D + 2) + D];
+    l1 = rec[(tid + kCombineThreads) * (D + 2) + D + 1];
+  }
+  float m = fmaxf(m0, m1);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
   if (lane == 0) part[warp] = m;
   __syncthreads();
   float M = part[0];
 #pragma unroll
-  for (int w = 1; w < NW; ++w) M = fmaxf(M, part[w]);
+  for (int w = 1; w < kCombineWarps; ++w) M = fmaxf(M, part[w]);
   __syncthreads();  // part[] is reused below
-
   float l = 0.f;
-  for (int s = tid; s < ns; s += kCombineThreads) {
-    const float w = exp2f(rec[s * (D + 2) + D] - M);
-    wsh[s] = w;
-    l = fmaf(rec[s * (D + 2) + D + 1], w, l);
+  if (tid < ns) {
+    const float w = exp2f(m0 - M);
+    wsh[tid] = w;
+    l = l0 * w;
+  }
+  if (tid + kCombineThreads < ns) {
+    const float w = exp2f(m1 - M);
+    wsh[tid + kCombineThreads] = w;
+    l = fmaf(l1, w, l);
   }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) l += __shfl_xor_sync(0xffffffffu, l, o);
@@ -572,42 +588,34 @@ decode_combine_kernel(DecodeArgs a) {
   __syncthreads();
   float lsum = 0.f;
 #pragma unroll
-  for (int w = 0; w < NW; ++w) lsum += part[w];
+  for (int w = 0; w < kCombineWarps; ++w) lsum += part[w];
 
-  float2 acc[PAIRS];
+  float v[kSplitsPerWarp];
 #pragma unroll
-  for (int e = 0; e < PAIRS; ++e) acc[e] = make_float2(0.f, 0.f);
-  if (lane < D / 2) {  // D = 64: lanes 0..31 hold one pair each
-#pragma unroll 4
-    for (int s = warp; s < ns; s += NW) {
-      const float w = wsh[s];
-      const float2 *r2 = reinterpret_cast<const float2 *>(rec + static_cast<size_t>(s) * (D + 2));
-#pragma unroll
-      for (int e = 0; e < PAIRS; ++e) {
-        const float2 v = r2[lane + 32 * e];
-        acc[e].x = fmaf(w, v.x, acc[e].x);
-        acc[e].y = fmaf(w, v.y, acc[e].y);
-      }
-    }
-#pragma unroll
-    for (int e = 0; e < PAIRS; ++e) {
-      red[warp][2 * (lane + 32 * e)] = acc[e].x;
-      red[warp][2 * (lane + 32 * e) + 1] = acc[e].y;
-    }
+  for (int k = 0; k < kSplitsPerWarp; ++k) {
+    const int sp = warp + kCombineWarps * k;
+    v[k] = (sp < ns && c < D) ? rec[static_cast<size_t>(sp) * (D + 2) + c] : 0.f;
   }
+  float acc = 0.f;
+#pragma unroll
+  for (int k = 0; k < kSplitsPerWarp; ++k) {
+    const int sp = warp + kCombineWarps * k;
+    if (sp < ns) acc = fmaf(wsh[sp], v[k], acc);
+  }
+  red[warp][lane] = acc;
   __syncthreads();
-  const float inv = 1.f / lsum;
-  for (int c = tid; c < D; c += kCombineThreads) {
+  if (tid < 32 && c < D) {
     float o = 0.f;
 #pragma unroll
-    for (int w = 0; w < NW; ++w) o += red[w][c];
+    for (int w = 0; w < kCombineWarps; ++w) o += red[w][tid];
+    o /= lsum;
     const size_t idx = static_cast<size_t>(bh) * D + c;
     if (a.out_f32)
-      reinterpret_cast<float *>(a.out)[idx] = o * inv;
+      reinterpret_cast<float *>(a.out)[idx] = o;
     else
-      reinterpret_cast<__nv_bfloat16 *>(a.out)[idx] = __float2bfloat16_rn(o * inv);
+      reinterpret_cast<__nv_bfloat16 *>(a.out)[idx] = __float2bfloat16_rn(o);
   }
-  if (tid == 0 && a.lse) {  // lse is [B, Hq, nq]
+  if (blockIdx.y == 0 && tid == 0 && a.lse) {  // lse is [B, Hq, nq]
     const int h = bh % a.Hq, bqi = bh / a.Hq;
     const int bb = bqi / a.nq, qi = bqi - bb * a.nq;
     a.lse[(static_cast<size_t>(bb) * a.Hq + h) * a.nq + qi] = (M + log2f(lsum)) * 0.69314718055994531f;
@@ -642,7 +650,7 @@ cudaError_t launch_decode_d(const DecodeArgs &a, cudaStream_t stream) {
   if (e != cudaSuccess) return e;
   if (a.n_split > kMaxSplit) return cudaErrorInvalidValue;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(a.B * a.nq * a.Hq));
+  cfg.gridDim = dim3(static_cast<unsigned>(a.B * a.nq * a.Hq), D / 32);
   cfg.blockDim = dim3(kCombineThreads);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = stream;
