@@ -21,6 +21,9 @@ Long-Context Extension with Dynamic Bifocal RoPE", full text):
   each pair directly).
 * §2.1: RoPE rotates channel pairs at geometrically spaced frequencies, so that
   a dot product depends only on the relative position.
+* §4.7 and Table 6 (ablation of the remote map): frequency interpolation in
+  place of position aliasing, in ``interp_freq`` and the ``*_interp``
+  functions; the readings it needs are stated above ``interp_scale``.
 * Appendix H ("Hardware, precision, and software"): BF16 Q/K/V, FP32 softmax
   and log-sum-exp statistics; the oracle works in float64 on the BF16 values.
 
@@ -54,6 +57,15 @@ __all__ = [
     "decode",
     "prefill_chunk",
     "merge_three_pass",
+    "interp_scale",
+    "interp_freq",
+    "rope_at_freq",
+    "prefill_interp_rows",
+    "prefill_interp",
+    "prefill_interp_literal",
+    "correction_rotate_interp",
+    "prefill_chunk_interp",
+    "decode_interp",
 ]
 
 
@@ -411,3 +423,227 @@ def merge_three_pass(q, k, v, w_pretrained: int, w0: int, theta: float):
             o[b, :, h] = (wa[:, None] * oa + wb[:, None] * ob - wc[:, None] * oc) / den[:, None]
             lse[b, h] = M + np.log(den)
     return o, lse
+
+
+# --------------------------------------------------------------------------
+# §4.7 ablation: frequency interpolation instead of position aliasing
+# --------------------------------------------------------------------------
+# Table 6 of the page compares the default remote map (positions aliased to
+# f(x) = floor(x / G)) with "YaRN-style frequency interpolation within the same
+# bifocal construction".  The page gives no formula for that variant; the
+# readings taken here (each also listed in the design notes):
+#
+# * The local band is untouched: pairs with 0 <= i - j <= w0 are scored at true
+#   positions with the pretrained frequencies.  Only the remote map changes.
+# * Remote pairs are scored at their TRUE positions with per-frequency
+#   interpolated frequencies theta'_t (YaRN's "NTK-by-parts" rule):
+#     r_t     = w_pretrained * theta_t / (2 pi)   turns of frequency t within the
+#                                                 pretrained window,
+#     gamma_t = clip((r_t - alpha) / (beta - alpha), 0, 1),
+#     theta'_t = theta_t * ((1 - gamma_t) / s + gamma_t),
+#   so slow frequencies (few turns, r_t < alpha) are divided by s and fast ones
+#   (r_t > beta) are kept.  alpha = 1, beta = 32 are YaRN's published defaults.
+# * s is the dynamic factor the page names for continuous rescaling in §3.1,
+#   s = max(1, L / w_pretrained), recomputed from the current length like G.
+# * No attention temperature: the softmax scale stays 1/sqrt(D) (the ablation
+#   changes the remote-window mapping only).
+# * The cache still holds RoPE(x_k, j) at true positions (§3.2); a cached key
+#   is turned into the remote form by the rotation of angle j (theta'_t - theta_t).
+def interp_scale(L: int, w_pretrained: int) -> float:
+    """Continuous dynamic factor of §3.1: s = max(1, L / w_pretrained)."""
+    L = int(L)
+    w = int(w_pretrained)
+    if L < 1 or w < 1:
+        raise ValueError("L and w_pretrained must be >= 1")
+    return max(1.0, L / w)
+
+
+def interp_freq(D: int, theta: float, L: int, w_pretrained: int, alpha: float = 1.0,
+                beta: float = 32.0) -> np.ndarray:
+    """Interpolated frequencies theta'_t, t < D/2, of the remote branch (float64)."""
+    if not beta > alpha:
+        raise ValueError("beta must exceed alpha")
+    base = inv_freq(D, theta)
+    s = interp_scale(L, w_pretrained)
+    turns = float(w_pretrained) * base / (2.0 * math.pi)
+    gamma = np.clip((turns - alpha) / (beta - alpha), 0.0, 1.0)
+    return base * ((1.0 - gamma) / s + gamma)
+
+
+def rope_at_freq(x, pos, freqs) -> np.ndarray:
+    """Rotate each channel pair (t, t + D/2) of x by angle pos * freqs[t]."""
+    x = np.asarray(x, dtype=np.float64)
+    h = x.shape[-1] // 2
+    ang = np.asarray(pos, dtype=np.float64)[..., None] * np.asarray(freqs, dtype=np.float64)
+    c = np.cos(ang)
+    s = np.sin(ang)
+    a = x[..., :h]
+    b = x[..., h:]
+    return np.concatenate([a * c - b * s, a * s + b * c], axis=-1)
+
+
+def prefill_interp_rows(q, k, v, w_pretrained: int, w0: int, theta: float, rows,
+                        alpha: float = 1.0, beta: float = 32.0):
+    """Frequency-interpolation variant of ``prefill_rows`` for the listed rows.
+
+      s_ij = RoPE(x_q[i], i) . RoPE(x_k[j], j) / sqrt(D)      if i - j <= w0
+      s_ij = RoPE'(x_q[i], i) . RoPE'(x_k[j], j) / sqrt(D)    otherwise
+
+    RoPE' rotates with ``interp_freq`` (one s for the prompt, from L =
+    k.shape[1]).  Returns (o [B, len(rows), Hq, D], lse [B, Hq, len(rows)]).
+    """
+    q = np.asarray(q)
+    k = np.asarray(k)
+    v = np.asarray(v)
+    B, L, Hq, Hkv, D = _check_shapes(q, k, v)
+    rows = np.asarray(rows, dtype=np.int64)
+    if rows.size and (rows.min() < 0 or rows.max() >= L):
+        raise ValueError("row out of range")
+    grp = Hq // Hkv
+    fr = interp_freq(D, theta, L, w_pretrained, alpha, beta)
+    scale = 1.0 / math.sqrt(D)
+    jmax = int(rows.max()) + 1 if rows.size else 0
+    jpos = np.arange(jmax, dtype=np.int64)
+    o = np.zeros((B, rows.size, Hq, D), dtype=np.float64)
+    lse = np.zeros((B, Hq, rows.size), dtype=np.float64)
+    for b in range(B):
+        for g in range(Hkv):
+            xk = k[b, :jmax, g, :].astype(np.float64)
+            vv = v[b, :jmax, g, :].astype(np.float64)
+            k_true = rope(xk, jpos, theta)
+            k_remote = rope_at_freq(xk, jpos, fr)
+            heads = np.arange(g * grp, (g + 1) * grp)
+            for r, i in enumerate(rows):
+                xq = q[b, i, heads, :].astype(np.float64)
+                q_true = rope(xq, np.int64(i), theta)
+                q_remote = rope_at_freq(xq, np.int64(i), fr)
+                n = i + 1
+                dist = (i - jpos[:n])[:, None]
+                s = np.where(dist <= w0, k_true[:n] @ q_true.T, k_remote[:n] @ q_remote.T) * scale
+                m = s.max(axis=0)
+                e = np.exp(s - m)
+                tot = e.sum(axis=0)
+                lse[b, heads, r] = m + np.log(tot)
+                o[b, r, heads, :] = (e / tot).T @ vv[:n]
+    return o, lse
+
+
+def prefill_interp(q, k, v, w_pretrained: int, w0: int, theta: float, alpha: float = 1.0,
+                   beta: float = 32.0):
+    """Frequency-interpolation variant over every query row: (o, lse)."""
+    L = np.asarray(q).shape[1]
+    return prefill_interp_rows(q, k, v, w_pretrained, w0, theta, np.arange(L), alpha, beta)
+
+
+def prefill_interp_literal(q, k, v, w_pretrained: int, w0: int, theta: float,
+                           alpha: float = 1.0, beta: float = 32.0):
+    """Pure-Python per-pair version of ``prefill_interp`` for tiny inputs.
+
+    Forms both frequency sets with scalar ``math`` calls, re-rotates the query
+    and key of every pair by hand, and runs a two-pass softmax; it shares no
+    intermediate with the vectorised version.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    B, L, Hq, Hkv, D = _check_shapes(q, k, v)
+    grp = Hq // Hkv
+    h2 = D // 2
+    s_fac = max(1.0, L / w_pretrained)
+    base, interp = [], []
+    for t in range(h2):
+        f = float(theta) ** (-2.0 * t / D)
+        turns = w_pretrained * f / (2.0 * math.pi)
+        gam = min(1.0, max(0.0, (turns - alpha) / (beta - alpha)))
+        base.append(f)
+        interp.append(f * ((1.0 - gam) / s_fac + gam))
+
+    def rot(x, p, freqs):
+        out = [0.0] * D
+        for t in range(h2):
+            a = p * freqs[t]
+            ca, sa = math.cos(a), math.sin(a)
+            out[t] = x[t] * ca - x[t + h2] * sa
+            out[t + h2] = x[t] * sa + x[t + h2] * ca
+        return out
+
+    o = np.zeros((B, L, Hq, D))
+    lse = np.zeros((B, Hq, L))
+    for b in range(B):
+        for h in range(Hq):
+            g = h // grp
+            for i in range(L):
+                scores = []
+                for j in range(i + 1):
+                    freqs = base if i - j <= w0 else interp
+                    qa = rot(list(q[b, i, h]), i, freqs)
+                    kb = rot(list(k[b, j, g]), j, freqs)
+                    scores.append(sum(x * y for x, y in zip(qa, kb)) / math.sqrt(D))
+                m = max(scores)
+                tot = sum(math.exp(s - m) for s in scores)
+                lse[b, h, i] = m + math.log(tot)
+                for j, s in enumerate(scores):
+                    o[b, i, h] += math.exp(s - m) / tot * v[b, j, g]
+    return o, lse
+
+
+def correction_rotate_interp(c, kpos, freq_interp, theta: float) -> np.ndarray:
+    """Turn a cached key c = RoPE(x, j) into RoPE'(x, j): rotate by angle
+    j * (theta'_t - theta_t) per channel pair (the §3.2 correction for this map)."""
+    D = np.asarray(c).shape[-1]
+    return rope_at_freq(c, kpos, np.asarray(freq_interp) - inv_freq(D, theta))
+
+
+def prefill_chunk_interp(q, k_cache, v_cache, P0: int, w_pretrained: int, w0: int,
+                         theta: float, alpha: float = 1.0, beta: float = 32.0):
+    """Frequency-interpolation variant of ``prefill_chunk``: queries at P0 ..
+    P0+n-1 on the true-position cache, one s from L = P0 + n.
+
+      local  (p - j <= w0): s = RoPE(x_q, p) . k_cache[j]
+      remote (p - j >  w0): s = RoPE'(x_q, p) . R(j (theta' - theta)) k_cache[j]
+
+    Returns (o [B, n, Hq, D], lse [B, Hq, n]) in float64.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    kc = np.asarray(k_cache)
+    vc = np.asarray(v_cache)
+    B, n, Hq, D = q.shape
+    Hkv = kc.shape[2]
+    L = P0 + n
+    if kc.shape[1] < L or vc.shape[:3] != kc.shape[:3]:
+        raise ValueError("cache shorter than P0 + n")
+    grp = Hq // Hkv
+    fr = interp_freq(D, theta, L, w_pretrained, alpha, beta)
+    scale = 1.0 / math.sqrt(D)
+    o = np.zeros((B, n, Hq, D))
+    lse = np.zeros((B, Hq, n))
+    jpos_all = np.arange(L, dtype=np.int64)
+    for b in range(B):
+        for g in range(Hkv):
+            c_all = kc[b, :L, g, :].astype(np.float64)
+            v_all = vc[b, :L, g, :].astype(np.float64)
+            cc_all = correction_rotate_interp(c_all, jpos_all, fr, theta)
+            heads = np.arange(g * grp, (g + 1) * grp)
+            for i in range(n):
+                p = P0 + i
+                local = (p - jpos_all[: p + 1]) <= w0
+                q_true = rope(q[b, i, heads], np.int64(p), theta)
+                q_remote = rope_at_freq(q[b, i, heads], np.int64(p), fr)
+                s = np.where(local[:, None], c_all[: p + 1] @ q_true.T,
+                             cc_all[: p + 1] @ q_remote.T) * scale
+                m = s.max(axis=0)
+                e = np.exp(s - m)
+                tot = e.sum(axis=0)
+                lse[b, heads, i] = m + np.log(tot)
+                o[b, i, heads, :] = (e / tot).T @ v_all[: p + 1]
+    return o, lse
+
+
+def decode_interp(q, k_cache, v_cache, L: int, w_pretrained: int, w0: int, theta: float,
+                  alpha: float = 1.0, beta: float = 32.0):
+    """One generation step of the frequency-interpolation variant at p = L - 1:
+    the one-token chunk.  Returns (o [B, Hq, D], lse [B, Hq])."""
+    q = np.asarray(q, dtype=np.float64)
+    o, lse = prefill_chunk_interp(q[:, None], k_cache, v_cache, L - 1, w_pretrained, w0, theta,
+                                  alpha, beta)
+    return o[:, 0], lse[:, :, 0]

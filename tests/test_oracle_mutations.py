@@ -12,6 +12,7 @@ import pytest
 
 import oracle
 import oracle.bifocal_ref as ref
+import test_oracle_interp as ipins
 import test_oracle_pins as pins
 
 
@@ -65,6 +66,28 @@ def chunk_pins():
             pins.test_one_token_chunk_is_a_decode_step]
 
 
+RAMP_PINS = [ipins.test_scale_is_the_continuous_dynamic_factor,
+             ipins.test_native_length_keeps_every_frequency,
+             ipins.test_slow_frequencies_are_divided_by_s,
+             ipins.test_fast_frequencies_are_kept,
+             ipins.test_ramp_is_linear_in_turns_within_the_pretrained_window,
+             ipins.test_default_ramp_on_the_tiny_workload]
+
+
+def interp_pins():
+    return [ipins.test_native_length_is_plain_rope_attention,
+            ipins.test_kept_frequencies_give_plain_rope_attention_at_any_length,
+            lambda: ipins.test_band_and_remote_parts_via_masked_library_attention(1.0, 32.0),
+            ipins.test_literal_per_pair_brute_force]
+
+
+def interp_cache_pins():
+    return [ipins.test_correction_rotation_turns_the_cache_into_the_interpolated_key,
+            ipins.test_chunk_of_the_whole_prompt_is_the_prefill,
+            lambda: ipins.test_chunk_tail_rows_are_the_prefill_rows(300),
+            lambda: ipins.test_decode_equals_last_prefill_row(300)]
+
+
 MUTANTS = [
     # schedule
     ("group_size", "max(1, -((-L) // w))", "max(1, L // w)",
@@ -109,6 +132,29 @@ MUTANTS = [
     ("prefill_chunk", "                p = P0 + i\n", "                p = P0 + i + 1\n", chunk_pins()),
     ("prefill_chunk", "c, cc, vv = c_all[: p + 1], c_corr_all[: p + 1], v_all[: p + 1]",
      "c, cc, vv = c_all[:p], c_corr_all[:p], v_all[:p]", chunk_pins()),
+    # frequency-interpolation remote map (§4.7)
+    ("interp_scale", "max(1.0, L / w)", "max(1.0, L // w)", RAMP_PINS),
+    ("interp_freq", "(1.0 - gamma) / s + gamma", "gamma / s + (1.0 - gamma)", RAMP_PINS),
+    ("interp_freq", "s = interp_scale(L, w_pretrained)", "s = group_size(L, w_pretrained)",
+     RAMP_PINS),
+    ("interp_freq", "turns = float(w_pretrained) * base", "turns = float(L) * base", RAMP_PINS),
+    ("interp_freq", "turns = float(w_pretrained) * base / (2.0 * math.pi)",
+     "turns = float(w_pretrained) / base / (2.0 * math.pi)", RAMP_PINS),
+    ("interp_freq", "(turns - alpha) / (beta - alpha)", "(turns - alpha) / beta", RAMP_PINS),
+    ("rope_at_freq", "a * c - b * s, a * s + b * c", "a * c + b * s, -a * s + b * c",
+     interp_pins()),
+    ("prefill_interp_rows", "dist <= w0", "dist < w0", interp_pins()),
+    ("prefill_interp_rows", "q_remote = rope_at_freq(xq, np.int64(i), fr)",
+     "q_remote = rope_at_freq(xq, remap(np.int64(i), group_size(L, w_pretrained)), fr)",
+     interp_pins()),
+    ("prefill_interp_rows", "k_true = rope(xk, jpos, theta)", "k_true = rope_at_freq(xk, jpos, fr)",
+     interp_pins()),
+    ("correction_rotate_interp", "np.asarray(freq_interp) - inv_freq(D, theta)",
+     "inv_freq(D, theta) - np.asarray(freq_interp)", interp_cache_pins()),
+    ("prefill_chunk_interp", "fr = interp_freq(D, theta, L, w_pretrained, alpha, beta)",
+     "fr = interp_freq(D, theta, P0 + 1, w_pretrained, alpha, beta)", interp_cache_pins()),
+    ("prefill_chunk_interp", "local = (p - jpos_all[: p + 1]) <= w0",
+     "local = (p - jpos_all[: p + 1]) < w0", interp_cache_pins()),
 ]
 
 
