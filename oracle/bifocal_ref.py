@@ -483,20 +483,27 @@ def rope_at_freq(x, pos, freqs) -> np.ndarray:
 
 
 def prefill_interp_rows(q, k, v, w_pretrained: int, w0: int, theta: float, rows,
-                        alpha: float = 1.0, beta: float = 32.0):
+                        alpha: float = 1.0, beta: float = 32.0, q_holds_rows: bool = False):
     """Frequency-interpolation variant of ``prefill_rows`` for the listed rows.
 
       s_ij = RoPE(x_q[i], i) . RoPE(x_k[j], j) / sqrt(D)      if i - j <= w0
       s_ij = RoPE'(x_q[i], i) . RoPE'(x_k[j], j) / sqrt(D)    otherwise
 
     RoPE' rotates with ``interp_freq`` (one s for the prompt, from L =
-    k.shape[1]).  Returns (o [B, len(rows), Hq, D], lse [B, Hq, len(rows)]).
+    k.shape[1]).  With ``q_holds_rows`` q is [B, len(rows), Hq, D] and holds
+    only the listed rows' queries.  Returns (o [B, len(rows), Hq, D],
+    lse [B, Hq, len(rows)]).
     """
     q = np.asarray(q)
     k = np.asarray(k)
     v = np.asarray(v)
-    B, L, Hq, Hkv, D = _check_shapes(q, k, v)
     rows = np.asarray(rows, dtype=np.int64)
+    if q_holds_rows:
+        if q.ndim != 4 or q.shape[1] != rows.size:
+            raise ValueError("q must be [B, len(rows), Hq, D]")
+        B, L, Hq, Hkv, D = _check_shapes(np.broadcast_to(q[:, :1], (q.shape[0], k.shape[1]) + q.shape[2:]), k, v)
+    else:
+        B, L, Hq, Hkv, D = _check_shapes(q, k, v)
     if rows.size and (rows.min() < 0 or rows.max() >= L):
         raise ValueError("row out of range")
     grp = Hq // Hkv
@@ -514,7 +521,7 @@ def prefill_interp_rows(q, k, v, w_pretrained: int, w0: int, theta: float, rows,
             k_remote = rope_at_freq(xk, jpos, fr)
             heads = np.arange(g * grp, (g + 1) * grp)
             for r, i in enumerate(rows):
-                xq = q[b, i, heads, :].astype(np.float64)
+                xq = q[b, r if q_holds_rows else i, heads, :].astype(np.float64)
                 q_true = rope(xq, np.int64(i), theta)
                 q_remote = rope_at_freq(xq, np.int64(i), fr)
                 n = i + 1

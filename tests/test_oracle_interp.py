@@ -203,3 +203,13 @@ def test_decode_equals_last_prefill_row(L):
     od, ld = oracle.decode_interp(q[:, L - 1], cache, v, L, w.w_pretrained, w.w0, w.theta)
     np.testing.assert_allclose(od, o[:, 0], atol=1e-10)
     np.testing.assert_allclose(ld, lse[:, :, 0], atol=1e-10)
+
+
+def test_rows_subset_matches_full():
+    w, q, k, v = tiny_inputs("tiny")
+    o, lse = oracle.prefill_interp(q, k, v, w.w_pretrained, w.w0, w.theta)
+    rows = [0, 32, 33, 128, 300, 511]
+    o2, l2 = oracle.prefill_interp_rows(q[:, rows], k, v, w.w_pretrained, w.w0, w.theta, rows,
+                                        q_holds_rows=True)
+    np.testing.assert_array_equal(o2, o[:, rows])
+    np.testing.assert_array_equal(l2, lse[:, :, rows])
