@@ -15,7 +15,9 @@ Both are also timed as a matched control -- the same kernels with the
 bifocal rule off (w_pretrained = L, so G = 1: plain causal RoPE attention at
 true positions) -- and the ratio is reported as the routing cost.  The
 prefill is also timed in its unfused three-pass form (jetlong_prefill_three_pass)
-to report what fusion saves.
+to report what fusion saves, and prefill and decode are timed once more with
+the frequency-interpolation remote map of the paper's remote-map ablation
+(jetlong_prefill_interp, jetlong_decode_interp).
 
 Every input is synthetic and seeded (zero_shot_rope_bifocal_b200.synth);
 each is larger than the 126 MB L2 (q alone is 1 GiB), so no flush is needed
@@ -385,6 +387,25 @@ def run_native(args):
     del ws3
     if jl.jetlong_device_status() != jl.JL_OK:
         raise RuntimeError("device status not OK after the three-pass prefill")
+    # ---- the frequency-interpolation remote map (the remote-map ablation):
+    # the same attention kernel on operands rotated with interpolated
+    # frequencies at true positions
+    def interp_step():
+        jl.jetlong_prefill_interp(x.q, x.k, x.v, w.w_pretrained, w.w0, w.theta, out=out, lse=lse,
+                                  workspace=ws, stream=stream)
+
+    interp_step()
+    barrier()
+    torch.cuda.synchronize(dev)
+    ev0.record(stream)
+    for _ in range(n_ctl):
+        interp_step()
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    interp_ms = reduce_max(ev0.elapsed_time(ev1), world, dev) / n_ctl
+    if jl.jetlong_device_status() != jl.JL_OK:
+        raise RuntimeError("device status not OK after the interpolation prefill")
     flops_rank = prefill_flops(B, Hq, L, D) * args.steps
     flops_all = reduce_sum(flops_rank, world, dev)
     value = flops_all / (t_max * 1e-3) / 1e12
@@ -481,6 +502,25 @@ def run_native(args):
     ctl_us_tok = 1e3 * reduce_max(ev0.elapsed_time(ev1), world, dev) / n_loop
     if jl.jetlong_device_status() != jl.JL_OK:
         raise RuntimeError("device status not OK after the control decode")
+
+    # the frequency-interpolation decode, host launches like host_loop_us
+    def dstep_interp():
+        jl.jetlong_decode_interp(dq, kc, d.v, wd.L, wd.w_pretrained, wd.w0, wd.theta, out=dout,
+                                 lse=dlse, workspace=dws, stream=stream)
+
+    for _ in range(3):
+        dstep_interp()
+    barrier()
+    torch.cuda.synchronize(dev)
+    ev0.record(stream)
+    for _ in range(n_loop):
+        dstep_interp()
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    interp_us_tok = 1e3 * reduce_max(ev0.elapsed_time(ev1), world, dev) / n_loop
+    if jl.jetlong_device_status() != jl.JL_OK:
+        raise RuntimeError("device status not OK after the interpolation decode")
 
     # a 64-token prefill chunk appended at the end of the same 128K cache
     n_chunk = 64
@@ -629,6 +669,15 @@ def run_native(args):
                 "ms_per_step": three_ms,
                 "tflops": prefill_flops(B, Hq, L, D) / (three_ms * 1e-3) / 1e12,
                 "fused_speedup": three_ms / (t_max / args.steps)},
+            "freq_interp": {
+                "what": "remote-map ablation: remote pairs at true positions with YaRN-style "
+                        "interpolated frequencies (ramp 1..32 turns, s = L / w_pretrained), "
+                        "same inputs; prefill = rotate + attend, decode host-launched",
+                "prefill_step_ms": interp_ms,
+                "prefill_tflops": prefill_flops(B, Hq, L, D) / (interp_ms * 1e-3) / 1e12,
+                "decode_us_per_token": interp_us_tok,
+                "vs_alias_prefill_step": interp_ms / (t_max / args.steps),
+                "vs_alias_decode_host_launched": interp_us_tok / host_loop_us},
             "e2e": {"value": e2e_val, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "steps": n_e2e,
                     "pipelined": "step i's H2D and step i-1's D2H overlap compute on two copy "

@@ -272,6 +272,48 @@ JL_API int jetlong_decode_noalloc(const void *q, const void *k_cache, const void
                                   jl_stream_t stream);
 
 /*
+ * Frequency-interpolation remote map: the ablation of §4.7 ("interpolate
+ * frequency or alias position", Table 6) of the Jet-Long paper.  The page
+ * gives no formula for it; these calls take the following reading.  The local
+ * band (i - j <= w0) is unchanged.  A remote pair is scored at TRUE positions
+ * with per-frequency interpolated frequencies (YaRN's per-frequency ramp):
+ *   r_t      = w_pretrained * theta_t / (2 pi)   (turns within the pretrained window)
+ *   gamma_t  = clamp((r_t - ramp_alpha) / (ramp_beta - ramp_alpha), 0, 1)
+ *   theta'_t = theta_t * ((1 - gamma_t) / s + gamma_t),  s = max(1, L / w_pretrained)
+ * where theta_t = rope_theta^(-2t/D) and s is §3.1's continuous dynamic
+ * factor, recomputed from L like G.  There is no attention temperature.
+ * YaRN's published bounds are ramp_alpha = 1, ramp_beta = 32.  The cache
+ * stays at true positions.  A remote cached key is turned by the angle
+ * j (theta'_t - theta_t), and the query is rotated by p theta'_t.  With
+ * L <= w_pretrained, s = 1 and the result is plain causal RoPE attention,
+ * as in the aliasing calls.
+ *
+ * Each call takes the arguments, layouts, workspace (the same
+ * *_workspace_size function) and error codes of its aliasing counterpart,
+ * plus ramp_alpha < ramp_beta, both finite (else JL_ERR_SHAPE, nothing
+ * launched).
+ */
+JL_API int jetlong_prefill_interp(const void *q, const void *k, const void *v, void *out,
+                                  float *lse, int B, int Hq, int Hkv, int L, int D,
+                                  int w_pretrained, int w0, float rope_theta, float ramp_alpha,
+                                  float ramp_beta, int out_dtype, void *k_cache_out,
+                                  int k_cache_capacity, void *workspace, size_t workspace_bytes,
+                                  jl_stream_t stream);
+
+JL_API int jetlong_decode_interp(const void *q, const void *k_cache, const void *v_cache,
+                                 void *out, float *lse, int B, int Hq, int Hkv, int L, int Lcap,
+                                 int D, int w_pretrained, int w0, float rope_theta,
+                                 float ramp_alpha, float ramp_beta, int out_dtype,
+                                 void *workspace, size_t workspace_bytes, jl_stream_t stream);
+
+JL_API int jetlong_prefill_chunk_interp(const void *q, const void *k_cache, const void *v_cache,
+                                        void *out, float *lse, int B, int Hq, int Hkv, int P0,
+                                        int n, int Lcap, int D, int w_pretrained, int w0,
+                                        float rope_theta, float ramp_alpha, float ramp_beta,
+                                        int out_dtype, void *workspace, size_t workspace_bytes,
+                                        jl_stream_t stream);
+
+/*
  * Write keys into the true-position cache (§3.2): for t < n,
  *   k_cache[b, pos0 + t, h, :] = RoPE(k[b, t, h, :], pos0 + t).
  *

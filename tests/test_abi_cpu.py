@@ -233,3 +233,35 @@ def test_stage_entry_points_check_their_own_buffers(lib):
     assert att(out=None) == jl.JL_ERR_NULL
     assert att(lse=ctypes.c_void_p(260)) == jl.JL_ERR_ALIGN
     assert att(ws=None) == jl.JL_ERR_WORKSPACE
+
+
+# ---------------------------------------------------------------- frequency-interpolation map
+def interp_calls(lib, alpha, beta, **kw):
+    """The three interpolation entry points with otherwise valid arguments."""
+    p = dict(q=P, k=P, v=P, out=P, lse=None, B=1, Hq=2, Hkv=1, L=512, D=64, wp=128, w0=32,
+             theta=1e4, od=0, kc=None, cap=0, ws=P, wsb=1 << 40, stream=None)
+    p.update(kw)
+    pre = lib.jetlong_prefill_interp(p["q"], p["k"], p["v"], p["out"], p["lse"], p["B"], p["Hq"],
+                                     p["Hkv"], p["L"], p["D"], p["wp"], p["w0"], p["theta"], alpha,
+                                     beta, p["od"], p["kc"], p["cap"], p["ws"], p["wsb"],
+                                     p["stream"])
+    dec = lib.jetlong_decode_interp(p["q"], P, P, p["out"], p["lse"], p["B"], p["Hq"], p["Hkv"],
+                                    p["L"], p["L"], p["D"], p["wp"], p["w0"], p["theta"], alpha,
+                                    beta, p["od"], p["ws"], p["wsb"], p["stream"])
+    chk = lib.jetlong_prefill_chunk_interp(p["q"], P, P, p["out"], p["lse"], p["B"], p["Hq"],
+                                           p["Hkv"], p["L"] - 8, 8, p["L"], p["D"], p["wp"],
+                                           p["w0"], p["theta"], alpha, beta, p["od"], p["ws"],
+                                           p["wsb"], p["stream"])
+    return pre, dec, chk
+
+
+@pytest.mark.parametrize("alpha,beta", [(32.0, 1.0), (4.0, 4.0), (float("nan"), 32.0),
+                                        (1.0, float("inf"))])
+def test_interp_rejects_bad_ramp_bounds(lib, alpha, beta):
+    assert interp_calls(lib, alpha, beta) == (jl.JL_ERR_SHAPE,) * 3
+
+
+def test_interp_checks_the_same_arguments_as_the_aliasing_calls(lib):
+    assert interp_calls(lib, 1.0, 32.0, q=None) == (jl.JL_ERR_NULL,) * 3
+    assert interp_calls(lib, 1.0, 32.0, D=96) == (jl.JL_ERR_UNSUPPORTED,) * 3
+    assert interp_calls(lib, 1.0, 32.0, wsb=0) == (jl.JL_ERR_WORKSPACE,) * 3

@@ -10,12 +10,15 @@ from .jetlong import (  # noqa: F401
     JL_F32,
     JetLongError,
     jetlong_decode,
+    jetlong_decode_interp,
     jetlong_decode_workspace_size,
     jetlong_device_status,
     jetlong_group_size,
     jetlong_prefill,
     jetlong_prefill_attend,
+    jetlong_prefill_interp,
     jetlong_prefill_chunk,
+    jetlong_prefill_chunk_interp,
     jetlong_prefill_chunk_workspace_size,
     jetlong_prefill_rotate,
     jetlong_prefill_three_pass,

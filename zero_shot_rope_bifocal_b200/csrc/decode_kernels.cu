@@ -203,15 +203,18 @@ __device__ __forceinline__ void qk_block(float (&sc)[4], const uint32_t (&q)[D /
 // theta_i / (2 pi) as a 64-bit binary fraction: the 64-bit product wraps
 // exactly, its top 32 bits are the signed phase in units of 2^-32 turn, and
 // the angle handed to the sine/cosine lies in [-pi, pi).  Warp w writes rows
-// w, w + nw, ... of the stage.
+// w, w + nw, ... of the stage.  Under the frequency-interpolation remote map
+// the correction angle is j (theta'_i - theta_i): Delta j = j, and omega_i
+// holds (theta'_i - theta_i) / (2 pi), a negative fraction in two's complement.
 template <int D>
-__device__ __forceinline__ void correction_rows(uint8_t *tab, int jt, int n, int G, int warp,
-                                                int nw, int lane, const uint64_t *omega) {
+__device__ __forceinline__ void correction_rows(uint8_t *tab, int jt, int n, int G, int interp,
+                                                int warp, int nw, int lane,
+                                                const uint64_t *omega) {
   using C = DecCfg<D>;
   constexpr float kTurnToRad = 1.4629180792671596e-09f;  // 2 pi / 2^32
   for (int tt = warp; tt < n; tt += nw) {
     const int j = jt + tt;
-    const uint64_t delta = static_cast<uint64_t>(static_cast<int64_t>(remap(j, G) - j));
+    const uint64_t delta = static_cast<uint64_t>(static_cast<int64_t>(interp ? j : remap(j, G) - j));
     if (lane < D / 4) {  // lane: channels 2 lane, 2 lane + 1
       const int i = 2 * lane;
       const int32_t p0 = static_cast<int32_t>((delta * omega[i]) >> 32);
@@ -303,8 +306,8 @@ decode_split_kernel(DecodeArgs a) {
     }
     const int ju = j_begin + u * P;
     if (p - ju > w0eff)
-      correction_rows<D>(dsm + C::CS + (u % kStages) * C::CS_TAB, ju, min(P, j_end - ju), G, warp, nh,
-                         lane, omega);
+      correction_rows<D>(dsm + C::CS + (u % kStages) * C::CS_TAB, ju, min(P, j_end - ju), G,
+                         a.interp, warp, nh, lane, omega);
     __syncwarp();
     if (lane == 0) mbar_arrive(tready(u % kStages));
     return true;
@@ -323,13 +326,26 @@ decode_split_kernel(DecodeArgs a) {
     // The first copies go out before the RoPE tables are computed.
     for (int u = 0; u < kStages && u < n_stage; ++u) issue(u);
   }
-  for (int i = tid; i < HALF; i += kDecThreads)
-    omega[i] = __double2ull_rn(rope_freq(i, D, static_cast<double>(a.theta)) *
-                               (0.15915494309189533577 * 18446744073709551616.0));
+  constexpr double kTurnsQ64 = 0.15915494309189533577 * 18446744073709551616.0;  // 2^64 / (2 pi)
+  for (int i = tid; i < HALF; i += kDecThreads) {
+    const double f = rope_freq(i, D, static_cast<double>(a.theta));
+    // interpolation: (theta' - theta) / (2 pi) lies in (-1/(2 pi), 0], inside int64 once scaled
+    omega[i] = a.interp
+                   ? static_cast<uint64_t>(__double2ll_rn(
+                         f * (interp_factor(f, a.L, a.w_pretrained, a.ramp_alpha, a.ramp_beta) - 1.0) *
+                         kTurnsQ64))
+                   : __double2ull_rn(f * kTurnsQ64);
+  }
   for (int idx = tid; idx < 2 * HALF; idx += kDecThreads) {
     const int i = idx < HALF ? idx : idx - HALF;
+    const double f = rope_freq(i, D, static_cast<double>(a.theta));
     float c, sn;
-    rope_cos_sin(idx < HALF ? p : remap(p, G), rope_freq(i, D, static_cast<double>(a.theta)), c, sn);
+    if (idx < HALF)
+      rope_cos_sin(p, f, c, sn);
+    else if (a.interp)  // RoPE'(x_q, p): true position, interpolated frequency
+      rope_cos_sin(p, f * interp_factor(f, a.L, a.w_pretrained, a.ramp_alpha, a.ramp_beta), c, sn);
+    else
+      rope_cos_sin(remap(p, G), f, c, sn);
     qcs[idx] = make_float2(c, sn);
   }
   __syncthreads();

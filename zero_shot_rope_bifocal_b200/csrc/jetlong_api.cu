@@ -4,6 +4,7 @@
 // Every check runs on the host before the first CUDA call, so an invalid call
 // returns its status without touching the device (and works on a machine with
 // no GPU at all).
+#include <cmath>
 #include <mutex>
 
 #include "../../include/jetlong.h"
@@ -88,6 +89,12 @@ int check_common(int B, int Hq, int Hkv, int L, int D) {
 int check_method(int w_pretrained, int w0, float theta) {
   if (w_pretrained < 1 || w0 < 0) return JL_ERR_SHAPE;
   if (!(theta > 0.f) || theta != theta) return JL_ERR_SHAPE;
+  return JL_OK;
+}
+
+// Ramp bounds of the frequency-interpolation remote map: finite, beta > alpha.
+int check_ramp(float alpha, float beta) {
+  if (!std::isfinite(alpha) || !std::isfinite(beta) || !(beta > alpha)) return JL_ERR_SHAPE;
   return JL_OK;
 }
 
@@ -235,6 +242,26 @@ int jetlong_prefill(const void *q, const void *k, const void *v, void *out, floa
   return JL_OK;
 }
 
+int jetlong_prefill_interp(const void *q, const void *k, const void *v, void *out, float *lse,
+                           int B, int Hq, int Hkv, int L, int D, int w_pretrained, int w0,
+                           float rope_theta, float ramp_alpha, float ramp_beta, int out_dtype,
+                           void *k_cache_out, int k_cache_capacity, void *workspace,
+                           size_t workspace_bytes, jl_stream_t stream) {
+  if (check_ramp(ramp_alpha, ramp_beta) != JL_OK) return JL_ERR_SHAPE;
+  PrefillArgs a;
+  const int st = prepare_prefill(kStageBoth, q, k, v, out, lse, B, Hq, Hkv, L, D, w_pretrained,
+                                 w0, rope_theta, out_dtype, k_cache_out, k_cache_capacity,
+                                 workspace, workspace_bytes, &a);
+  if (st != JL_OK) return st;
+  a.interp = 1;
+  a.ramp_alpha = ramp_alpha;
+  a.ramp_beta = ramp_beta;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (launch_rope_qk(a, s) != cudaSuccess) return JL_ERR_CUDA;
+  if (launch_prefill_attention(a, s) != cudaSuccess) return JL_ERR_CUDA;
+  return JL_OK;
+}
+
 int jetlong_prefill_rotate(const void *q, const void *k, const void *v, int B, int Hq, int Hkv,
                            int L, int D, int w_pretrained, float rope_theta, void *k_cache_out,
                            int k_cache_capacity, void *workspace, size_t workspace_bytes,
@@ -315,8 +342,10 @@ namespace {
 int cache_attention(const void *q, const void *k_cache, const void *v_cache, void *out, float *lse,
                     int B, int Hq, int Hkv, int nq, int q_pos0, int Lcap, int D, int w_pretrained,
                     int w0, float rope_theta, int out_dtype, void *workspace,
-                    size_t workspace_bytes, jl_stream_t stream) {
+                    size_t workspace_bytes, jl_stream_t stream, int interp = 0,
+                    float ramp_alpha = 0.f, float ramp_beta = 0.f) {
   if (!q || !k_cache || !v_cache || !out) return JL_ERR_NULL;
+  if (interp && check_ramp(ramp_alpha, ramp_beta) != JL_OK) return JL_ERR_SHAPE;
   if (nq < 1 || q_pos0 < 0) return JL_ERR_SHAPE;
   const long long L_ll = static_cast<long long>(q_pos0) + nq;
   if (L_ll > (1ll << 31) - 1) return JL_ERR_SHAPE;
@@ -359,6 +388,9 @@ int cache_attention(const void *q, const void *k_cache, const void *v_cache, voi
   a.theta = rope_theta;
   a.nq = nq;
   a.q_pos0 = q_pos0;
+  a.interp = interp;
+  a.ramp_alpha = ramp_alpha;
+  a.ramp_beta = ramp_beta;
   decode_plan(B * nq, Hkv, L, &a.n_split, &a.chunk);
   a.dev_error = dev->err;
   if (launch_decode(a, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return JL_ERR_CUDA;
@@ -393,6 +425,27 @@ int jetlong_prefill_chunk(const void *q, const void *k_cache, const void *v_cach
   return cache_attention(q, k_cache, v_cache, out, lse, B, Hq, Hkv, n, P0, Lcap, D,
                          w_pretrained, w0, rope_theta, out_dtype, workspace, workspace_bytes,
                          stream);
+}
+
+int jetlong_decode_interp(const void *q, const void *k_cache, const void *v_cache, void *out,
+                          float *lse, int B, int Hq, int Hkv, int L, int Lcap, int D,
+                          int w_pretrained, int w0, float rope_theta, float ramp_alpha,
+                          float ramp_beta, int out_dtype, void *workspace, size_t workspace_bytes,
+                          jl_stream_t stream) {
+  if (L < 1) return JL_ERR_SHAPE;
+  return cache_attention(q, k_cache, v_cache, out, lse, B, Hq, Hkv, 1, L - 1, Lcap, D,
+                         w_pretrained, w0, rope_theta, out_dtype, workspace, workspace_bytes,
+                         stream, 1, ramp_alpha, ramp_beta);
+}
+
+int jetlong_prefill_chunk_interp(const void *q, const void *k_cache, const void *v_cache,
+                                 void *out, float *lse, int B, int Hq, int Hkv, int P0, int n,
+                                 int Lcap, int D, int w_pretrained, int w0, float rope_theta,
+                                 float ramp_alpha, float ramp_beta, int out_dtype, void *workspace,
+                                 size_t workspace_bytes, jl_stream_t stream) {
+  return cache_attention(q, k_cache, v_cache, out, lse, B, Hq, Hkv, n, P0, Lcap, D,
+                         w_pretrained, w0, rope_theta, out_dtype, workspace, workspace_bytes,
+                         stream, 1, ramp_alpha, ramp_beta);
 }
 
 int jetlong_rope_cache(const void *k, void *k_cache, int B, int n, int Hkv, int D, int pos0,

@@ -70,6 +70,21 @@ __device__ __forceinline__ void rope_cos_sin(long long pos, double freq, float &
   sincosf(static_cast<float>(r), &s, &c);
 }
 
+// Frequency-interpolation remote map (the §4.7 / Table 6 ablation): the
+// remote branch scores pairs at their true positions with frequencies
+// theta'_t = theta_t * ((1 - gamma_t) / s + gamma_t), YaRN's per-frequency
+// ramp gamma_t = clamp((r_t - alpha) / (beta - alpha), 0, 1) over the turns
+// r_t = w_pretrained * theta_t / (2 pi) that frequency t makes within the
+// pretrained window, and s = max(1, L / w_pretrained), the continuous dynamic
+// factor of §3.1.  Returns theta'_t / theta_t.
+__device__ __forceinline__ double interp_factor(double freq, int L, int w_pretrained,
+                                                double alpha, double beta) {
+  const double s = fmax(1.0, static_cast<double>(L) / static_cast<double>(w_pretrained));
+  const double turns = static_cast<double>(w_pretrained) * freq * 0.15915494309189533577;
+  const double gam = fmin(1.0, fmax(0.0, (turns - alpha) / (beta - alpha)));
+  return (1.0 - gam) / s + gam;
+}
+
 __device__ __forceinline__ float bf2f(__nv_bfloat16 x) { return __bfloat162float(x); }
 
 // ---------------------------------------------------------------- launchers
@@ -97,6 +112,10 @@ struct PrefillArgs {
   int B, Hq, Hkv, L, D, w_pretrained, w0, G;
   float theta;
   int pass;  // PrefillPass
+  // remote map: 0 = positions aliased by f (the method), 1 = frequency
+  // interpolation with ramp bounds (ramp_alpha, ramp_beta) (the ablation)
+  int interp;
+  float ramp_alpha, ramp_beta;
   unsigned int *dev_error;
 };
 
@@ -127,6 +146,8 @@ struct DecodeArgs {
   // query i sees keys [0, q_pos0 + i].  q is [B, nq, Hq, D], out likewise,
   // lse [B, Hq, nq]; L is the longest key range, q_pos0 + nq.
   int nq, q_pos0;
+  int interp;  // remote map, as in PrefillArgs
+  float ramp_alpha, ramp_beta;
   unsigned int *dev_error;
 };
 

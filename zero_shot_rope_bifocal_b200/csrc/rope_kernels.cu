@@ -18,6 +18,9 @@
 // the native-window case of Appendix H) f is the identity and only the
 // true-position arrays are written.
 //
+// With the frequency-interpolation remote map (the §4.7 ablation) the remote
+// arrays hold RoPE'(x, i): true position, interpolated frequencies theta'_t.
+//
 // Cache writer (§3.2): k_cache[b, pos0 + t] = RoPE(k[b, t], pos0 + t).
 //
 // Each CTA forms the frequencies once, evaluates cos/sin once per (position,
@@ -66,7 +69,7 @@ __device__ __forceinline__ bool store_f16(__half *dst, int i, int half, const Ro
 
 __global__ void __launch_bounds__(kRopeThreads)
 rope_qk_kernel(PrefillArgs a) {
-  extern __shared__ float2 cs_smem[];  // [2][kPosPerCta][D/2] (cos, sin), then [D/2] freq
+  extern __shared__ float2 cs_smem[];  // [2][kPosPerCta][D/2] (cos, sin), then 2 x [D/2] freq
   const int half = a.D / 2;
   const int b = blockIdx.y;
   const int p_begin = blockIdx.x * kPosPerCta;
@@ -76,17 +79,23 @@ rope_qk_kernel(PrefillArgs a) {
   float2 *cs_remote = cs_smem + kPosPerCta * half;
 
   double *freq = reinterpret_cast<double *>(cs_smem + 2 * kPosPerCta * half);
+  double *freq_remote = freq + half;  // theta'_t (interpolation) or theta_t
   const double theta = static_cast<double>(a.theta);
-  for (int i = threadIdx.x; i < half; i += blockDim.x) freq[i] = rope_freq(i, a.D, theta);
+  for (int i = threadIdx.x; i < half; i += blockDim.x) {
+    const double f = rope_freq(i, a.D, theta);
+    freq[i] = f;
+    freq_remote[i] =
+        a.interp ? f * interp_factor(f, a.L, a.w_pretrained, a.ramp_alpha, a.ramp_beta) : f;
+  }
   __syncthreads();
   for (int idx = threadIdx.x; idx < npos * half * (two ? 2 : 1); idx += blockDim.x) {
     const int var = idx / (npos * half);
     const int rem = idx - var * npos * half;
     const int t = rem / half, i = rem - t * half;
     const int pos = p_begin + t;
-    const long long ppos = var == 0 ? pos : remap(pos, a.G);
+    const long long ppos = (var == 0 || a.interp) ? pos : remap(pos, a.G);
     float c, s;
-    rope_cos_sin(ppos, freq[i], c, s);
+    rope_cos_sin(ppos, var == 0 ? freq[i] : freq_remote[i], c, s);
     (var == 0 ? cs_true : cs_remote)[t * half + i] = make_float2(c, s);
   }
   __syncthreads();
@@ -171,7 +180,7 @@ rope_cache_kernel(const __nv_bfloat16 *__restrict__ k, __nv_bfloat16 *__restrict
 
 cudaError_t launch_rope_qk(const PrefillArgs &a, cudaStream_t stream) {
   const dim3 grid((a.L + kPosPerCta - 1) / kPosPerCta, a.B);
-  const size_t smem = 2 * kPosPerCta * (a.D / 2) * sizeof(float2) + (a.D / 2) * sizeof(double);
+  const size_t smem = 2 * kPosPerCta * (a.D / 2) * sizeof(float2) + 2 * (a.D / 2) * sizeof(double);
   rope_qk_kernel<<<grid, kRopeThreads, smem, stream>>>(a);
   return cudaGetLastError();
 }

@@ -56,6 +56,12 @@ SIGNATURES = {
                             _VP, _SZ, _VP]),
     "jetlong_decode_noalloc": (_I, [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _I, _I, _F,
                                     _I, _VP]),
+    "jetlong_prefill_interp": (_I, [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _I, _F, _F,
+                                    _F, _I, _VP, _I, _VP, _SZ, _VP]),
+    "jetlong_decode_interp": (_I, [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _I, _I, _F,
+                                   _F, _F, _I, _VP, _SZ, _VP]),
+    "jetlong_prefill_chunk_interp": (_I, [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _I,
+                                          _I, _I, _F, _F, _F, _I, _VP, _SZ, _VP]),
     "jetlong_rope_cache": (_I, [_VP, _VP, _I, _I, _I, _I, _I, _I, _F, _VP]),
     "jetlong_device_status": (_I, [_VP]),
     "jetlong_check_device_timeout": (_I, [_I, _VP]),
@@ -156,6 +162,23 @@ def jetlong_prefill(q, k, v, w_pretrained: int, w0: int, rope_theta: float, *,
                     out=None, lse=None, out_dtype=torch.bfloat16, want_lse: bool = True,
                     k_cache_out=None, workspace=None, stream=None):
     """Bifocal causal attention over a prompt.  Returns (out, lse or None)."""
+    return _prefill("jetlong_prefill", q, k, v, w_pretrained, w0, (float(rope_theta),), out, lse,
+                    out_dtype, want_lse, k_cache_out, workspace, stream)
+
+
+def jetlong_prefill_interp(q, k, v, w_pretrained: int, w0: int, rope_theta: float,
+                           ramp_alpha: float = 1.0, ramp_beta: float = 32.0, *, out=None,
+                           lse=None, out_dtype=torch.bfloat16, want_lse: bool = True,
+                           k_cache_out=None, workspace=None, stream=None):
+    """jetlong_prefill with the frequency-interpolation remote map (remote
+    pairs at true positions, interpolated frequencies).  Returns (out, lse)."""
+    return _prefill("jetlong_prefill_interp", q, k, v, w_pretrained, w0,
+                    (float(rope_theta), float(ramp_alpha), float(ramp_beta)), out, lse, out_dtype,
+                    want_lse, k_cache_out, workspace, stream)
+
+
+def _prefill(fn, q, k, v, w_pretrained, w0, method, out, lse, out_dtype, want_lse, k_cache_out,
+             workspace, stream):
     if q.dim() != 4 or k.dim() != 4:
         raise ValueError("q, k, v must be [B, L, H, D]")
     B, L, Hq, D = q.shape
@@ -181,11 +204,10 @@ def jetlong_prefill(q, k, v, w_pretrained: int, w0: int, rope_theta: float, *,
     need = jetlong_prefill_workspace_size(B, Hq, Hkv, L, D)
     if workspace is None:
         workspace = _ws(need, q.device)
-    st = lib().jetlong_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, L, D,
-                               int(w_pretrained), int(w0), float(rope_theta), od,
-                               _ptr(k_cache_out), cap, _ptr(workspace), workspace.numel(),
-                               _stream_ptr(stream))
-    _check("jetlong_prefill", st)
+    st = getattr(lib(), fn)(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, L, D,
+                            int(w_pretrained), int(w0), *method, od, _ptr(k_cache_out), cap,
+                            _ptr(workspace), workspace.numel(), _stream_ptr(stream))
+    _check(fn, st)
     return out, lse
 
 
@@ -256,6 +278,22 @@ def jetlong_decode(q, k_cache, v_cache, L: int, w_pretrained: int, w0: int, rope
                    out=None, lse=None, out_dtype=torch.bfloat16, want_lse: bool = True,
                    workspace=None, stream=None):
     """One decode step at position L-1 on a true-position cache.  Returns (out, lse)."""
+    return _decode("jetlong_decode", q, k_cache, v_cache, L, w_pretrained, w0,
+                   (float(rope_theta),), out, lse, out_dtype, want_lse, workspace, stream)
+
+
+def jetlong_decode_interp(q, k_cache, v_cache, L: int, w_pretrained: int, w0: int,
+                          rope_theta: float, ramp_alpha: float = 1.0, ramp_beta: float = 32.0, *,
+                          out=None, lse=None, out_dtype=torch.bfloat16, want_lse: bool = True,
+                          workspace=None, stream=None):
+    """jetlong_decode with the frequency-interpolation remote map."""
+    return _decode("jetlong_decode_interp", q, k_cache, v_cache, L, w_pretrained, w0,
+                   (float(rope_theta), float(ramp_alpha), float(ramp_beta)), out, lse, out_dtype,
+                   want_lse, workspace, stream)
+
+
+def _decode(fn, q, k_cache, v_cache, L, w_pretrained, w0, method, out, lse, out_dtype, want_lse,
+            workspace, stream):
     if q.dim() != 3 or k_cache.dim() != 4:
         raise ValueError("q must be [B, Hq, D] and the caches [B, Lcap, Hkv, D]")
     B, Hq, D = q.shape
@@ -274,10 +312,10 @@ def jetlong_decode(q, k_cache, v_cache, L: int, w_pretrained: int, w0: int, rope
         _require(lse, "lse", (B, Hq), torch.float32)
     if workspace is None:
         workspace = _ws(jetlong_decode_workspace_size(B, Hq, Hkv, int(L), D), q.device)
-    st = lib().jetlong_decode(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(out), _ptr(lse), B, Hq,
-                              Hkv, int(L), Lcap, D, int(w_pretrained), int(w0), float(rope_theta),
-                              od, _ptr(workspace), workspace.numel(), _stream_ptr(stream))
-    _check("jetlong_decode", st)
+    st = getattr(lib(), fn)(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(out), _ptr(lse), B, Hq,
+                            Hkv, int(L), Lcap, D, int(w_pretrained), int(w0), *method, od,
+                            _ptr(workspace), workspace.numel(), _stream_ptr(stream))
+    _check(fn, st)
     return out, lse
 
 
@@ -290,6 +328,23 @@ def jetlong_prefill_chunk(q, k_cache, v_cache, P0: int, w_pretrained: int, w0: i
                           want_lse: bool = True, workspace=None, stream=None):
     """Queries of a chunk at positions P0.. against a true-position cache that
     already holds the chunk's keys; one G from P0 + n.  Returns (out, lse)."""
+    return _chunk("jetlong_prefill_chunk", q, k_cache, v_cache, P0, w_pretrained, w0,
+                  (float(rope_theta),), out, lse, out_dtype, want_lse, workspace, stream)
+
+
+def jetlong_prefill_chunk_interp(q, k_cache, v_cache, P0: int, w_pretrained: int, w0: int,
+                                 rope_theta: float, ramp_alpha: float = 1.0,
+                                 ramp_beta: float = 32.0, *, out=None, lse=None,
+                                 out_dtype=torch.bfloat16, want_lse: bool = True, workspace=None,
+                                 stream=None):
+    """jetlong_prefill_chunk with the frequency-interpolation remote map."""
+    return _chunk("jetlong_prefill_chunk_interp", q, k_cache, v_cache, P0, w_pretrained, w0,
+                  (float(rope_theta), float(ramp_alpha), float(ramp_beta)), out, lse, out_dtype,
+                  want_lse, workspace, stream)
+
+
+def _chunk(fn, q, k_cache, v_cache, P0, w_pretrained, w0, method, out, lse, out_dtype, want_lse,
+           workspace, stream):
     if q.dim() != 4 or k_cache.dim() != 4:
         raise ValueError("q must be [B, n, Hq, D] and the caches [B, Lcap, Hkv, D]")
     B, n, Hq, D = q.shape
@@ -309,11 +364,10 @@ def jetlong_prefill_chunk(q, k_cache, v_cache, P0: int, w_pretrained: int, w0: i
     if workspace is None:
         workspace = _ws(jetlong_prefill_chunk_workspace_size(B, Hq, Hkv, int(P0), n, D),
                         q.device)
-    st = lib().jetlong_prefill_chunk(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(out), _ptr(lse),
-                                     B, Hq, Hkv, int(P0), n, Lcap, D, int(w_pretrained), int(w0),
-                                     float(rope_theta), od, _ptr(workspace), workspace.numel(),
-                                     _stream_ptr(stream))
-    _check("jetlong_prefill_chunk", st)
+    st = getattr(lib(), fn)(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(out), _ptr(lse), B, Hq,
+                            Hkv, int(P0), n, Lcap, D, int(w_pretrained), int(w0), *method, od,
+                            _ptr(workspace), workspace.numel(), _stream_ptr(stream))
+    _check(fn, st)
     return out, lse
 
 
