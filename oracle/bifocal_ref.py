@@ -429,9 +429,9 @@ def merge_three_pass(q, k, v, w_pretrained: int, w0: int, theta: float):
 # §4.7 ablation: frequency interpolation instead of position aliasing
 # --------------------------------------------------------------------------
 # Table 6 of the page compares the default remote map (positions aliased to
-# f(x) = floor(x / G)) with "YaRN-style frequency interpolation within the same
-# bifocal construction".  The page gives no formula for that variant; the
-# readings taken here (each also listed in the design notes):
+# f(x) = floor(x / G)) with a YaRN-like interpolation of the frequencies inside
+# the same bifocal scheme, but gives no formula for it; the readings taken
+# here (each also listed in the design notes):
 #
 # * The local band is untouched: pairs with 0 <= i - j <= w0 are scored at true
 #   positions with the pretrained frequencies.  Only the remote map changes.
