@@ -8,9 +8,11 @@ Decode and chunk comparisons read the same BF16 cache, built by the oracle
 """
 import pytest
 import torch
+from hypothesis import given, settings, strategies as st
 
 import oracle
 from parity_util import assert_lse, assert_o, f64
+from test_random_gpu import workloads
 from zero_shot_rope_bifocal_b200 import jetlong as jl
 from zero_shot_rope_bifocal_b200.synth import (WORKLOADS, Workload, decode_inputs,
                                                generation_inputs, prefill_inputs, sample_rows)
@@ -146,3 +148,53 @@ def test_chunks(B, Hq, Hkv, D, wp, w0, P0, n):
                                                  w.theta)
     assert_o(f64(out), o_ref, f"chunk P0={P0}")
     assert_lse(f64(lse), lse_ref, f"chunk P0={P0}")
+
+
+# ---------------------------------------------------------------- random shapes
+RAMPS = st.sampled_from([(1.0, 32.0), (0.5, 3.0), (-2.0, -1.0), (1e6, 2e6), (2.0, 8.0)])
+RANDOM = settings(max_examples=8, deadline=None, derandomize=True)
+
+
+@RANDOM
+@given(workloads(grps=[1, 2, 3, 4], max_L=700), RAMPS)
+def test_prefill_random_shapes(w, ramp):
+    x = prefill_inputs(w)
+    out, lse = jl.jetlong_prefill_interp(x.q.cuda(), x.k.cuda(), x.v.cuda(), w.w_pretrained, w.w0,
+                                         w.theta, *ramp, out_dtype=torch.float32)
+    assert jl.jetlong_device_status() == jl.JL_OK
+    o_ref, lse_ref = oracle.prefill_interp(f64(x.q), f64(x.k), f64(x.v), w.w_pretrained, w.w0,
+                                           w.theta, *ramp)
+    assert_o(f64(out), o_ref, f"{w} {ramp}")
+    assert_lse(f64(lse), lse_ref, f"{w} {ramp}")
+
+
+@RANDOM
+@given(workloads(grps=[1, 2, 4, 8], max_L=3000), RAMPS)
+def test_decode_random_shapes(w, ramp):
+    d = decode_inputs(w, Lcap=w.L + 2)
+    cache = cache_bf16(d.k_raw, w.theta)
+    out, lse = jl.jetlong_decode_interp(d.q.cuda(), cache.cuda(), d.v.cuda(), w.L, w.w_pretrained,
+                                        w.w0, w.theta, *ramp, out_dtype=torch.float32)
+    assert jl.jetlong_device_status() == jl.JL_OK
+    o_ref, lse_ref = oracle.decode_interp(f64(d.q), f64(cache), f64(d.v), w.L, w.w_pretrained,
+                                          w.w0, w.theta, *ramp)
+    assert_o(f64(out), o_ref, f"{w} {ramp}")
+    assert_lse(f64(lse), lse_ref, f"{w} {ramp}")
+
+
+@RANDOM
+@given(workloads(grps=[1, 2, 4, 8], max_L=1500), RAMPS, st.data())
+def test_prefill_chunk_random_shapes(w, ramp, data):
+    n = data.draw(st.integers(1, min(w.L, 40)))
+    P0 = w.L - n
+    x = prefill_inputs(w)
+    cache = cache_bf16(x.k, w.theta)
+    qc = x.q[:, P0:].contiguous()
+    out, lse = jl.jetlong_prefill_chunk_interp(qc.cuda(), cache.cuda(), x.v.cuda(), P0,
+                                               w.w_pretrained, w.w0, w.theta, *ramp,
+                                               out_dtype=torch.float32)
+    assert jl.jetlong_device_status() == jl.JL_OK
+    o_ref, lse_ref = oracle.prefill_chunk_interp(f64(qc), f64(cache), f64(x.v), P0,
+                                                 w.w_pretrained, w.w0, w.theta, *ramp)
+    assert_o(f64(out), o_ref, f"{w} {ramp}")
+    assert_lse(f64(lse), lse_ref, f"{w} {ramp}")

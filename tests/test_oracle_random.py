@@ -64,3 +64,30 @@ def test_cache_formulation_equals_the_direct_rule(prob, data):
     o, lse = oracle.prefill(q, k, v, wp, w0, theta)
     np.testing.assert_allclose(oc, o[:, P0:], atol=1e-10)
     np.testing.assert_allclose(lc, lse[:, :, P0:], atol=1e-10)
+
+
+# ---------------------------------------------------------------- frequency-interpolation map
+RAMPS = st.sampled_from([(1.0, 32.0), (0.5, 3.0), (-2.0, -1.0), (1e6, 2e6), (2.0, 8.0)])
+
+
+@SETTINGS
+@given(problems(max_L=14), RAMPS)
+def test_interp_vectorised_prefill_equals_the_literal_per_pair_loop(prob, ramp):
+    q, k, v, wp, w0, theta = prob
+    o1, l1 = oracle.prefill_interp(q, k, v, wp, w0, theta, *ramp)
+    o2, l2 = oracle.prefill_interp_literal(q, k, v, wp, w0, theta, *ramp)
+    np.testing.assert_allclose(o1, o2, atol=1e-11)
+    np.testing.assert_allclose(l1, l2, atol=1e-11)
+
+
+@SETTINGS
+@given(problems(), RAMPS, st.data())
+def test_interp_cache_formulation_equals_the_direct_rule(prob, ramp, data):
+    q, k, v, wp, w0, theta = prob
+    L = q.shape[1]
+    P0 = data.draw(st.integers(0, L - 1))
+    cache = oracle.rope_cache(k, 0, theta)
+    oc, lc = oracle.prefill_chunk_interp(q[:, P0:], cache, v, P0, wp, w0, theta, *ramp)
+    o, lse = oracle.prefill_interp(q, k, v, wp, w0, theta, *ramp)
+    np.testing.assert_allclose(oc, o[:, P0:], atol=1e-10)
+    np.testing.assert_allclose(lc, lse[:, :, P0:], atol=1e-10)
