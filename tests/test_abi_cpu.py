@@ -265,3 +265,22 @@ def test_interp_checks_the_same_arguments_as_the_aliasing_calls(lib):
     assert interp_calls(lib, 1.0, 32.0, q=None) == (jl.JL_ERR_NULL,) * 3
     assert interp_calls(lib, 1.0, 32.0, D=96) == (jl.JL_ERR_UNSUPPORTED,) * 3
     assert interp_calls(lib, 1.0, 32.0, wsb=0) == (jl.JL_ERR_WORKSPACE,) * 3
+
+
+def test_decode_split_plan_fills_at_most_one_wave():
+    # The decode grid is splits x ceil(Hkv / 8) x B CTAs at two CTAs per SM on
+    # 148 SMs: the plan never starts a second wave (unless one split per
+    # unit already does), and never splits finer than one 16-token stage.
+    for B in (1, 2, 3, 4, 64, 300):
+        for Hkv, Hq, D in ((8, 32, 128), (16, 16, 128), (2, 16, 64), (12, 24, 64)):
+            units = B * -(-Hkv // 8)
+            for L in (1, 15, 16, 17, 100, 4096, 32768, 131072, 1 << 20):
+                ws = jl.jetlong_decode_workspace_size(B, Hq, Hkv, L, D)
+                if B * L * Hq > 1 << 31:                  # beyond the index range: refused
+                    assert ws == 0
+                    continue
+                per_split = B * Hq * (D + 2) * 4
+                ns = ws // per_split
+                assert ws - ns * per_split < 256          # only alignment padding left
+                assert 1 <= ns <= -(-L // 16)
+                assert units * ns <= max(2 * 148, units)
