@@ -7,7 +7,8 @@ One step = one prefill of a Qwen3-8B-shaped attention layer at L = 131072
 (B=1, Hq=32, Hkv=8, D=128, w_pretrained=32768, w0=4096, theta=1e6, G=4):
 the RoPE operand pass (jetlong_prefill_rotate) followed by the attention
 kernel (jetlong_prefill_attend), with inputs resident in HBM.  The headline
-``value`` is algorithmic prefill TFLOP/s = 4 * B * Hq * D * L(L+1)/2 / time.
+``value`` is algorithmic prefill TFLOP/s = 4 * B * Hq * D * L(L+1)/2 / time
+(also given as prompt tokens per second, ``tokens_per_s``).
 After the prefill steps, 256 decode steps on a 131072-token true-position
 cache (Qwen3-8B shapes) are timed the same way and reported as microseconds
 per token and achieved HBM bandwidth over the K+V bytes a step must read.
@@ -625,7 +626,9 @@ def run_native(args):
         peak = peaks["bf16_tflops_sustained"]
         line = {
             "metric": "bifocal-attn prefill TFLOP/s @128K (Qwen3-8B layer); decode us/token",
-            "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "value": value, "unit": "TFLOP/s",
+            "tokens_per_s": value * 1e12 / prefill_flops(B, Hq, L, D) * B * L,
+            "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": t_max / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f16",
             "precision": "BF16 inputs and outputs; FP16 tensor-core operands (rotated Q/K, V, "
@@ -639,7 +642,8 @@ def run_native(args):
                          "kernel": "bifocal_prefill_kernel<128>", "kernel_ms": attn_ms,
                          "traffic": None},
             "breakdown_ms": {"rotate": rot_ms, "attend": attn_ms},
-            "decode": {"workload": DECODE_WORKLOAD, "us_per_token": us_tok, "steps": n_dec,
+            "decode": {"workload": DECODE_WORKLOAD, "us_per_token": us_tok,
+                       "tokens_per_s": wd.B * 1e6 / us_tok, "steps": n_dec,
                        "loop": dec_loop, "host_loop_us_per_token": host_loop_us,
                        "achieved_gbs": dec_gbs, "peak_gbs": peaks["hbm_gbs"],
                        "frac": dec_gbs / peaks["hbm_gbs"],
