@@ -44,6 +44,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
+METRIC = "bifocal-attn prefill TFLOP/s (% BF16 peak) @128K; decode µs/token (% HBM BW)"
 PREFILL_WORKLOAD = "qwen3_8b_128k"
 DECODE_WORKLOAD = "decode_8b_128k"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -259,7 +260,7 @@ def run_reference(args):
         tot_f, tot_t, nrows = tot_f + f, tot_t + t, nrows + len(done)
     value = tot_f / tot_t / 1e12
     line = {
-        "impl": "reference", "metric": "bifocal-attn prefill TFLOP/s @128K (Qwen3-8B layer)",
+        "impl": "reference", "metric": METRIC,
         "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": 1e3 * tot_t / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
@@ -625,7 +626,7 @@ def run_native(args):
         attn_tflops = prefill_flops(B, Hq, L, D) / (attn_ms * 1e-3) / 1e12
         peak = peaks["bf16_tflops_sustained"]
         line = {
-            "metric": "bifocal-attn prefill TFLOP/s @128K (Qwen3-8B layer); decode us/token",
+            "metric": METRIC,
             "value": value, "unit": "TFLOP/s",
             "tokens_per_s": value * 1e12 / prefill_flops(B, Hq, L, D) * B * L,
             "n_gpus": world, "steps": args.steps,
