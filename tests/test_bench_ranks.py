@@ -90,3 +90,31 @@ def test_work_accounting():
     assert bench.prefill_flops(1, 32, 131072, 128) == 4 * 32 * 128 * 131072 * 131073 // 2
     assert bench.decode_bytes(1, 8, 131072, 128) == 2 * 131072 * 8 * 128 * 2
     assert bench.row_flops(32, 128, [0, 9]) == 4 * 32 * 128 * (1 + 10)
+
+
+def test_reference_arm_line(monkeypatch, capsys):
+    # The oracle arm on this machine's cores: one JSON line with the native
+    # arm's metric and config, a cpu_baseline describing the run, and an e2e
+    # entry with no host-device traffic.  (Run on the tiny workload here, to
+    # keep the CPU suite short; the format does not depend on the size.)
+    import json
+    for k in ("RANK", "WORLD_SIZE", "LOCAL_RANK"):
+        monkeypatch.delenv(k, raising=False)
+    monkeypatch.setattr(bench, "PREFILL_WORKLOAD", "tiny")
+    assert bench.main(["--impl", "reference", "--steps", "1", "--warmup", "3",
+                       "--reference-seconds", "8"]) == 0
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["metric"] == bench.METRIC
+    assert line["unit"] == "TFLOP/s" and line["higher_is_better"] is True
+    assert line["config"]["workload"] == bench.PREFILL_WORKLOAD
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["value"] == line["value"]
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0
+    assert line["value"] > 0
+
+
+def test_reference_arm_other_ranks_exit_without_work(monkeypatch, capsys):
+    monkeypatch.setenv("RANK", "1")
+    monkeypatch.setenv("WORLD_SIZE", "2")
+    monkeypatch.setenv("LOCAL_RANK", "1")
+    assert bench.main(["--impl", "reference", "--steps", "1"]) == 0
+    assert capsys.readouterr().out == ""
