@@ -446,7 +446,7 @@ def merge_three_pass(q, k, v, w_pretrained: int, w0: int, theta: float):
 # * s is the dynamic factor the page names for continuous rescaling in §3.1,
 #   s = max(1, L / w_pretrained), recomputed from the current length like G.
 # * No attention temperature: the softmax scale stays 1/sqrt(D) (the ablation
-#   changes the remote-window mapping only).
+#   changes only how remote positions are mapped).
 # * The cache still holds RoPE(x_k, j) at true positions (§3.2); a cached key
 #   is turned into the remote form by the rotation of angle j (theta'_t - theta_t).
 def interp_scale(L: int, w_pretrained: int) -> float:
