@@ -91,3 +91,15 @@ def test_interp_cache_formulation_equals_the_direct_rule(prob, ramp, data):
     o, lse = oracle.prefill_interp(q, k, v, wp, w0, theta, *ramp)
     np.testing.assert_allclose(oc, o[:, P0:], atol=1e-10)
     np.testing.assert_allclose(lc, lse[:, :, P0:], atol=1e-10)
+
+
+@SETTINGS
+@given(problems(), RAMPS)
+def test_interp_decode_equals_the_last_prefill_row(prob, ramp):
+    q, k, v, wp, w0, theta = prob
+    L = q.shape[1]
+    cache = oracle.rope_cache(k, 0, theta)
+    od, ld = oracle.decode_interp(q[:, L - 1], cache, v, L, wp, w0, theta, *ramp)
+    o, lse = oracle.prefill_interp_rows(q, k, v, wp, w0, theta, [L - 1], *ramp)
+    np.testing.assert_allclose(od, o[:, 0], atol=1e-10)
+    np.testing.assert_allclose(ld, lse[:, :, 0], atol=1e-10)
