@@ -8,6 +8,9 @@ a prompt) do not divide by ~0.  A BF16 output adds its own rounding
 """
 import numpy as np
 import torch
+from hypothesis import strategies as st
+
+from zero_shot_rope_bifocal_b200.synth import Workload
 
 O_ATOL = 1e-2
 LSE_RTOL = 1e-3
@@ -43,3 +46,20 @@ def assert_lse(gpu, ref, what=""):
     e = lse_err(gpu, ref)
     assert e <= LSE_RTOL, f"{what} LSE relative error {e:.3e} > {LSE_RTOL}"
     return e
+
+
+@st.composite
+def workloads(draw, grps, max_L):
+    """Random small workloads for the randomised parity tests: ragged L,
+    GQA ratios from ``grps``, both head dimensions, w0 from 0 to beyond L,
+    G from 1 up (w_pretrained from 1 to beyond L)."""
+    L = draw(st.integers(1, max_L))
+    Hkv = draw(st.sampled_from([1, 2, 3]))
+    grp = draw(st.sampled_from(grps))
+    D = draw(st.sampled_from([64, 128]))
+    wp = draw(st.integers(1, L + 64))
+    w0 = draw(st.integers(0, L + 8))
+    B = draw(st.integers(1, 2))
+    theta = draw(st.sampled_from([1e4, 1e6]))
+    seed = draw(st.integers(0, 10**6))
+    return Workload("rand", B, Hkv * grp, Hkv, D, L, wp, w0, theta, seed, seed % 2 == 0)

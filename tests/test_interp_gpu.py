@@ -11,8 +11,7 @@ import torch
 from hypothesis import given, settings, strategies as st
 
 import oracle
-from parity_util import assert_lse, assert_o, f64
-from test_random_gpu import workloads
+from parity_util import assert_lse, assert_o, f64, workloads
 from zero_shot_rope_bifocal_b200 import jetlong as jl
 from zero_shot_rope_bifocal_b200.synth import (WORKLOADS, Workload, decode_inputs,
                                                generation_inputs, prefill_inputs, sample_rows)

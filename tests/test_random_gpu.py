@@ -9,26 +9,12 @@ import torch
 from hypothesis import given, settings, strategies as st
 
 import oracle
-from parity_util import assert_lse, assert_o, f64
+from parity_util import assert_lse, assert_o, f64, workloads
 from zero_shot_rope_bifocal_b200 import jetlong as jl
-from zero_shot_rope_bifocal_b200.synth import Workload, decode_inputs, prefill_inputs
+from zero_shot_rope_bifocal_b200.synth import decode_inputs, prefill_inputs
 
 pytestmark = pytest.mark.gpu
 SETTINGS = settings(max_examples=12, deadline=None, derandomize=True)
-
-
-@st.composite
-def workloads(draw, grps, max_L):
-    L = draw(st.integers(1, max_L))
-    Hkv = draw(st.sampled_from([1, 2, 3]))
-    grp = draw(st.sampled_from(grps))
-    D = draw(st.sampled_from([64, 128]))
-    wp = draw(st.integers(1, L + 64))
-    w0 = draw(st.integers(0, L + 8))
-    B = draw(st.integers(1, 2))
-    theta = draw(st.sampled_from([1e4, 1e6]))
-    seed = draw(st.integers(0, 10**6))
-    return Workload("rand", B, Hkv * grp, Hkv, D, L, wp, w0, theta, seed, seed % 2 == 0)
 
 
 @SETTINGS
