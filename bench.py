@@ -205,6 +205,16 @@ def oracle_rows_per_sec(w, seconds: float, q_rows_src, k, v, rows):
     return flops, time.perf_counter() - t0, done_rows
 
 
+def oracle_rate_extras(w, flops: float, seconds: float, rows_done) -> dict:
+    """Rows per second of the timed oracle sample, and the time the whole
+    prefill of ``w`` would take at the sample's FLOP rate (an extrapolation:
+    row costs grow with the row index, so the rate, not the row count, is
+    scaled)."""
+    rate = flops / seconds
+    return {"rows_per_s": len(rows_done) / seconds,
+            "extrapolated_full_prefill_s": prefill_flops(w.B, w.Hq, w.L, w.D) / rate}
+
+
 def cpu_sample_inputs(w, n_rows: int, device):
     """Inputs of ``w`` for oracle timing: the query rows to time and K/V as fp32 numpy."""
     import numpy as np
@@ -252,12 +262,13 @@ def run_reference(args):
     per_step = max(2.0, args.reference_seconds / max(1, args.steps + args.warmup))
     for _ in range(args.warmup):
         oracle_rows_per_sec(w, per_step, q_rows, k, v, rows)
-    tot_f, tot_t, nrows = 0, 0.0, 0
+    tot_f, tot_t, all_done = 0, 0.0, []
     for s in range(args.steps):
         rot = rows[s % len(rows):] + rows[:s % len(rows)]
         qrot = q_rows[:, [rows.index(r) for r in rot]]
         f, t, done = oracle_rows_per_sec(w, per_step, qrot, k, v, rot)
-        tot_f, tot_t, nrows = tot_f + f, tot_t + t, nrows + len(done)
+        tot_f, tot_t, all_done = tot_f + f, tot_t + t, all_done + done
+    nrows = len(all_done)
     value = tot_f / tot_t / 1e12
     line = {
         "impl": "reference", "metric": METRIC,
@@ -269,7 +280,8 @@ def run_reference(args):
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads_used(),
                          "kind": "oracle",
                          "sample": f"{nrows} query rows (all 32 heads) of the 128K prefill, "
-                                   f"random rows in [L/2, L), ~{per_step:.0f} s per step"},
+                                   f"random rows in [L/2, L), ~{per_step:.0f} s per step",
+                         **oracle_rate_extras(w, tot_f, tot_t, all_done)},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -619,7 +631,8 @@ def run_native(args):
         f, t, done = oracle_rows_per_sec(w, args.cpu_seconds, q_rows, kk, vv, rows)
         cpu = {"value": f / t / 1e12, "unit": "TFLOP/s", "cores": threads_used(), "kind": "oracle",
                "sample": f"{len(done)} query rows (all 32 heads) of the 128K prefill, random rows "
-                         f"in [L/2, L), {t:.1f} s of fp64 NumPy"}
+                         f"in [L/2, L), {t:.1f} s of fp64 NumPy",
+               **oracle_rate_extras(w, f, t, done)}
 
     if rank == 0:
         peaks, src = load_peaks()

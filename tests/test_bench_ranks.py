@@ -109,6 +109,8 @@ def test_reference_arm_line(monkeypatch, capsys):
     assert line["config"]["workload"] == bench.PREFILL_WORKLOAD
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["value"] == line["value"]
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0
+    assert line["cpu_baseline"]["rows_per_s"] > 0
+    assert line["cpu_baseline"]["extrapolated_full_prefill_s"] > 0
     assert line["value"] > 0
 
 
@@ -118,3 +120,12 @@ def test_reference_arm_other_ranks_exit_without_work(monkeypatch, capsys):
     monkeypatch.setenv("LOCAL_RANK", "1")
     assert bench.main(["--impl", "reference", "--steps", "1"]) == 0
     assert capsys.readouterr().out == ""
+
+
+def test_oracle_rate_extras():
+    from zero_shot_rope_bifocal_b200.synth import WORKLOADS
+    w = WORKLOADS["qwen3_8b_128k"]
+    full = bench.prefill_flops(w.B, w.Hq, w.L, w.D)
+    x = bench.oracle_rate_extras(w, full / 1000.0, 2.0, [5, 6, 7, 8])
+    assert x["rows_per_s"] == 2.0
+    assert abs(x["extrapolated_full_prefill_s"] - 2000.0) < 1e-6
