@@ -217,9 +217,8 @@ def oracle_rate_extras(w, flops: float, seconds: float, rows_done) -> dict:
 
 def cpu_sample_inputs(w, n_rows: int, device):
     """Inputs of ``w`` for oracle timing: the query rows to time and K/V as fp32 numpy."""
-    import numpy as np
     import torch
-    from zero_shot_rope_bifocal_b200.synth import prefill_inputs, sample_rows
+    from zero_shot_rope_bifocal_b200.synth import prefill_inputs
     x = prefill_inputs(w, device=device)
     g = torch.Generator().manual_seed(1234)
     rows = sorted(torch.randint(w.L // 2, w.L, (n_rows,), generator=g).tolist())

@@ -6,7 +6,6 @@ device times and the sum of their work.  No collective touches the data path.
 import os
 import socket
 
-import pytest
 import torch.multiprocessing as mp
 
 import bench

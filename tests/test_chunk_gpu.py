@@ -6,7 +6,6 @@ call from P0 + n (Jet-Long paper, §3.1, §3.2).
 Both sides read the same BF16 cache, built by the oracle (true-position RoPE
 in fp64, rounded to BF16), as in the decode tests.
 """
-import numpy as np
 import pytest
 import torch
 

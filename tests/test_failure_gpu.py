@@ -2,7 +2,6 @@
 without a fault: a wait on an mbarrier that nothing completes gives up after
 its limit, the kernel records a timeout, the host reads it through
 jetlong_device_status(), and the context keeps working."""
-import numpy as np
 import pytest
 import torch
 

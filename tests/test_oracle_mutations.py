@@ -7,7 +7,6 @@ import contextlib
 import inspect
 import textwrap
 
-import numpy as np
 import pytest
 
 import oracle

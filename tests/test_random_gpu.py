@@ -3,7 +3,6 @@ small random shapes: ragged lengths, every supported GQA ratio, both head
 dimensions, w0 from 0 to beyond L, G from 1 up.  Hypothesis is derandomised,
 so every run draws the same cases; inputs come from the seeded generators.
 """
-import numpy as np
 import pytest
 import torch
 from hypothesis import given, settings, strategies as st

@@ -6,7 +6,6 @@ merged as (W_A O_A + W_B O_B - W_C O_C) / (W_A + W_B - W_C).
 It must agree with the fp64 oracle's direct rule (same tolerances as the
 fused kernel) and with the fused GPU kernel on the same inputs.
 """
-import numpy as np
 import pytest
 import torch
 
