@@ -127,7 +127,9 @@ JL_API size_t jetlong_prefill_workspace_size(int B, int Hq, int Hkv, int L, int 
  *   out [B, L, Hq,  D] out_dtype (JL_BF16 or JL_F32)    (written)
  *   lse [B, Hq, L] float32, natural-log log-sum-exp of the scaled scores per
  *       row (written; may be NULL)
- *   w_pretrained >= 1, w0 >= 0, rope_theta > 0.
+ *   w_pretrained >= 1, w0 >= 0, rope_theta > 0.  D is 64 or 128; Hq is a
+ *   multiple of Hkv; B * L * Hq <= 2^31; B <= 65535 and
+ *   Hkv * ceil(Hq / Hkv / 2) <= 65535 (CUDA grid limits).
  *   k_cache_out: NULL, or [B, k_cache_capacity, Hkv, D] BF16; rows [0, L) are
  *       written with RoPE(x_k, k) at true positions (§3.2), the cache decode
  *       expects.  k_cache_capacity >= L (ignored when k_cache_out is NULL).
@@ -243,7 +245,8 @@ JL_API size_t jetlong_decode_workspace_size(int B, int Hq, int Hkv, int L, int D
  *      scored against RoPE(x_q, f(L-1)).
  *   workspace: >= jetlong_decode_workspace_size(B, Hq, Hkv, L, D) bytes,
  *      256-byte aligned; contents on entry do not matter.
- *   Hq / Hkv must be 1, 2, 4 or 8 (JL_ERR_UNSUPPORTED otherwise).
+ *   Hq / Hkv must be 1, 2, 4 or 8 (JL_ERR_UNSUPPORTED otherwise);
+ *   Hkv <= 8 * 65535 (CUDA grid limit).
  */
 JL_API int jetlong_decode(const void *q, const void *k_cache, const void *v_cache, void *out,
                    float *lse, int B, int Hq, int Hkv, int L, int Lcap, int D,
@@ -324,7 +327,7 @@ JL_API int jetlong_prefill_chunk_interp(const void *q, const void *k_cache, cons
  *
  *   k        [B, n, Hkv, D] BF16 pre-RoPE keys (read)
  *   k_cache  [B, Lcap, Hkv, D] BF16 (rows [pos0, pos0 + n) written)
- *   0 <= pos0, n >= 1, pos0 + n <= Lcap.
+ *   0 <= pos0, n >= 1, pos0 + n <= Lcap, 1 <= B <= 65535.
  */
 JL_API int jetlong_rope_cache(const void *k, void *k_cache, int B, int n, int Hkv, int D,
                        int pos0, int Lcap, float rope_theta, jl_stream_t stream);

@@ -109,6 +109,8 @@ def prefill_call(lib, **kw):
     (dict(ws=None), jl.JL_ERR_WORKSPACE),
     (dict(wsb=10), jl.JL_ERR_WORKSPACE),
     (dict(ws=ctypes.c_void_p(272)), jl.JL_ERR_ALIGN),
+    (dict(B=65536, L=1), jl.JL_ERR_SHAPE),              # grid z (batch) beyond 65535
+    (dict(Hq=70000, Hkv=70000, L=1), jl.JL_ERR_SHAPE),  # grid y (head pairs) beyond 65535
 ])
 def test_prefill_rejects_bad_arguments(lib, kw, status):
     assert prefill_call(lib, **kw) == status
@@ -204,6 +206,7 @@ def decode_call(lib, **kw):
     (dict(w0=-5), jl.JL_ERR_SHAPE),
     (dict(vc=ctypes.c_void_p(8)), jl.JL_ERR_ALIGN),
     (dict(wsb=0), jl.JL_ERR_WORKSPACE),
+    (dict(Hq=524288, Hkv=524288, L=1, Lcap=1), jl.JL_ERR_SHAPE),  # grid y beyond 65535
 ])
 def test_decode_rejects_bad_arguments(lib, kw, status):
     assert decode_call(lib, **kw) == status
@@ -215,6 +218,7 @@ def test_decode_rejects_bad_arguments(lib, kw, status):
     ((P, P, 1, 0, 2, 128, 0, 8, 1e4, None), jl.JL_ERR_SHAPE),
     ((P, P, 1, 4, 2, 48, 0, 8, 1e4, None), jl.JL_ERR_UNSUPPORTED),
     ((P, P, 1, 4, 2, 128, -1, 8, 1e4, None), jl.JL_ERR_SHAPE),
+    ((P, P, 65536, 4, 2, 128, 0, 8, 1e4, None), jl.JL_ERR_SHAPE),  # grid y (batch) > 65535
 ])
 def test_rope_cache_rejects_bad_arguments(lib, args, status):
     assert lib.jetlong_rope_cache(*args) == status

@@ -20,6 +20,7 @@ __device__ unsigned int g_device_error;
 namespace {
 
 constexpr size_t kAlign = 256;
+constexpr long long kMaxGridYZ = 65535;  // CUDA's limit on gridDim.y and gridDim.z
 
 size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
@@ -178,6 +179,10 @@ int prepare_prefill(int stage, const void *q, const void *k, const void *v, void
   if (att && !out) return JL_ERR_NULL;
   int st = check_common(B, Hq, Hkv, L, D);
   if (st != JL_OK) return st;
+  // grids: (positions, batch) for the operand pass, (query tiles, KV heads x
+  // head pairs, batch) for the attention kernel
+  if (B > kMaxGridYZ || static_cast<long long>(Hkv) * ((Hq / Hkv + 1) / 2) > kMaxGridYZ)
+    return JL_ERR_SHAPE;
   if ((st = check_method(w_pretrained, w0, rope_theta)) != JL_OK) return st;
   if (att && out_dtype != JL_BF16 && out_dtype != JL_F32) return JL_ERR_UNSUPPORTED;
   if (rot && k_cache_out && k_cache_capacity < L) return JL_ERR_SHAPE;
@@ -356,6 +361,7 @@ int cache_attention(const void *q, const void *k_cache, const void *v_cache, voi
   if (static_cast<long long>(B) * nq * Hq * L > (1ll << 40)) return JL_ERR_SHAPE;
   if (Lcap < L) return JL_ERR_SHAPE;
   if (!decode_supports_group(Hq / Hkv)) return JL_ERR_UNSUPPORTED;
+  if ((Hkv + 7) / 8 > kMaxGridYZ) return JL_ERR_SHAPE;  // grid y: groups of 8 KV heads
   if ((st = check_method(w_pretrained, w0, rope_theta)) != JL_OK) return st;
   if (out_dtype != JL_BF16 && out_dtype != JL_F32) return JL_ERR_UNSUPPORTED;
   if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out) ||
@@ -451,7 +457,7 @@ int jetlong_prefill_chunk_interp(const void *q, const void *k_cache, const void 
 int jetlong_rope_cache(const void *k, void *k_cache, int B, int n, int Hkv, int D, int pos0,
                        int Lcap, float rope_theta, jl_stream_t stream) {
   if (!k || !k_cache) return JL_ERR_NULL;
-  if (B < 1 || n < 1 || Hkv < 1 || pos0 < 0 || Lcap < 1) return JL_ERR_SHAPE;
+  if (B < 1 || B > kMaxGridYZ || n < 1 || Hkv < 1 || pos0 < 0 || Lcap < 1) return JL_ERR_SHAPE;
   if (static_cast<long long>(pos0) + n > Lcap) return JL_ERR_SHAPE;
   if (D != 64 && D != 128) return JL_ERR_UNSUPPORTED;
   if (!(rope_theta > 0.f)) return JL_ERR_SHAPE;
