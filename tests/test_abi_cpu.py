@@ -288,3 +288,14 @@ def test_decode_split_plan_fills_at_most_one_wave():
                 assert ws - ns * per_split < 256          # only alignment padding left
                 assert 1 <= ns <= -(-L // 16)
                 assert units * ns <= max(2 * 148, units)
+
+
+def test_binding_refuses_host_memory_as_workspace_or_operand():
+    # a host pointer handed to the kernels would be dereferenced on the GPU
+    import torch
+    with pytest.raises(ValueError, match="workspace must be a CUDA tensor"):
+        jl._workspace(torch.empty(64, dtype=torch.uint8), 64, None)
+    with pytest.raises(ValueError, match="workspace must be a CUDA tensor"):
+        jl._workspace(bytearray(64), 64, None)
+    with pytest.raises(ValueError, match="must be a CUDA tensor"):
+        jl._require(torch.empty((1, 2), dtype=torch.bfloat16), "q", (1, 2), torch.bfloat16)

@@ -116,6 +116,10 @@ def _require(t, name, shape, dtype):
         raise TypeError(f"{name} must be a torch.Tensor")
     if not t.is_cuda:
         raise ValueError(f"{name} must be a CUDA tensor")
+    if t.device.index != torch.cuda.current_device():
+        # the library launches on the current device (and its stream)
+        raise ValueError(f"{name} is on {t.device}, but the current CUDA device is "
+                         f"cuda:{torch.cuda.current_device()}; use torch.cuda.set_device")
     if tuple(t.shape) != tuple(shape):
         raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
     if t.dtype != dtype:
@@ -135,6 +139,21 @@ def _out_dtype(dtype) -> int:
 def _ws(nbytes: int, device) -> torch.Tensor:
     # torch's caching allocator returns blocks aligned to at least 512 bytes.
     return torch.empty(max(int(nbytes), 1), dtype=torch.uint8, device=device)
+
+
+def _workspace(workspace, nbytes: int, device):
+    """The caller's workspace (checked: a contiguous tensor on the current
+    CUDA device), or a new one of ``nbytes``.  Returns (tensor, its bytes)."""
+    if workspace is None:
+        workspace = _ws(nbytes, device)
+    elif not isinstance(workspace, torch.Tensor) or not workspace.is_cuda:
+        raise ValueError("workspace must be a CUDA tensor")
+    elif workspace.device.index != torch.cuda.current_device():
+        raise ValueError(f"workspace is on {workspace.device}, but the current CUDA device is "
+                         f"cuda:{torch.cuda.current_device()}")
+    elif not workspace.is_contiguous():
+        raise ValueError("workspace must be contiguous")
+    return workspace, workspace.numel() * workspace.element_size()
 
 
 # ---------------------------------------------------------------- host-only helpers
@@ -201,12 +220,11 @@ def _prefill(fn, q, k, v, w_pretrained, w0, method, out, lse, out_dtype, want_ls
             raise ValueError("k_cache_out must be [B, Lcap, Hkv, D]")
         cap = k_cache_out.shape[1]
         _require(k_cache_out, "k_cache_out", (B, cap, Hkv, D), torch.bfloat16)
-    need = jetlong_prefill_workspace_size(B, Hq, Hkv, L, D)
-    if workspace is None:
-        workspace = _ws(need, q.device)
+    workspace, ws_bytes = _workspace(
+        workspace, jetlong_prefill_workspace_size(B, Hq, Hkv, L, D), q.device)
     st = getattr(lib(), fn)(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, L, D,
                             int(w_pretrained), int(w0), *method, od, _ptr(k_cache_out), cap,
-                            _ptr(workspace), workspace.numel(), _stream_ptr(stream))
+                            _ptr(workspace), ws_bytes, _stream_ptr(stream))
     _check(fn, st)
     return out, lse
 
@@ -222,9 +240,10 @@ def jetlong_prefill_rotate(q, k, v, w_pretrained: int, rope_theta: float, worksp
     cap = 0 if k_cache_out is None else k_cache_out.shape[1]
     if k_cache_out is not None:
         _require(k_cache_out, "k_cache_out", (B, cap, Hkv, D), torch.bfloat16)
+    workspace, ws_bytes = _workspace(workspace, 0, q.device)
     st = lib().jetlong_prefill_rotate(_ptr(q), _ptr(k), _ptr(v), B, Hq, Hkv, L, D,
                                       int(w_pretrained), float(rope_theta), _ptr(k_cache_out), cap,
-                                      _ptr(workspace), workspace.numel(), _stream_ptr(stream))
+                                      _ptr(workspace), ws_bytes, _stream_ptr(stream))
     _check("jetlong_prefill_rotate", st)
 
 
@@ -237,9 +256,10 @@ def jetlong_prefill_attend(out, lse, Hkv: int, w_pretrained: int, w0: int, works
     _require(out, "out", (B, L, Hq, D), out.dtype)
     if lse is not None:
         _require(lse, "lse", (B, Hq, L), torch.float32)
+    workspace, ws_bytes = _workspace(workspace, 0, out.device)
     st = lib().jetlong_prefill_attend(_ptr(out), _ptr(lse), B, Hq, int(Hkv), L, D,
                                       int(w_pretrained), int(w0), _out_dtype(out.dtype),
-                                      _ptr(workspace), workspace.numel(), _stream_ptr(stream))
+                                      _ptr(workspace), ws_bytes, _stream_ptr(stream))
     _check("jetlong_prefill_attend", st)
 
 
@@ -264,12 +284,12 @@ def jetlong_prefill_three_pass(q, k, v, w_pretrained: int, w0: int, rope_theta: 
         lse = torch.empty((B, Hq, L), dtype=torch.float32, device=q.device)
     if lse is not None:
         _require(lse, "lse", (B, Hq, L), torch.float32)
-    if workspace is None:
-        workspace = _ws(jetlong_prefill_three_pass_workspace_size(B, Hq, Hkv, L, D), q.device)
+    workspace, ws_bytes = _workspace(
+        workspace, jetlong_prefill_three_pass_workspace_size(B, Hq, Hkv, L, D), q.device)
     st = lib().jetlong_prefill_three_pass(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq,
                                           Hkv, L, D, int(w_pretrained), int(w0),
-                                          float(rope_theta), od, _ptr(workspace),
-                                          workspace.numel(), _stream_ptr(stream))
+                                          float(rope_theta), od, _ptr(workspace), ws_bytes,
+                                          _stream_ptr(stream))
     _check("jetlong_prefill_three_pass", st)
     return out, lse
 
@@ -310,11 +330,11 @@ def _decode(fn, q, k_cache, v_cache, L, w_pretrained, w0, method, out, lse, out_
         lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
     if lse is not None:
         _require(lse, "lse", (B, Hq), torch.float32)
-    if workspace is None:
-        workspace = _ws(jetlong_decode_workspace_size(B, Hq, Hkv, int(L), D), q.device)
+    workspace, ws_bytes = _workspace(
+        workspace, jetlong_decode_workspace_size(B, Hq, Hkv, int(L), D), q.device)
     st = getattr(lib(), fn)(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(out), _ptr(lse), B, Hq,
                             Hkv, int(L), Lcap, D, int(w_pretrained), int(w0), *method, od,
-                            _ptr(workspace), workspace.numel(), _stream_ptr(stream))
+                            _ptr(workspace), ws_bytes, _stream_ptr(stream))
     _check(fn, st)
     return out, lse
 
@@ -361,12 +381,11 @@ def _chunk(fn, q, k_cache, v_cache, P0, w_pretrained, w0, method, out, lse, out_
         lse = torch.empty((B, Hq, n), dtype=torch.float32, device=q.device)
     if lse is not None:
         _require(lse, "lse", (B, Hq, n), torch.float32)
-    if workspace is None:
-        workspace = _ws(jetlong_prefill_chunk_workspace_size(B, Hq, Hkv, int(P0), n, D),
-                        q.device)
+    workspace, ws_bytes = _workspace(
+        workspace, jetlong_prefill_chunk_workspace_size(B, Hq, Hkv, int(P0), n, D), q.device)
     st = getattr(lib(), fn)(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(out), _ptr(lse), B, Hq,
                             Hkv, int(P0), n, Lcap, D, int(w_pretrained), int(w0), *method, od,
-                            _ptr(workspace), workspace.numel(), _stream_ptr(stream))
+                            _ptr(workspace), ws_bytes, _stream_ptr(stream))
     _check(fn, st)
     return out, lse
 
