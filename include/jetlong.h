@@ -16,6 +16,8 @@
  *   - KV cache (§3.2): keys are stored once, rotated to their true positions,
  *     k_cache[k] = RoPE(x_k, k); decode applies the correction rotation by
  *     Delta k = f(k) - k on the fly and never rewrites the cache.
+ *   - The *_interp entry points replace the remote map by the frequency
+ *     interpolation of the paper's remote-map ablation (§4.7); see below.
  *
  * RoPE pairs channel i with channel i + D/2 and rotates the pair by the angle
  * p * theta^(-2i/D); angles are formed in double precision and reduced before
@@ -29,9 +31,11 @@
  *   - GQA: query head h reads KV head h / (Hq / Hkv).
  *   - Supported head dims: D = 64 or 128.  Hq must be a multiple of Hkv.
  *   - Device pointers must be 16-byte aligned.
- *   - Ownership: the caller owns every buffer; the library keeps no buffer and
- *     performs no device allocation.  Scratch space is passed in as a
- *     caller-owned workspace whose size the *_workspace_size functions return.
+ *   - Ownership: the caller owns every buffer, and the library performs no
+ *     device allocation.  Its only device storage is static in its image:
+ *     the error word and the 8 MiB buffer of jetlong_decode_noalloc.
+ *     Scratch space is passed in as a caller-owned workspace whose size the
+ *     *_workspace_size functions return.
  *   - Execution: asynchronous on `stream` (NULL = the legacy default stream) on
  *     the current CUDA device.  Arguments are validated on the host before
  *     anything is launched; a call that returns an error launched nothing.
