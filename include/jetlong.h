@@ -47,8 +47,15 @@
  *     Q/K, V, and the probabilities P) are FP16, which holds the rotated
  *     values with three more mantissa bits than BF16; accumulation, softmax
  *     statistics and LSE are FP32.  Inputs must stay inside the FP16 range
- *     (|x| <= 65504 after rotation); a prefill that meets a larger value
- *     records JL_ERR_RANGE for jetlong_device_status().
+ *     (|x| <= 65504 after rotation).  The range is a contract on the
+ *     inputs, not a status of the call: a call returns before its kernels
+ *     run, so a call that meets a larger value still returns JL_OK, and its
+ *     outputs may hold non-finite values.  A prefill (every form) records
+ *     the event, and the next jetlong_device_status() returns JL_ERR_RANGE;
+ *     read it before trusting outputs of inputs that may be that large.
+ *     The decode and chunk calls (whose queries and corrected keys pass
+ *     through FP16 too) record nothing: out-of-range values there show up
+ *     only as non-finite outputs.
  *   - Calls on different streams may run concurrently as long as they do not
  *     share output or workspace buffers.
  */

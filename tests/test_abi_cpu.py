@@ -299,3 +299,51 @@ def test_binding_refuses_host_memory_as_workspace_or_operand():
         jl._workspace(bytearray(64), 64, None)
     with pytest.raises(ValueError, match="must be a CUDA tensor"):
         jl._require(torch.empty((1, 2), dtype=torch.bfloat16), "q", (1, 2), torch.bfloat16)
+
+
+def noalloc_call(lib, **kw):
+    a = dict(q=P, kc=P, vc=P, out=P, lse=None, B=1, Hq=32, Hkv=8, L=1000, Lcap=1000, D=128,
+             wp=32768, w0=4096, theta=1e6, od=0, stream=None)
+    a.update(kw)
+    return lib.jetlong_decode_noalloc(a["q"], a["kc"], a["vc"], a["out"], a["lse"], a["B"],
+                                      a["Hq"], a["Hkv"], a["L"], a["Lcap"], a["D"], a["wp"],
+                                      a["w0"], a["theta"], a["od"], a["stream"])
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(q=None), jl.JL_ERR_NULL),
+    (dict(out=None), jl.JL_ERR_NULL),
+    (dict(L=0), jl.JL_ERR_SHAPE),
+    (dict(Lcap=999), jl.JL_ERR_SHAPE),                 # L > Lcap
+    (dict(Hq=48, Hkv=8), jl.JL_ERR_UNSUPPORTED),       # group of 6 query heads
+    (dict(D=80), jl.JL_ERR_UNSUPPORTED),
+    (dict(w0=-1), jl.JL_ERR_SHAPE),
+    (dict(theta=float("nan")), jl.JL_ERR_SHAPE),
+    (dict(od=3), jl.JL_ERR_UNSUPPORTED),
+    (dict(kc=ctypes.c_void_p(264)), jl.JL_ERR_ALIGN),
+    (dict(lse=ctypes.c_void_p(260)), jl.JL_ERR_ALIGN),
+    (dict(B=512, L=16, Lcap=16), jl.JL_ERR_WORKSPACE),  # partials beyond its fixed buffer
+])
+def test_noalloc_decode_rejects_bad_arguments_without_a_device(lib, kw, status):
+    # the same host checks as jetlong_decode, all before any CUDA call
+    assert noalloc_call(lib, **kw) == status
+
+
+def test_binding_refuses_an_out_that_is_not_a_tensor():
+    import torch
+    with pytest.raises(TypeError, match="out must be a torch.Tensor"):
+        jl._out_code([0.0], torch.float32)
+    with pytest.raises(ValueError, match="out dtype"):
+        jl._out_code(torch.empty(1, dtype=torch.float16), None)
+    assert jl._out_code(None, torch.float32) == jl.JL_F32
+
+
+def test_header_states_the_fp16_range_contract():
+    # a call that meets an input beyond FP16 still returns JL_OK; the report
+    # comes from jetlong_device_status (prefill) or non-finite outputs (decode)
+    text = " ".join(ln.strip().lstrip("*").strip() for ln in open(HEADER).read().splitlines())
+    text = " ".join(text.split())
+    assert "|x| <= 65504 after rotation" in text
+    assert "still returns JL_OK, and its outputs may hold non-finite values" in text
+    assert "the next jetlong_device_status() returns JL_ERR_RANGE" in text
+    assert "record nothing" in text

@@ -154,3 +154,28 @@ def test_decode_calls_replay_from_a_cuda_graph():
     assert jl.jetlong_device_status() == jl.JL_OK
     for (eo, el), o, l in zip(eager, outs, lses):
         assert torch.equal(eo, o) and torch.equal(el, l)
+
+
+@pytest.mark.parametrize("D,grp,wp,w0,L,jstar", [
+    (64, 2, 64, 64, 40, 10),    # G = 1, the jump in the second 8-token block of a stage
+    (64, 4, 16, 35, 40, 26),    # G = 3, the key that jumps is local
+    (64, 1, 8, 3, 48, 42),      # G = 6, the key that jumps is remote
+    (128, 4, 16, 35, 40, 26),   # 8-token stages: one block per stage
+])
+def test_running_max_jumps_inside_a_stage(D, grp, wp, w0, L, jstar):
+    # One cached key is aligned with the first query head's rotated query, so
+    # its score stands about 16 nats above the rest and the running max jumps
+    # by far more than the lazy-rescale threshold in the middle of a stage.
+    # Every block of the stage must then be weighed against the new max.
+    w = Workload("jump", 1, grp, 1, D, L, wp, w0, 1e4, 81 + jstar, False, kind="decode")
+    d = decode_inputs(w, Lcap=L)
+    cache = oracle.rope_cache(f64(d.k_raw), 0, w.theta)
+    p = L - 1
+    G = oracle.group_size(L, wp)
+    target = p if p - jstar <= w0 else p // G - jstar // G + jstar
+    cache[0, jstar, 0] = 2.0 * oracle.rope(f64(d.q)[0, 0], np.int64(target), w.theta)
+    cache = torch.from_numpy(cache).to(torch.bfloat16)
+    out, lse, o_ref, lse_ref = decode_both(w, L, d.q, cache, d.v)
+    assert lse_ref[0, 0] > 10.0  # the planted key dominates head 0
+    assert_o(f64(out), o_ref, f"jump at {jstar}")
+    assert_lse(f64(lse), lse_ref, f"jump at {jstar}")

@@ -181,10 +181,7 @@ def test_decode_random_shapes(w, ramp):
     assert_lse(f64(lse), lse_ref, f"{w} {ramp}")
 
 
-@RANDOM
-@given(workloads(grps=[1, 2, 4, 8], max_L=1500), RAMPS, st.data())
-def test_prefill_chunk_random_shapes(w, ramp, data):
-    n = data.draw(st.integers(1, min(w.L, 40)))
+def chunk_case(w, ramp, n):
     P0 = w.L - n
     x = prefill_inputs(w)
     cache = cache_bf16(x.k, w.theta)
@@ -197,3 +194,22 @@ def test_prefill_chunk_random_shapes(w, ramp, data):
                                                  w.w_pretrained, w.w0, w.theta, *ramp)
     assert_o(f64(out), o_ref, f"{w} {ramp}")
     assert_lse(f64(lse), lse_ref, f"{w} {ramp}")
+
+
+@RANDOM
+@given(workloads(grps=[1, 2, 4, 8], max_L=1500), RAMPS, st.data())
+def test_prefill_chunk_random_shapes(w, ramp, data):
+    chunk_case(w, ramp, data.draw(st.integers(1, min(w.L, 40))))
+
+
+# The random draw that exposed a lost rescale in the D = 64 decode kernel: a
+# running max that jumps inside a 16-token stage must reweigh the stage's
+# first 8-token block too.  Pinned, with its neighbours, so that a change of
+# the random strategy cannot drop it.
+PINNED_D64 = Workload("rand", 1, 4, 1, 64, 1484, 1, 0, 1e4, 0, True)
+
+
+@pytest.mark.parametrize("wp", [1, 2, 8, 64])
+@pytest.mark.parametrize("n", [1, 7])
+def test_prefill_chunk_pinned_d64(wp, n):
+    chunk_case(PINNED_D64.with_(w_pretrained=wp), (1.0, 32.0), n)

@@ -11,9 +11,10 @@ import ctypes
 import pytest
 import torch
 
+import oracle
 from parity_util import assert_lse, assert_o, f64
 from zero_shot_rope_bifocal_b200 import jetlong as jl
-from zero_shot_rope_bifocal_b200.synth import Workload, decode_inputs
+from zero_shot_rope_bifocal_b200.synth import WORKLOADS, Workload, decode_inputs
 
 pytestmark = pytest.mark.gpu
 
@@ -42,6 +43,23 @@ def test_noalloc_decode_matches_decode_on_two_calls_in_a_row():
         assert jl.jetlong_device_status() == jl.JL_OK
         assert_o(f64(out), f64(ref_o), f"noalloc L={L}")
         assert_lse(f64(lse), f64(ref_l), f"noalloc L={L}")
+
+
+def test_noalloc_decode_matches_the_oracle_on_the_tiny_case():
+    # the tiny workload (G = 4 at L = 512) against the fp64 oracle directly
+    w = WORKLOADS["tiny"].with_(kind="decode")
+    d = decode_inputs(w)
+    kc = torch.from_numpy(oracle.rope_cache(f64(d.k_raw), 0, w.theta)).to(torch.bfloat16)
+    q, kc, v = d.q.cuda(), kc.cuda(), d.v.cuda()
+    for L in (w.L, w.L - 200):
+        out = torch.full((w.B, w.Hq, w.D), float("nan"), device="cuda")
+        lse = torch.full((w.B, w.Hq), float("nan"), device="cuda")
+        assert _call_noalloc(w, L, q, kc, v, out, lse) == jl.JL_OK
+        assert jl.jetlong_device_status() == jl.JL_OK
+        o_ref, l_ref = oracle.decode(f64(d.q), f64(kc), f64(d.v), L, w.w_pretrained, w.w0,
+                                     w.theta)
+        assert_o(f64(out), o_ref, f"noalloc tiny L={L}")
+        assert_lse(f64(lse), l_ref, f"noalloc tiny L={L}")
 
 
 def test_noalloc_rejects_sizes_beyond_its_buffer():

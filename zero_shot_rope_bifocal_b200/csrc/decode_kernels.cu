@@ -415,7 +415,10 @@ decode_split_kernel(DecodeArgs a) {
       const uint32_t kst = sb + slot * C::STAGE + warp_col;
       const uint32_t vst = kst + C::HALF_STAGE;
       const uint8_t *tab = dsm + C::CS + slot * C::CS_TAB;
-      uint32_t pfrag[NBLK];  // P^T fragments (BF16), one per 8-token block
+      // Scores of head gq for tokens tb + 2tq, tb + 2tq + 1 of each 8-token
+      // block; every block of the stage is scored before the running max
+      // moves, since one P.V product covers all of them.
+      float sv[NBLK][2];
 #pragma unroll
       for (int nb = 0; nb < NBLK; ++nb) {
         const int tb = nb * 8;
@@ -439,34 +442,39 @@ decode_split_kernel(DecodeArgs a) {
           if (p - (jb + 2 * tq) <= w0eff) sc[0] = sl[0];
           if (p - (jb + 2 * tq + 1) <= w0eff) sc[1] = sl[1];
         }
-        // scores of head gq for tokens tb + 2tq, tb + 2tq + 1
-        const float s0 = 2 * tq < nb_valid ? sc[0] : -INFINITY;
-        const float s1 = 2 * tq + 1 < nb_valid ? sc[1] : -INFINITY;
-        float bm = fmaxf(s0, s1);
-        bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 1));
-        bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 2));
-        // lazy online softmax: the reference max moves only when it grows by
-        // more than 2^8 (O and l share it, so the result is exact)
-        float alpha = 1.f;
-        if (bm > m_run + kRescaleThreshold || (m_run == -INFINITY && bm > -INFINITY)) {
-          if (m_run != -INFINITY) alpha = exp2f(m_run - bm);
-          m_run = bm;
-        }
-        if (__any_sync(0xffffffffu, alpha != 1.f)) {
-          // O^T columns are heads 2tq, 2tq+1; their factors live in lanes 4*head
-          const float a0 = __shfl_sync(0xffffffffu, alpha, (2 * tq) * 4);
-          const float a1 = __shfl_sync(0xffffffffu, alpha, (2 * tq + 1) * 4);
+        sv[nb][0] = 2 * tq < nb_valid ? sc[0] : -INFINITY;
+        sv[nb][1] = 2 * tq + 1 < nb_valid ? sc[1] : -INFINITY;
+      }
+      float bm = fmaxf(sv[0][0], sv[0][1]);
 #pragma unroll
-          for (int mb = 0; mb < MB; ++mb) {
-            o[mb][0] *= a0;
-            o[mb][1] *= a1;
-            o[mb][2] *= a0;
-            o[mb][3] *= a1;
-          }
-          l_part *= alpha;
+      for (int nb = 1; nb < NBLK; ++nb) bm = fmaxf(bm, fmaxf(sv[nb][0], sv[nb][1]));
+      bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 1));
+      bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 2));
+      // lazy online softmax: the reference max moves only when it grows by
+      // more than 2^8 (O and l share it, so the result is exact)
+      float alpha = 1.f;
+      if (bm > m_run + kRescaleThreshold || (m_run == -INFINITY && bm > -INFINITY)) {
+        if (m_run != -INFINITY) alpha = exp2f(m_run - bm);
+        m_run = bm;
+      }
+      if (__any_sync(0xffffffffu, alpha != 1.f)) {
+        // O^T columns are heads 2tq, 2tq+1; their factors live in lanes 4*head
+        const float a0 = __shfl_sync(0xffffffffu, alpha, (2 * tq) * 4);
+        const float a1 = __shfl_sync(0xffffffffu, alpha, (2 * tq + 1) * 4);
+#pragma unroll
+        for (int mb = 0; mb < MB; ++mb) {
+          o[mb][0] *= a0;
+          o[mb][1] *= a1;
+          o[mb][2] *= a0;
+          o[mb][3] *= a1;
         }
-        const float neg_m = m_run == -INFINITY ? 0.f : -m_run;
-        const float p0 = ex2_sfu(s0 + neg_m), p1 = ex2_sfu(s1 + neg_m);
+        l_part *= alpha;
+      }
+      const float neg_m = m_run == -INFINITY ? 0.f : -m_run;
+      uint32_t pfrag[NBLK];  // P^T fragments (BF16), one per 8-token block
+#pragma unroll
+      for (int nb = 0; nb < NBLK; ++nb) {
+        const float p0 = ex2_sfu(sv[nb][0] + neg_m), p1 = ex2_sfu(sv[nb][1] + neg_m);
         l_part += p0 + p1;
         pfrag[nb] = pack_bf16(p0, p1);
       }

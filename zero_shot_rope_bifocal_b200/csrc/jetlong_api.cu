@@ -344,11 +344,12 @@ namespace {
 // Queries at positions q_pos0 .. q_pos0 + nq - 1 (per batch entry) against the
 // true-position cache, each over keys [0, its position], with one G from the
 // longest range L = q_pos0 + nq: a decode step (nq = 1) or a prefill chunk.
-int cache_attention(const void *q, const void *k_cache, const void *v_cache, void *out, float *lse,
-                    int B, int Hq, int Hkv, int nq, int q_pos0, int Lcap, int D, int w_pretrained,
-                    int w0, float rope_theta, int out_dtype, void *workspace,
-                    size_t workspace_bytes, jl_stream_t stream, int interp = 0,
-                    float ramp_alpha = 0.f, float ramp_beta = 0.f) {
+// Every host check of such a call except the workspace's; sets *L_out to the
+// key range q_pos0 + nq.  Makes no CUDA call.
+int check_cache_call(const void *q, const void *k_cache, const void *v_cache, const void *out,
+                     const float *lse, int B, int Hq, int Hkv, int nq, int q_pos0, int Lcap, int D,
+                     int w_pretrained, int w0, float rope_theta, int out_dtype, int interp,
+                     float ramp_alpha, float ramp_beta, int *L_out) {
   if (!q || !k_cache || !v_cache || !out) return JL_ERR_NULL;
   if (interp && check_ramp(ramp_alpha, ramp_beta) != JL_OK) return JL_ERR_SHAPE;
   if (nq < 1 || q_pos0 < 0) return JL_ERR_SHAPE;
@@ -367,6 +368,20 @@ int cache_attention(const void *q, const void *k_cache, const void *v_cache, voi
   if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(out) ||
       (lse && !aligned16(lse)))
     return JL_ERR_ALIGN;
+  *L_out = L;
+  return JL_OK;
+}
+
+int cache_attention(const void *q, const void *k_cache, const void *v_cache, void *out, float *lse,
+                    int B, int Hq, int Hkv, int nq, int q_pos0, int Lcap, int D, int w_pretrained,
+                    int w0, float rope_theta, int out_dtype, void *workspace,
+                    size_t workspace_bytes, jl_stream_t stream, int interp = 0,
+                    float ramp_alpha = 0.f, float ramp_beta = 0.f) {
+  int L = 0;
+  int st = check_cache_call(q, k_cache, v_cache, out, lse, B, Hq, Hkv, nq, q_pos0, Lcap, D,
+                            w_pretrained, w0, rope_theta, out_dtype, interp, ramp_alpha,
+                            ramp_beta, &L);
+  if (st != JL_OK) return st;
   const size_t need = decode_ws_bytes(B * nq, Hq, Hkv, L, D);
   if (!workspace || workspace_bytes < need) return JL_ERR_WORKSPACE;
   if (reinterpret_cast<uintptr_t>(workspace) % kAlign) return JL_ERR_ALIGN;
@@ -550,11 +565,19 @@ extern "C" int jetlong_decode_noalloc(const void *q, const void *k_cache, const 
                                       void *out, float *lse, int B, int Hq, int Hkv, int L,
                                       int Lcap, int D, int w_pretrained, int w0, float rope_theta,
                                       int out_dtype, jl_stream_t stream) {
-  if (check_common(B, Hq, Hkv, L, D) != JL_OK) return check_common(B, Hq, Hkv, L, D);
-  if (decode_ws_bytes(B, Hq, Hkv, L, D) > kNoAllocScratchBytes) return JL_ERR_WORKSPACE;
-  void *scratch = nullptr;
-  const int st = noalloc_scratch(&scratch);
+  // Every argument check first, as for jetlong_decode: an invalid call
+  // returns its status with no CUDA call.
+  if (L < 1) return JL_ERR_SHAPE;
+  int L_checked = 0;
+  int st = check_cache_call(q, k_cache, v_cache, out, lse, B, Hq, Hkv, 1, L - 1, Lcap, D,
+                            w_pretrained, w0, rope_theta, out_dtype, 0, 0.f, 0.f, &L_checked);
   if (st != JL_OK) return st;
+  if (decode_ws_bytes(B, Hq, Hkv, L, D) > kNoAllocScratchBytes) return JL_ERR_WORKSPACE;
+  // Then the device (an sm_100 one), and only then the buffer's address.
+  DeviceState *dev = nullptr;
+  if ((st = current_device(&dev)) != JL_OK) return st;
+  void *scratch = nullptr;
+  if ((st = noalloc_scratch(&scratch)) != JL_OK) return st;
   return jetlong_decode(q, k_cache, v_cache, out, lse, B, Hq, Hkv, L, Lcap, D, w_pretrained, w0,
                         rope_theta, out_dtype, scratch, kNoAllocScratchBytes, stream);
 }

@@ -136,6 +136,15 @@ def _out_dtype(dtype) -> int:
     raise ValueError("out dtype must be torch.bfloat16 or torch.float32")
 
 
+def _out_code(out, out_dtype) -> int:
+    """The jl_dtype of a caller's ``out`` tensor, or of ``out_dtype`` if none."""
+    if out is None:
+        return _out_dtype(out_dtype)
+    if not isinstance(out, torch.Tensor):
+        raise TypeError("out must be a torch.Tensor")
+    return _out_dtype(out.dtype)
+
+
 def _ws(nbytes: int, device) -> torch.Tensor:
     # torch's caching allocator returns blocks aligned to at least 512 bytes.
     return torch.empty(max(int(nbytes), 1), dtype=torch.uint8, device=device)
@@ -205,7 +214,7 @@ def _prefill(fn, q, k, v, w_pretrained, w0, method, out, lse, out_dtype, want_ls
     _require(q, "q", (B, L, Hq, D), torch.bfloat16)
     _require(k, "k", (B, L, Hkv, D), torch.bfloat16)
     _require(v, "v", (B, L, Hkv, D), torch.bfloat16)
-    od = _out_dtype(out_dtype if out is None else out.dtype)
+    od = _out_code(out, out_dtype)
     if out is None:
         out = torch.empty((B, L, Hq, D), dtype=torch.bfloat16 if od == JL_BF16 else torch.float32,
                           device=q.device)
@@ -250,6 +259,7 @@ def jetlong_prefill_rotate(q, k, v, w_pretrained: int, rope_theta: float, worksp
 def jetlong_prefill_attend(out, lse, Hkv: int, w_pretrained: int, w0: int, workspace, *,
                            stream=None):
     """Stage 2 of jetlong_prefill: the attention kernel on the operands in ``workspace``."""
+    od = _out_code(out, None)
     if out.dim() != 4:
         raise ValueError("out must be [B, L, Hq, D]")
     B, L, Hq, D = out.shape
@@ -258,8 +268,8 @@ def jetlong_prefill_attend(out, lse, Hkv: int, w_pretrained: int, w0: int, works
         _require(lse, "lse", (B, Hq, L), torch.float32)
     workspace, ws_bytes = _workspace(workspace, 0, out.device)
     st = lib().jetlong_prefill_attend(_ptr(out), _ptr(lse), B, Hq, int(Hkv), L, D,
-                                      int(w_pretrained), int(w0), _out_dtype(out.dtype),
-                                      _ptr(workspace), ws_bytes, _stream_ptr(stream))
+                                      int(w_pretrained), int(w0), od, _ptr(workspace), ws_bytes,
+                                      _stream_ptr(stream))
     _check("jetlong_prefill_attend", st)
 
 
@@ -275,7 +285,7 @@ def jetlong_prefill_three_pass(q, k, v, w_pretrained: int, w0: int, rope_theta: 
     _require(q, "q", (B, L, Hq, D), torch.bfloat16)
     _require(k, "k", (B, L, Hkv, D), torch.bfloat16)
     _require(v, "v", (B, L, Hkv, D), torch.bfloat16)
-    od = _out_dtype(out_dtype if out is None else out.dtype)
+    od = _out_code(out, out_dtype)
     if out is None:
         out = torch.empty((B, L, Hq, D), dtype=torch.bfloat16 if od == JL_BF16 else torch.float32,
                           device=q.device)
@@ -321,7 +331,7 @@ def _decode(fn, q, k_cache, v_cache, L, w_pretrained, w0, method, out, lse, out_
     _require(q, "q", (B, Hq, D), torch.bfloat16)
     _require(k_cache, "k_cache", (B, Lcap, Hkv, D), torch.bfloat16)
     _require(v_cache, "v_cache", (B, Lcap, Hkv, D), torch.bfloat16)
-    od = _out_dtype(out_dtype if out is None else out.dtype)
+    od = _out_code(out, out_dtype)
     if out is None:
         out = torch.empty((B, Hq, D), dtype=torch.bfloat16 if od == JL_BF16 else torch.float32,
                           device=q.device)
@@ -372,7 +382,7 @@ def _chunk(fn, q, k_cache, v_cache, P0, w_pretrained, w0, method, out, lse, out_
     _require(q, "q", (B, n, Hq, D), torch.bfloat16)
     _require(k_cache, "k_cache", (B, Lcap, Hkv, D), torch.bfloat16)
     _require(v_cache, "v_cache", (B, Lcap, Hkv, D), torch.bfloat16)
-    od = _out_dtype(out_dtype if out is None else out.dtype)
+    od = _out_code(out, out_dtype)
     if out is None:
         out = torch.empty((B, n, Hq, D), dtype=torch.bfloat16 if od == JL_BF16 else torch.float32,
                           device=q.device)
@@ -400,13 +410,13 @@ def jetlong_decode_noalloc(q, k_cache, v_cache, L: int, w_pretrained: int, w0: i
     _require(q, "q", (B, Hq, D), torch.bfloat16)
     _require(k_cache, "k_cache", (B, Lcap, Hkv, D), torch.bfloat16)
     _require(v_cache, "v_cache", (B, Lcap, Hkv, D), torch.bfloat16)
+    od = _out_code(out, None)
     _require(out, "out", (B, Hq, D), out.dtype)
     if lse is not None:
         _require(lse, "lse", (B, Hq), torch.float32)
     st = lib().jetlong_decode_noalloc(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(out), _ptr(lse),
                                       B, Hq, Hkv, int(L), Lcap, D, int(w_pretrained), int(w0),
-                                      float(rope_theta), _out_dtype(out.dtype),
-                                      _stream_ptr(stream))
+                                      float(rope_theta), od, _stream_ptr(stream))
     _check("jetlong_decode_noalloc", st)
     return out, lse
 
