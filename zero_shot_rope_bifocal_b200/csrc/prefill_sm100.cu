@@ -26,24 +26,21 @@
 //
 // CTA = two 128-row query tiles of the same 128 positions, for two query
 // heads of one KV group (GQA packing: each K/V tile staged in shared memory
-// serves 256 query rows).  Warp-specialised, 20 warps:
-//   * warps 0-3 / 4-7: softmax for query tile 0 / 1, score columns [0, 64);
-//     warps 8-11 / 12-15: the same rows, columns [64, 128).  Two threads (one
-//     per column half) own each row of a tile (a TMEM lane); they trade their
-//     half-row maxima through shared memory and one mbarrier per warp pair,
-//     rescale their halves of the O row when needed and run the epilogue;
-//   * warp 16: TMA producer (queries once per variant, K and V tiles through
+// serves 256 query rows).  Warp-specialised, 10 warps:
+//   * warps 0-3 / 4-7: softmax for query tile 0 / 1, one thread per row (a
+//     TMEM lane).  A thread holds its row's 128 scores in registers: one TMEM
+//     read, the row max, the exponentials, P stored back, with no exchange
+//     between threads; it rescales its O row when the max grows and runs the
+//     epilogue of its row;
+//   * warp 8: TMA producer (queries once per variant, K and V tiles through
 //     a four-slot ring);
-//   * warp 17: tcgen05.mma issuer, in the order
+//   * warp 9: tcgen05.mma issuer, in the order
 //       S0(j+1) = Q0 K(j+1)^T after O0 += P0(j) V(j), and likewise for tile 1,
 //     so the tensor core works on one tile while the other tile's softmax
-//     runs;
-//   * warps 18-19 hold no role.
-// Two threads per row keep 32 scores live at a time, so the softmax fits the
-// 96 registers per thread that 20 warps leave, without spills.
-// TMEM (512 columns): S0 | S1 | O0 | O1; each half of a row writes its P
-// (packed FP16) over the first 32 columns of its own 64-column half of S
-// once those scores are in registers.
+//     runs.
+// Ten warps leave up to 200 registers per thread, which holds a whole row.
+// TMEM (512 columns): S0 | S1 | O0 | O1; a row's P (packed FP16) is written
+// over the first 64 columns of its S once the scores are in registers.
 // Each wait is bounded in time (jl::kWaitLimitNs) and also gives up when
 // another role has given up; the CTA then records a device error, drains its
 // MMAs and in-flight copies, frees TMEM and exits.
@@ -58,18 +55,17 @@ namespace {
 constexpr int BM = 128;  // query rows per tile (= TMEM lanes)
 constexpr int BN = 128;  // keys per tile
 constexpr int NS = 4;    // K/V ring slots (one K or V tile each)
-constexpr int kSoftmaxWarps = 16;  // 4 warpgroups: (tile, column half)
-constexpr int kWarps = 20;
+constexpr int kSoftmaxWarps = 8;  // 2 warpgroups: one per query tile
+constexpr int kWarps = 10;
 constexpr int kThreads = kWarps * 32;
-constexpr int kProducerWarp = 16;
-constexpr int kMmaWarp = 17;
-constexpr int HBN = BN / 2;  // score columns per softmax thread
-// Registers: 20 warps put 5 on each of the 4 SM sub-partitions, whose
-// register files hold 16,384 each, so every thread gets 96 and the softmax
-// is written to fit (32 scores live at a time).  No setmaxnreg: an increase
-// can only be served from what other warps release with a decrease, and the
-// four non-softmax warps could not release enough to lift the 16 softmax
-// warps to a useful size.
+constexpr int kProducerWarp = 8;
+constexpr int kMmaWarp = 9;
+// Column pairs per 8 whose exponential runs on the FMA pipe (the rest on the
+// special-function unit, which would otherwise be the softmax's limit).
+#ifndef JL_PREFILL_FMA_PAIRS
+#define JL_PREFILL_FMA_PAIRS 2
+#endif
+constexpr int kFmaPairsPer8 = JL_PREFILL_FMA_PAIRS;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 constexpr uint32_t kF16 = 0;               // operand format code of kind::f16
 
@@ -83,12 +79,8 @@ struct Layout {
   // barrier indices (8 bytes each)
   static constexpr int kQFull = 0, kQEmpty = 2, kKvFull = 4, kKvEmpty = 4 + NS,
                        kSFull = 4 + 2 * NS, kPFull = 6 + 2 * NS, kOFull = 8 + 2 * NS,
-                       kDrain = 10 + 2 * NS, kPair = 11 + 2 * NS,  // 8 pair barriers
-                       kNumBars = 19 + 2 * NS;
-  // half-row maxima (and, at the end, half-row sums) traded by the two
-  // threads of a row: [parity][tile][half][row] floats
-  static constexpr int XCHG = BAR + 8 * kNumBars;
-  static constexpr int TMEM_SLOT = XCHG + 2 * 2 * 2 * BM * 4;
+                       kDrain = 10 + 2 * NS, kNumBars = 11 + 2 * NS;
+  static constexpr int TMEM_SLOT = BAR + 8 * kNumBars;
   static constexpr int ABORT = TMEM_SLOT + 4;
   static constexpr int SKIP = TMEM_SLOT + 8;
   static constexpr int BYTES = TMEM_SLOT + 16;
@@ -218,12 +210,10 @@ bifocal_prefill_kernel(const __grid_constant__ CUtensorMap tm_qt,
 
   if (tid == 0) {
     // P-ready barriers take one arrival from every softmax thread of the
-    // tile (two per row), pair barriers one from each thread of a warp pair;
-    // all others one arrival (plus transaction bytes for TMA).
+    // tile (one per row); all others one arrival (plus transaction bytes for
+    // TMA).
     for (int i = 0; i < LY::kNumBars; ++i)
-      mbar_init(bar(i), (i == LY::kPFull || i == LY::kPFull + 1) ? 2 * BM
-                        : (i >= LY::kPair && i < LY::kPair + 8)   ? 64
-                                                                  : 1);
+      mbar_init(bar(i), (i == LY::kPFull || i == LY::kPFull + 1) ? BM : 1);
     fence_mbar_init();
   }
   if (warp == kProducerWarp && lane == 0) {
@@ -311,8 +301,8 @@ bifocal_prefill_kernel(const __grid_constant__ CUtensorMap tm_qt,
       auto pv = [&](int s, uint32_t vslot, bool acc) {
         const uint64_t dv = smem_desc_sw128(sb + LY::RING + vslot * LY::TILE, LY::BOX, 1024);
 #pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk)  // P of keys [16kk, 16kk+16): half kk/4's columns
-          mma_f16kind_ts(tO(s), tS(s) + (kk >> 2) * HBN + (kk & 3) * 8,
+        for (int kk = 0; kk < BN / 16; ++kk)  // P of keys [16kk, 16kk+16): columns [8kk, 8kk+8)
+          mma_f16kind_ts(tO(s), tS(s) + kk * 8,
                          dv + static_cast<uint64_t>((kk * 16 * 128) >> 4), IDESC_PV,
                          (acc || kk > 0) ? 1u : 0u);
       };
@@ -391,24 +381,17 @@ bifocal_prefill_kernel(const __grid_constant__ CUtensorMap tm_qt,
     }
   } else {
     // ------------------------------------------------------------ softmax
-    const int s = (warp >> 2) & 1;       // query tile of this warpgroup
-    const int half = warp >> 3;          // score columns [half * 64, half * 64 + 64)
+    const int s = warp >> 2;             // query tile of this warpgroup
     const int wq = warp & 3;             // TMEM lane quarter
     const int rloc = tid & (BM - 1);     // row inside the tile
     const int row = p0 + rloc;
     const bool active = s == 0 || has1;
     const bool row_ok = active && row < prm.L;
     const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
-    const uint32_t pair_bar = bar(LY::kPair + s * 4 + wq);  // this warp and its other half
-    float *xchg = reinterpret_cast<float *>(smem + LY::XCHG);
-    // slot of (parity, tile, half, row) in the exchange buffer
-    auto xslot = [&](int par, int h) { return ((par * 2 + s) * 2 + h) * BM + rloc; };
-    const int c0 = half * HBN;           // first score column of this thread
-    float m_used = -INFINITY;  // reference max of this row (base 2), same in both halves
-    float l_sum = 0.f;         // this half's share of the row sum
+    float m_used = -INFINITY;  // reference max of this row (base 2)
+    float l_sum = 0.f;         // running row sum, relative to m_used
     bool ok = active;
-    int j = 0;
-    for (; j < nv && ok; ++j) {
+    for (int j = 0; j < nv && ok; ++j) {
       const bool remote = j < n_rem;
       const int kt = remote ? kr0 + j : kl0 + (j - n_rem);
       ok = wait_or_abort(bar(LY::kSFull + s), static_cast<uint32_t>(j) & 1u, abort);
@@ -417,56 +400,43 @@ bifocal_prefill_kernel(const __grid_constant__ CUtensorMap tm_qt,
         break;
       }
       tc_fence_after();
-      const int k0 = kt * BN + c0;  // key of this thread's first score column
+      const int k0 = kt * BN;  // key of column 0
       bool whole;
       if (remote)
-        whole = row_ok && (row - (k0 + HBN - 1) >= dlo) && (row - k0 <= dhi);
+        whole = row_ok && (row - (k0 + BN - 1) >= dlo) && (row - k0 <= dhi);
       else
-        whole = row_ok && (k0 + HBN - 1 <= row) && (row - k0 <= w0);
-      // This thread's scores, 32 columns at a time, with the mask applied
-      // (raw scores; the scale is positive and applied later).
-      auto load_chunk = [&](int cc, float (&x)[32]) {
-        uint32_t(&xr)[32] = reinterpret_cast<uint32_t(&)[32]>(x);
-        tmem_ld32(tS(s) + lane_base + c0 + cc * 32, xr);
+        whole = row_ok && (k0 + BN - 1 <= row) && (row - k0 <= w0);
+      // The row's raw scores (the scale is positive and applied later), one
+      // TMEM read of all 128 columns, then the mask on edge tiles only.
+      float x[BN];
+      {
+        uint32_t(&xr)[BN / 32][32] = reinterpret_cast<uint32_t(&)[BN / 32][32]>(x);
+#pragma unroll
+        for (int cc = 0; cc < BN / 32; ++cc) tmem_ld32(tS(s) + lane_base + cc * 32, xr[cc]);
         tmem_wait_ld();
-        reg_fence(xr);
-        if (!whole) {
 #pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            const int d = row - (k0 + cc * 32 + c);
-            const bool valid = row_ok && d >= 0 && (remote ? (d >= dlo && d <= dhi) : (d <= w0));
-            if (!valid) x[c] = -INFINITY;
-          }
-        }
-      };
-      // pass 1: the half-row max (a tree of three-input maxima per chunk),
-      // then the other half's through shared memory
-      float hmax = -INFINITY;
-#pragma unroll 1
-      for (int cc = 0; cc < HBN / 32; ++cc) {
-        float x[32];
-        load_chunk(cc, x);
-        float mx[4] = {x[0], x[1], x[2], x[3]};
+        for (int cc = 0; cc < BN / 32; ++cc) reg_fence(xr[cc]);
+      }
+      if (!whole) {
 #pragma unroll
-        for (int c = 4; c < 32; c += 8) {
-          mx[0] = fmax3(mx[0], x[c], x[c + 1]);
-          mx[1] = fmax3(mx[1], x[c + 2], x[c + 3]);
-          if (c + 4 < 32) {
-            mx[2] = fmax3(mx[2], x[c + 4], x[c + 5]);
-            mx[3] = fmax3(mx[3], x[c + 6], x[c + 7]);
-          }
+        for (int c = 0; c < BN; ++c) {
+          const int d = row - (k0 + c);
+          const bool valid = row_ok && d >= 0 && (remote ? (d >= dlo && d <= dhi) : (d <= w0));
+          if (!valid) x[c] = -INFINITY;
         }
-        hmax = fmax3(hmax, fmax3(mx[0], mx[1], mx[2]), mx[3]);
       }
-      xchg[xslot(j & 1, half)] = hmax;
-      mbar_arrive(pair_bar);
-      ok = wait_or_abort(pair_bar, static_cast<uint32_t>(j) & 1u, abort);
-      if (__any_sync(0xffffffffu, !ok)) {
-        ok = false;
-        break;
+      // row max: four chains of three-input maxima
+      float mx[4] = {x[0], x[1], x[2], x[3]};
+#pragma unroll
+      for (int c = 4; c < BN; c += 8) {
+        mx[0] = fmax3(mx[0], x[c], x[c + 1]);
+        mx[1] = fmax3(mx[1], x[c + 2], x[c + 3]);
+        if (c + 4 < BN) {
+          mx[2] = fmax3(mx[2], x[c + 4], x[c + 5]);
+          mx[3] = fmax3(mx[3], x[c + 6], x[c + 7]);
+        }
       }
-      const float tmax = fmaxf(hmax, xchg[xslot(j & 1, half ^ 1)]) * prm.scale_log2;
-      // both halves see the same tmax and m_used, so they take the same step
+      const float tmax = fmax3(fmax3(mx[0], mx[1], mx[2]), mx[3], mx[3]) * prm.scale_log2;
       const bool grow =
           tmax > m_used + kRescaleThreshold || (m_used == -INFINITY && tmax > -INFINITY);
       float alpha = 1.f;
@@ -475,82 +445,66 @@ bifocal_prefill_kernel(const __grid_constant__ CUtensorMap tm_qt,
         m_used = tmax;
       }
       l_sum *= alpha;
-      // pass 2: p = 2^(s * scale - m) per chunk, written back as packed FP16
-      // P over the first half of this thread's own columns (chunk cc lands on
-      // columns already read).  Masked entries are -inf and give 0 (or 2^-125
-      // on the FMA path, which rounds to 0 in FP16); a row with nothing valid
-      // yet has all entries -inf.  One column pair in eight takes the FMA-pipe
+      // p = 2^(s * scale - m), written back as packed FP16 P over the first
+      // 64 columns in one store (all scores are already in registers).
+      // Masked entries are -inf and give 0 (or 2^-125 on the FMA path, which
+      // rounds to 0 in FP16); a row with nothing valid yet has all entries
+      // -inf.  kFmaPairsPer8 column pairs in eight take the FMA-pipe
       // exponential, the rest the special-function unit.
       const float neg_m = m_used == -INFINITY ? 0.f : -m_used;
       const float2 sc2 = make_float2(prm.scale_log2, prm.scale_log2);
       const float2 nm2 = make_float2(neg_m, neg_m);
       float2 acc2[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-#pragma unroll 1
-      for (int cc = 0; cc < HBN / 32; ++cc) {
-        float x[32];
-        load_chunk(cc, x);
-        uint32_t pr[16];
+      uint32_t pr[BN / 2];
 #pragma unroll
-        for (int c = 0; c < 32; c += 2) {
-          float2 v = ffma2(make_float2(x[c], x[c + 1]), sc2, nm2);
-          if ((c & 15) == 0) {
-            v = exp2_fma2(v);
-          } else {
-            v.x = ex2_sfu(v.x);
-            v.y = ex2_sfu(v.y);
-          }
-          acc2[(c >> 1) & 1] = fadd2(acc2[(c >> 1) & 1], v);
-          const __half2 h2 = __floats2half2_rn(v.x, v.y);
-          pr[c >> 1] = *reinterpret_cast<const uint32_t *>(&h2);
+      for (int c = 0; c < BN; c += 2) {
+        float2 v = ffma2(make_float2(x[c], x[c + 1]), sc2, nm2);
+        if (((c >> 1) & 7) < kFmaPairsPer8) {
+          v = exp2_fma2(v);
+        } else {
+          v.x = ex2_sfu(v.x);
+          v.y = ex2_sfu(v.y);
         }
-        __syncwarp();
-        tmem_st16(tS(s) + lane_base + c0 + cc * 16, pr);
-        tmem_wait_st();
+        acc2[(c >> 1) & 1] = fadd2(acc2[(c >> 1) & 1], v);
+        const __half2 h2 = __floats2half2_rn(v.x, v.y);
+        pr[c >> 1] = *reinterpret_cast<const uint32_t *>(&h2);
       }
+      tmem_st64(tS(s) + lane_base, pr);
+      tmem_wait_st();
       const float2 a = fadd2(acc2[0], acc2[1]);
       l_sum += a.x + a.y;
       // O of this tile holds visits 0..j-1 (all complete: S(j) was issued
-      // after P(j-1) V(j-1)); rows whose max was -inf hold 0 there.  Each
-      // half rescales its half of the O row before PV(j) may start.
+      // after P(j-1) V(j-1)); rows whose max was -inf hold 0 there.  The row
+      // is rescaled before PV(j) may start.
       if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
-        __syncwarp();
 #pragma unroll 1
-        for (int c = 0; c < D / 64; ++c) {  // one 32-column chunk at a time (registers)
+        for (int c = 0; c < D / 32; ++c) {  // one 32-column chunk at a time
           uint32_t rr[32];
-          const uint32_t col = tO(s) + lane_base + half * (D / 2) + c * 32;
+          const uint32_t col = tO(s) + lane_base + c * 32;
           tmem_ld32(col, rr);
           tmem_wait_ld();
           reg_fence(rr);
 #pragma unroll
           for (int e = 0; e < 32; ++e) rr[e] = __float_as_uint(u2f(rr[e]) * alpha);
           tmem_st32(col, rr);
-          tmem_wait_st();
         }
+        tmem_wait_st();
       }
       tc_fence_before();
       mbar_arrive(bar(LY::kPFull + s));
     }
-    // ---- epilogue: the row sum is the two halves' sums
+    // ---- epilogue: O / l and the log-sum-exp of this row
     if (ok) ok = wait_or_abort(bar(LY::kOFull + s), 0u, abort);
-    if (__all_sync(0xffffffffu, ok) && active) {
-      xchg[xslot(j & 1, half)] = l_sum;
-      mbar_arrive(pair_bar);
-      ok = wait_or_abort(pair_bar, static_cast<uint32_t>(j) & 1u, abort);
-    } else {
-      ok = false;
-    }
     if (__all_sync(0xffffffffu, ok)) {
-      const float l_row = l_sum + xchg[xslot(j & 1, half ^ 1)];
       tc_fence_after();
-      const float inv_l = row_ok ? 1.f / l_row : 0.f;
+      const float inv_l = row_ok ? 1.f / l_sum : 0.f;
       const int head = head0 + s;
-      const int ch0 = half * (D / 2);  // first output channel of this thread
-      const size_t obase = ((static_cast<size_t>(b) * prm.L + row) * prm.Hq + head) * D + ch0;
+      const size_t obase = ((static_cast<size_t>(b) * prm.L + row) * prm.Hq + head) * D;
 #pragma unroll 1
-      for (int c = 0; c < D / 64; ++c) {
+      for (int c = 0; c < D / 32; ++c) {
         uint32_t rr[32];
         __syncwarp();
-        tmem_ld32(tO(s) + lane_base + ch0 + c * 32, rr);  // whole warp, valid row or not
+        tmem_ld32(tO(s) + lane_base + c * 32, rr);  // whole warp, valid row or not
         tmem_wait_ld();
         reg_fence(rr);
         if (!row_ok) continue;
@@ -575,9 +529,9 @@ bifocal_prefill_kernel(const __grid_constant__ CUtensorMap tm_qt,
           }
         }
       }
-      if (row_ok && half == 0 && prm.lse)
+      if (row_ok && prm.lse)
         prm.lse[(static_cast<size_t>(b) * prm.Hq + head) * prm.L + row] =
-            (m_used + log2f(l_row)) * 0.69314718055994531f;
+            (m_used + log2f(l_sum)) * 0.69314718055994531f;
     }
   }
 
