@@ -44,6 +44,7 @@
 // Traffic: K and V once (2 * L * Hkv * D * 2 bytes per token of output);
 // everything else is O(Hq * D * n_split).
 #include <cmath>
+#include <type_traits>
 
 #include "jl_common.cuh"
 #include "sm100_ptx.cuh"
@@ -207,14 +208,15 @@ __device__ __forceinline__ void qk_block(float (&sc)[4], const uint32_t (&q)[D /
 // the correction angle is j (theta'_i - theta_i): Delta j = j, and omega_i
 // holds (theta'_i - theta_i) / (2 pi), a negative fraction in two's complement.
 template <int D>
-__device__ __forceinline__ void correction_rows(uint8_t *tab, int jt, int n, int G, int interp,
-                                                int warp, int nw, int lane,
-                                                const uint64_t *omega) {
+__device__ __forceinline__ void correction_rows(uint8_t *tab, int jt, int n,
+                                                const GroupDivider &gdiv, int interp, int warp,
+                                                int nw, int lane, const uint64_t *omega) {
   using C = DecCfg<D>;
   constexpr float kTurnToRad = 1.4629180792671596e-09f;  // 2 pi / 2^32
   for (int tt = warp; tt < n; tt += nw) {
     const int j = jt + tt;
-    const uint64_t delta = static_cast<uint64_t>(static_cast<int64_t>(interp ? j : remap(j, G) - j));
+    const uint64_t delta =
+        static_cast<uint64_t>(static_cast<int64_t>(interp ? j : remap_fast(j, gdiv) - j));
     if (lane < D / 4) {  // lane: channels 2 lane, 2 lane + 1
       const int i = 2 * lane;
       const int32_t p0 = static_cast<int32_t>((delta * omega[i]) >> 32);
@@ -306,7 +308,7 @@ decode_split_kernel(DecodeArgs a) {
     }
     const int ju = j_begin + u * P;
     if (p - ju > w0eff)
-      correction_rows<D>(dsm + C::CS + (u % kStages) * C::CS_TAB, ju, min(P, j_end - ju), G,
+      correction_rows<D>(dsm + C::CS + (u % kStages) * C::CS_TAB, ju, min(P, j_end - ju), a.gdiv,
                          a.interp, warp, nh, lane, omega);
     __syncwarp();
     if (lane == 0) mbar_arrive(tready(u % kStages));
@@ -403,6 +405,11 @@ decode_split_kernel(DecodeArgs a) {
 
   int slot = 0;
   uint32_t phase = 0;
+  // The stage loop, in two copies: CTAs whose whole chunk lies beyond the
+  // local window (all but the last few splits) run one without the local and
+  // window-edge paths, which needs fewer live registers.
+  auto stage_loop = [&](auto remote_only_tag) {
+  constexpr bool RO = decltype(remote_only_tag)::value;
   for (int t = 0; t < n_stage && ok; ++t) {
     const int jt = j_begin + t * P;
     const int n = min(P, j_end - jt);
@@ -431,7 +438,7 @@ decode_split_kernel(DecodeArgs a) {
         float sc[4] = {0.f, 0.f, 0.f, 0.f};
         if (!BIFOCAL) {
           qk_block<D, false>(sc, qt, krow, cs_row, tq, mat);
-        } else if (all_remote) {
+        } else if (RO || all_remote) {
           qk_block<D, true>(sc, qr, krow, cs_row, tq, mat);
         } else if (all_local) {
           qk_block<D, false>(sc, qt, krow, cs_row, tq, mat);
@@ -510,6 +517,11 @@ decode_split_kernel(DecodeArgs a) {
       phase ^= 1u;
     }
   }
+  };
+  if (BIFOCAL && p - (j_end - 1) > w0eff)
+    stage_loop(std::true_type{});
+  else
+    stage_loop(std::false_type{});
   if (!ok || *abort) {
     // This warp stops.  Warp 0 first lets the copies it posted land
     // (bounded), so none writes into shared memory after the CTA exits: only

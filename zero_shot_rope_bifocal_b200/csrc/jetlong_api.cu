@@ -406,6 +406,7 @@ int cache_attention(const void *q, const void *k_cache, const void *v_cache, voi
   a.w_pretrained = w_pretrained;
   a.w0 = w0;
   a.G = group_size(L, w_pretrained);
+  a.gdiv = make_group_divider(a.G);
   a.theta = rope_theta;
   a.nq = nq;
   a.q_pos0 = q_pos0;

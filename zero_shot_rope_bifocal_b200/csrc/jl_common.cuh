@@ -51,6 +51,29 @@ __host__ __device__ __forceinline__ int group_size(int L, int w_pretrained) {
 // §3.1: remote position f(x) = floor(x / G) for x >= 0.
 __host__ __device__ __forceinline__ int remap(int x, int G) { return x / G; }
 
+// floor(x / G) for 0 <= x < 2^32 by one multiply-high, shift and add
+// (Granlund and Montgomery, "Division by invariant integers using
+// multiplication", 1994, unsigned case): with l = ceil(log2 G),
+// m = floor(2^32 (2^l - G) / G) + 1, t = mulhi(m, x), the quotient is
+// (t + ((x - t) >> min(l, 1))) >> max(l - 1, 0).  The kernels use it where
+// a division by the run-time G would sit in a per-token loop.
+struct GroupDivider {
+  uint32_t m;
+  int sh1, sh2;
+};
+inline GroupDivider make_group_divider(int G) {
+  int l = 0;
+  while ((1ull << l) < static_cast<unsigned long long>(G)) ++l;
+  const unsigned long long m =
+      ((1ull << 32) * ((1ull << l) - static_cast<unsigned long long>(G))) / static_cast<unsigned long long>(G) + 1ull;
+  return GroupDivider{static_cast<uint32_t>(m), l < 1 ? l : 1, l > 1 ? l - 1 : 0};
+}
+__device__ __forceinline__ int remap_fast(int x, const GroupDivider &dv) {
+  const uint32_t u = static_cast<uint32_t>(x);
+  const uint32_t t = __umulhi(dv.m, u);
+  return static_cast<int>((t + ((u - t) >> dv.sh1)) >> dv.sh2);
+}
+
 // RoPE frequency theta^(-2i/D) in double precision.
 __device__ __forceinline__ double rope_freq(int i, int D, double theta) {
   return exp(-2.0 * static_cast<double>(i) / static_cast<double>(D) * log(theta));
@@ -148,6 +171,7 @@ struct DecodeArgs {
   int nq, q_pos0;
   int interp;  // remote map, as in PrefillArgs
   float ramp_alpha, ramp_beta;
+  GroupDivider gdiv;  // floor(x / G) by multiplication
   unsigned int *dev_error;
 };
 
