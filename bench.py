@@ -48,6 +48,17 @@ METRIC = "bifocal-attn prefill TFLOP/s (% BF16 peak) @128K; decode µs/token (% 
 PREFILL_WORKLOAD = "qwen3_8b_128k"
 DECODE_WORKLOAD = "decode_8b_128k"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# DRAM bytes (read + write) of one attention-kernel launch at the headline
+# workload, from an ncu capture (dram__bytes_read.sum + dram__bytes_write.sum)
+# of the kernel sources whose SHA-256 is recorded here; the capture and its
+# command are summarised in the profile named below.  The line reports it only
+# while the sources are unchanged, and null otherwise.
+TRAFFIC_RECORD = {"bytes": 6.95e9, "read_bytes": 5.83e9, "write_bytes": 1.12e9,
+                  "sources_sha256": "141800bd62e5fd0e832ce8f7a10900aea6deca9288c007446025643f4de0c9e2",
+                  "profile": "profiles/prefill_attention_qwen3_8b_L131072_dram.md"}
+TRAFFIC_SOURCES = ("zero_shot_rope_bifocal_b200/csrc/prefill_sm100.cu",
+                   "zero_shot_rope_bifocal_b200/csrc/sm100_ptx.cuh",
+                   "zero_shot_rope_bifocal_b200/csrc/jl_common.cuh")
 NOMINAL = {"hbm_gbs": 8000.0, "bf16_tflops": 2250.0}
 
 
@@ -57,6 +68,13 @@ def prefill_flops(B: int, Hq: int, L: int, D: int) -> int:
     return 4 * B * Hq * D * (L * (L + 1) // 2)
 
 
+def prefill_operand_bytes(B: int, Hq: int, Hkv: int, L: int, D: int) -> int:
+    """Bytes the attention kernel must move at least: the FP16 operands read
+    once (q at true and remote positions, k at true and remote positions, v)
+    and the BF16 output written once."""
+    return (2 * B * Hq * L * D + 3 * B * Hkv * L * D) * 2 + B * L * Hq * D * 2
+
+
 def row_flops(Hq: int, D: int, rows) -> int:
     return sum(4 * Hq * D * (int(i) + 1) for i in rows)
 
@@ -64,6 +82,24 @@ def row_flops(Hq: int, D: int, rows) -> int:
 def decode_bytes(B: int, Hkv: int, L: int, D: int) -> int:
     """K and V BF16 bytes one decode step must stream."""
     return 2 * B * L * Hkv * D * 2
+
+
+def kernel_sources_sha256() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for rel in TRAFFIC_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def measured_traffic():
+    """(bytes, source) of the recorded capture if it is of the current kernel, else (None, why)."""
+    if TRAFFIC_RECORD is None:
+        return None, "no capture recorded"
+    if TRAFFIC_RECORD["sources_sha256"] != kernel_sources_sha256():
+        return None, "kernel changed since the recorded capture"
+    return TRAFFIC_RECORD["bytes"], TRAFFIC_RECORD["profile"]
 
 
 def load_peaks():
@@ -288,6 +324,110 @@ def run_reference(args):
 
 
 # ---------------------------------------------------------------- native arm
+# ---------------------------------------------------------------- per-config sweep
+L2_BYTES = 126 * 2 ** 20
+
+
+def sweep_prefill(jl, torch, dev, stream, name: str, w0: int | None = None, reps: int = 3) -> dict:
+    """One named prefill workload (the RoPE operand pass plus the attention
+    kernel): median per-step and per-kernel times over ``reps`` steps, each
+    preceded by an L2 flush outside the timed events."""
+    from zero_shot_rope_bifocal_b200.synth import WORKLOADS, prefill_inputs
+    w = WORKLOADS[name] if w0 is None else WORKLOADS[name].with_(w0=w0)
+    x = prefill_inputs(w, device=dev)
+    B, L, Hq, Hkv, D = w.B, w.L, w.Hq, w.Hkv, w.D
+    out = torch.empty((B, L, Hq, D), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((B, Hq, L), dtype=torch.float32, device=dev)
+    ws = torch.empty(jl.jetlong_prefill_workspace_size(B, Hq, Hkv, L, D), dtype=torch.uint8,
+                     device=dev)
+    flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
+
+    def rotate():
+        jl.jetlong_prefill_rotate(x.q, x.k, x.v, w.w_pretrained, w.theta, ws, stream=stream)
+
+    def attend():
+        jl.jetlong_prefill_attend(out, lse, Hkv, w.w_pretrained, w.w0, ws, stream=stream)
+
+    for _ in range(2):
+        rotate()
+        attend()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    step_ms, attn_ms = [], []
+    for _ in range(reps):
+        flush.zero_()
+        ev[0].record(stream)
+        rotate()
+        ev[1].record(stream)
+        attend()
+        ev[2].record(stream)
+        torch.cuda.synchronize(dev)
+        step_ms.append(ev[0].elapsed_time(ev[2]))
+        attn_ms.append(ev[1].elapsed_time(ev[2]))
+    if jl.jetlong_device_status() != jl.JL_OK:
+        raise RuntimeError(f"device status not OK after the {name} prefill")
+    flops = prefill_flops(B, Hq, L, D)
+    t_step, t_attn = statistics.median(step_ms), statistics.median(attn_ms)
+    return {"workload": name, "Hq": Hq, "Hkv": Hkv, "L": L, "w_pretrained": w.w_pretrained,
+            "w0": w.w0, "G": -(-L // w.w_pretrained) if L > w.w_pretrained else 1,
+            "step_ms": t_step, "attend_ms": t_attn, "tflops": flops / (t_step * 1e-3) / 1e12,
+            "attend_tflops": flops / (t_attn * 1e-3) / 1e12,
+            "tokens_per_s": B * L / (t_step * 1e-3), "steps": reps,
+            "l2": "flushed before every timed step"}
+
+
+def sweep_decode(jl, torch, dev, stream, name: str, n_cache: int, n_loop: int = 256,
+                 reps: int = 8) -> dict:
+    """Decode steps on ``n_cache`` distinct true-position caches used in
+    turn (so that, together larger than L2, no step is served from L2),
+    captured once as a CUDA graph of ``n_loop`` steps and replayed."""
+    from zero_shot_rope_bifocal_b200.synth import WORKLOADS, decode_inputs
+    w = WORKLOADS[name]
+    caches = []
+    for c in range(n_cache):
+        d = decode_inputs(w.with_(seed=w.seed + 1000 * c), device=dev)
+        kc = torch.empty_like(d.k_raw)
+        jl.jetlong_rope_cache(d.k_raw, kc, 0, w.theta, stream=stream)
+        caches.append((d.q, kc, d.v))
+        del d
+    out = torch.empty((w.B, w.Hq, w.D), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((w.B, w.Hq), dtype=torch.float32, device=dev)
+    ws = torch.empty(jl.jetlong_decode_workspace_size(w.B, w.Hq, w.Hkv, w.L, w.D),
+                     dtype=torch.uint8, device=dev)
+
+    def dstep(i, st):
+        q, kc, v = caches[i % n_cache]
+        jl.jetlong_decode(q, kc, v, w.L, w.w_pretrained, w.w0, w.theta, out=out, lse=lse,
+                          workspace=ws, stream=st)
+
+    for i in range(3 * n_cache):
+        dstep(i, stream)
+    torch.cuda.synchronize(dev)
+    cap = torch.cuda.Stream(dev)
+    cap.wait_stream(stream)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=cap):
+        for i in range(n_loop):
+            dstep(i, cap)
+    g.replay()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        g.replay()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    del g
+    if jl.jetlong_device_status() != jl.JL_OK:
+        raise RuntimeError(f"device status not OK after the {name} decode")
+    us = 1e3 * e0.elapsed_time(e1) / (n_loop * reps)
+    nbytes = decode_bytes(w.B, w.Hkv, w.L, w.D)
+    return {"workload": name, "L": w.L, "G": -(-w.L // w.w_pretrained) if w.L > w.w_pretrained
+            else 1, "us_per_token": us, "tokens_per_s": w.B * 1e6 / us,
+            "achieved_gbs": nbytes / (us * 1e-6) / 1e9, "bytes_per_token": nbytes,
+            "steps": n_loop * reps, "caches": n_cache,
+            "l2": f"{n_cache} distinct caches of {nbytes / 2 ** 20:.0f} MiB used in turn"}
+
+
 def run_native(args):
     import torch
     import torch.distributed as dist
@@ -623,6 +763,17 @@ def run_native(args):
     h2d = (hq.numel() + hk.numel() + hv.numel()) * 2
     d2h = hbuf[0][0].numel() * 2 + hbuf[0][1].numel() * 4
 
+    # ---- every workload of the benchmark plan: prefill at 16K / 64K (with the
+    # w0 sweep) and 128K, decode at 32K / 64K / 128K
+    sweep = {"prefill": [], "decode": []}
+    if not args.no_sweep:
+        for name, w0s in (("qwen3_1p7b_16k", [None]), ("qwen3_1p7b_64k", [None]),
+                          ("qwen3_8b_64k", [2048, 4096, 8192]), ("qwen3_8b_128k", [None])):
+            for w0 in w0s:
+                sweep["prefill"].append(sweep_prefill(jl, torch, dev, stream, name, w0))
+        for name, n_cache in (("decode_8b_32k", 3), ("decode_8b_64k", 2), ("decode_8b_128k", 1)):
+            sweep["decode"].append(sweep_decode(jl, torch, dev, stream, name, n_cache))
+
     # ---- CPU oracle baseline (rank 0, N=1 only)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -635,6 +786,7 @@ def run_native(args):
 
     if rank == 0:
         peaks, src = load_peaks()
+        traffic, traffic_src = measured_traffic()
         attn_tflops = prefill_flops(B, Hq, L, D) / (attn_ms * 1e-3) / 1e12
         peak = peaks["bf16_tflops_sustained"]
         line = {
@@ -653,7 +805,8 @@ def run_native(args):
                          "peak_source": f"{src} bf16_tflops_sustained",
                          "nominal_frac": attn_tflops / NOMINAL["bf16_tflops"],
                          "kernel": "bifocal_prefill_kernel<128>", "kernel_ms": attn_ms,
-                         "traffic": None},
+                         "traffic": traffic, "traffic_source": traffic_src,
+                         "algorithmic_bytes": prefill_operand_bytes(B, Hq, Hkv, L, D)},
             "breakdown_ms": {"rotate": rot_ms, "attend": attn_ms},
             "decode": {"workload": DECODE_WORKLOAD, "us_per_token": us_tok,
                        "tokens_per_s": wd.B * 1e6 / us_tok, "steps": n_dec,
@@ -695,6 +848,13 @@ def run_native(args):
                 "decode_us_per_token": interp_us_tok,
                 "vs_alias_prefill_step": interp_ms / (t_max / args.steps),
                 "vs_alias_decode_host_launched": interp_us_tok / host_loop_us},
+            "configs": {
+                "what": "each workload of the benchmark plan on this rank: prefill = RoPE operand "
+                        "pass + attention kernel, median of 3 steps after an L2 flush; decode = "
+                        "graph replays of 256-step loops",
+                "prefill": [dict(c, attend_frac=c["attend_tflops"] / peak) for c in sweep["prefill"]],
+                "decode": [dict(c, frac=c["achieved_gbs"] / peaks["hbm_gbs"])
+                           for c in sweep["decode"]]},
             "e2e": {"value": e2e_val, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "steps": n_e2e,
                     "pipelined": "step i's H2D and step i-1's D2H overlap compute on two copy "
@@ -716,10 +876,12 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["native", "reference"], default="native")
     ap.add_argument("--decode-steps", type=int, default=256)
-    ap.add_argument("--decode-reps", type=int, default=8)
+    ap.add_argument("--decode-reps", type=int, default=80)
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--reference-seconds", type=float, default=120.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-sweep", action="store_true",
+                    help="skip the per-workload sweep (16K-128K prefill, 32K-128K decode)")
     args = ap.parse_args(argv)
     args.warmup = max(3, args.warmup)  # at least three untimed warm-up steps
     if args.impl == "reference":
