@@ -675,6 +675,49 @@ def run_native(args):
     if jl.jetlong_device_status() != jl.JL_OK:
         raise RuntimeError("device status not OK after the interpolation decode")
 
+    # the two-form key cache: the remote form of every key written once for
+    # this G (timed), then decode steps that read remote keys from it
+    kr = torch.empty(kc.shape, dtype=torch.float16, device=dev)
+    jl.jetlong_remote_cache(kc, kr, 0, wd.L, wd.L, wd.w_pretrained, wd.theta, stream=stream)
+    barrier()
+    torch.cuda.synchronize(dev)
+    ev0.record(stream)
+    jl.jetlong_remote_cache(kc, kr, 0, wd.L, wd.L, wd.w_pretrained, wd.theta, stream=stream)
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    rebuild_ms = reduce_max(ev0.elapsed_time(ev1), world, dev)
+
+    def dstep_two(st=None):
+        jl.jetlong_decode_two_form(dq, kc, kr, d.v, wd.L, wd.w_pretrained, wd.w0, wd.theta,
+                                   out=dout, lse=dlse, workspace=dws,
+                                   stream=stream if st is None else st)
+
+    for _ in range(3):
+        dstep_two()
+    torch.cuda.synchronize(dev)
+    cap2 = torch.cuda.Stream(dev)
+    cap2.wait_stream(stream)
+    g2 = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g2, stream=cap2):
+        for _ in range(n_loop):
+            dstep_two(cap2)
+    g2.replay()
+    n_rep2 = 8
+    barrier()
+    torch.cuda.synchronize(dev)
+    ev0.record(stream)
+    for _ in range(n_rep2):
+        g2.replay()
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    del g2
+    two_us_tok = 1e3 * reduce_max(ev0.elapsed_time(ev1), world, dev) / (n_loop * n_rep2)
+    del kr
+    if jl.jetlong_device_status() != jl.JL_OK:
+        raise RuntimeError("device status not OK after the two-form decode")
+
     # a 64-token prefill chunk appended at the end of the same 128K cache
     n_chunk = 64
     P0 = wd.L - n_chunk
@@ -855,6 +898,15 @@ def run_native(args):
                 "prefill": [dict(c, attend_frac=c["attend_tflops"] / peak) for c in sweep["prefill"]],
                 "decode": [dict(c, frac=c["achieved_gbs"] / peaks["hbm_gbs"])
                            for c in sweep["decode"]]},
+            "two_form": {
+                "what": "decode reading remote keys from an FP16 remote form of the cache "
+                        "(jetlong_remote_cache once per G, jetlong_decode_two_form per step), "
+                        "CUDA-graph replays of 256-step loops like the headline decode",
+                "decode_us_per_token": two_us_tok,
+                "achieved_gbs": decode_bytes(wd.B, wd.Hkv, wd.L, wd.D) / (two_us_tok * 1e-6) / 1e9,
+                "vs_rotating_decode": two_us_tok / us_tok,
+                "rebuild_ms_all_rows": rebuild_ms,
+                "rebuild_every_tokens": wd.w_pretrained},
             "e2e": {"value": e2e_val, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "steps": n_e2e,
                     "pipelined": "step i's H2D and step i-1's D2H overlap compute on two copy "

@@ -333,6 +333,36 @@ JL_API int jetlong_prefill_chunk_interp(const void *q, const void *k_cache, cons
                                         jl_stream_t stream);
 
 /*
+ * Two-form key cache for decode (a layout choice of this library; the paper
+ * keeps one cache and rotates remote keys on every step, §3.2).  Beside the
+ * true-position cache, the caller keeps k_remote [B, Lcap, Hkv, D] FP16:
+ *
+ *   k_remote[b, j, g, :] = FP16(R(f(j) - j) k_cache[b, j, g, :]),  G = G(L),
+ *
+ * the remote form of each key for the G of the length L it is read at.
+ * jetlong_remote_cache writes rows [j0, j1) of it for the G of L
+ * (0 <= j0 <= j1 <= L <= Lcap; j0 == j1 does nothing).  A generation loop
+ * writes the new token's row after appending it, and rewrites rows [0, L)
+ * whenever G changes (once per w_pretrained tokens).
+ *
+ * jetlong_decode_two_form is jetlong_decode with remote keys read from
+ * k_remote instead of being rotated on the fly.  Rows [0, L - 1 - w0) of
+ * k_remote must hold the remote form for G(L).  Same arguments, layouts,
+ * workspace and results as jetlong_decode.  The rotation and FP16 rounding
+ * are the ones the on-the-fly path applies, so the tensor-core operands are
+ * identical.
+ */
+JL_API int jetlong_remote_cache(const void *k_cache, void *k_remote, int B, int Lcap, int Hkv,
+                                int D, int j0, int j1, int L, int w_pretrained, float rope_theta,
+                                jl_stream_t stream);
+
+JL_API int jetlong_decode_two_form(const void *q, const void *k_cache, const void *k_remote,
+                                   const void *v_cache, void *out, float *lse, int B, int Hq,
+                                   int Hkv, int L, int Lcap, int D, int w_pretrained, int w0,
+                                   float rope_theta, int out_dtype, void *workspace,
+                                   size_t workspace_bytes, jl_stream_t stream);
+
+/*
  * Write keys into the true-position cache (§3.2): for t < n,
  *   k_cache[b, pos0 + t, h, :] = RoPE(k[b, t, h, :], pos0 + t).
  *

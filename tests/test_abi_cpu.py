@@ -347,3 +347,31 @@ def test_header_states_the_fp16_range_contract():
     assert "still returns JL_OK, and its outputs may hold non-finite values" in text
     assert "the next jetlong_device_status() returns JL_ERR_RANGE" in text
     assert "record nothing" in text
+
+
+# ---------------------------------------------------------------- two-form key cache
+@pytest.mark.parametrize("args,status", [
+    ((None, P, 1, 100, 8, 128, 0, 10, 100, 32, 1e4, None), jl.JL_ERR_NULL),
+    ((P, P, 1, 100, 8, 128, 0, 10, 101, 32, 1e4, None), jl.JL_ERR_SHAPE),   # L > Lcap
+    ((P, P, 1, 100, 8, 128, 5, 4, 100, 32, 1e4, None), jl.JL_ERR_SHAPE),    # j1 < j0
+    ((P, P, 1, 100, 8, 128, 0, 60, 50, 32, 1e4, None), jl.JL_ERR_SHAPE),    # j1 > L
+    ((P, P, 1, 100, 8, 96, 0, 10, 100, 32, 1e4, None), jl.JL_ERR_UNSUPPORTED),
+    ((P, P, 1, 100, 8, 128, 0, 10, 100, 0, 1e4, None), jl.JL_ERR_SHAPE),    # w_pretrained
+    ((P, ctypes.c_void_p(264), 1, 100, 8, 128, 0, 10, 100, 32, 1e4, None), jl.JL_ERR_ALIGN),
+    ((P, P, 1, 100, 8, 128, 7, 7, 100, 32, 1e4, None), jl.JL_OK),          # nothing to write
+])
+def test_remote_cache_rejects_bad_arguments(lib, args, status):
+    assert lib.jetlong_remote_cache(*args) == status
+
+
+def test_two_form_decode_checks_its_remote_cache(lib):
+    a = [P, P, P, P, P, None, 1, 32, 8, 1000, 1000, 128, 32768, 4096, 1e6, 0, P, 1 << 40, None]
+    bad = list(a)
+    bad[2] = None
+    assert lib.jetlong_decode_two_form(*bad) == jl.JL_ERR_NULL
+    bad = list(a)
+    bad[2] = ctypes.c_void_p(264)
+    assert lib.jetlong_decode_two_form(*bad) == jl.JL_ERR_ALIGN
+    bad = list(a)
+    bad[17] = 0
+    assert lib.jetlong_decode_two_form(*bad) == jl.JL_ERR_WORKSPACE

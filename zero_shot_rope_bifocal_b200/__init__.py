@@ -11,6 +11,7 @@ from .jetlong import (  # noqa: F401
     JetLongError,
     jetlong_decode,
     jetlong_decode_interp,
+    jetlong_decode_two_form,
     jetlong_decode_workspace_size,
     jetlong_device_status,
     jetlong_group_size,
@@ -24,6 +25,7 @@ from .jetlong import (  # noqa: F401
     jetlong_prefill_three_pass,
     jetlong_prefill_three_pass_workspace_size,
     jetlong_prefill_workspace_size,
+    jetlong_remote_cache,
     jetlong_rope_cache,
 )
 

@@ -153,7 +153,14 @@ __device__ __forceinline__ float bf_hi(uint32_t u) { return __uint_as_float(u & 
 // k-blocks [kb0, kb0 + 2) and their RoPE partners [kb0 + KB/2, kb0 + KB/2 + 2).
 // K is read with ldmatrix as FP16-converted B fragments; remote tokens are
 // first turned by the correction rotation (channel c pairs with c + D/2).
-template <int D, bool REMOTE>
+// How a stage's key rows are turned into FP16 B fragments.
+enum KeyKind : int {
+  kKeyBf16 = 0,    // cached BF16 key at its true position: converted
+  kKeyRotate = 1,  // cached BF16 key of a remote token: turned by R(Delta j), converted
+  kKeyF16 = 2,     // remote form of the key, stored as FP16: used as read
+};
+
+template <int D, int KIND>
 __device__ __forceinline__ void qk_pair(float (&sc)[4], const uint32_t (&q)[D / 16][2],
                                         uint32_t krow_addr, const uint8_t *cs_row, int kb0,
                                         int tq, int mat) {
@@ -161,11 +168,12 @@ __device__ __forceinline__ void qk_pair(float (&sc)[4], const uint32_t (&q)[D / 
   uint32_t lo[4], hi[4];      // k-blocks kb0, kb0 + 1 and their partners
   ldsm_x4(krow_addr + (16 * kb0 + 8 * (mat & 1) + 16 * (mat >> 1)) * 2, lo);
   ldsm_x4(krow_addr + (16 * (kb0 + HK) + 8 * (mat & 1) + 16 * (mat >> 1)) * 2, hi);
+  // kKeyF16: the ldmatrix fragments are the FP16 operand already
 #pragma unroll
-  for (int r = 0; r < 4; ++r) {
+  for (int r = 0; r < (KIND == kKeyF16 ? 0 : 4); ++r) {
     const float x0 = bf_lo(lo[r]), x1 = bf_hi(lo[r]);
     const float y0 = bf_lo(hi[r]), y1 = bf_hi(hi[r]);
-    if constexpr (REMOTE) {
+    if constexpr (KIND == kKeyRotate) {
       // lo[r]: channels c, c + 1 with c = 16 (kb0 + r / 2) + 8 (r % 2) + 2 tq
       const int c = 16 * (kb0 + (r >> 1)) + 8 * (r & 1) + 2 * tq;
       const float4 cs = *reinterpret_cast<const float4 *>(cs_row + c * 8);  // cos c, c+1, sin c, c+1
@@ -186,7 +194,7 @@ __device__ __forceinline__ void qk_pair(float (&sc)[4], const uint32_t (&q)[D / 
   mma_f16(sc, q[kb0 + HK + 1][0], 0u, q[kb0 + HK + 1][1], 0u, hi[2], hi[3]);
 }
 
-template <int D, bool REMOTE>
+template <int D, int KIND>
 __device__ __forceinline__ void qk_block(float (&sc)[4], const uint32_t (&q)[D / 16][2],
                                          uint32_t krow_addr, const uint8_t *cs_row, int tq,
                                          int mat) {
@@ -194,7 +202,7 @@ __device__ __forceinline__ void qk_block(float (&sc)[4], const uint32_t (&q)[D /
   // two interleaved chains (more registers live) measured slower
 #pragma unroll
   for (int kb0 = 0; kb0 < D / 32; kb0 += 2)
-    qk_pair<D, REMOTE>(sc, q, krow_addr, cs_row, kb0, tq, mat);
+    qk_pair<D, KIND>(sc, q, krow_addr, cs_row, kb0, tq, mat);
 }
 
 // Rows of the correction table of one stage: cos and sin of Delta j * theta_i
@@ -246,8 +254,11 @@ __device__ __forceinline__ bool dec_wait(uint32_t bar, uint32_t parity, volatile
 }
 
 // BIFOCAL = false is the G = 1 instantiation: every key is local, so it has
-// no remote query, no correction table and no rotation code.
-template <int D, int GRP, bool BIFOCAL>
+// no remote query, no correction table and no rotation code.  TWO_FORM (with
+// BIFOCAL) reads remote tokens' keys from the FP16 remote form of the cache
+// (a.k_remote, already turned by R(Delta j)) instead of rotating them: no
+// correction table either.
+template <int D, int GRP, bool BIFOCAL, bool TWO_FORM = false>
 __global__ void __launch_bounds__(kDecThreads, kCtasPerSm)
 decode_split_kernel(DecodeArgs a) {
   using C = DecCfg<D>;
@@ -295,7 +306,10 @@ decode_split_kernel(DecodeArgs a) {
       const int j = min(ju + t2, j_end - 1);
       const size_t off = (static_cast<size_t>(b) * a.Lcap + j) * cache_row + static_cast<size_t>(g0) * D;
       const uint32_t dst = sb + slot * C::STAGE + (lane & 1) * C::HALF_STAGE + t2 * C::ROW;
-      bulk_copy(dst, ((lane & 1) ? a.v_cache : a.k_cache) + off, head_bytes, full(slot));
+      const void *src = (lane & 1) ? static_cast<const void *>(a.v_cache + off)
+                        : (TWO_FORM && p - j > w0eff) ? static_cast<const void *>(a.k_remote + off)
+                                                      : static_cast<const void *>(a.k_cache + off);
+      bulk_copy(dst, src, head_bytes, full(slot));
     }
   };
   // This warp's rows of the correction table of stage u (table u % kStages),
@@ -353,7 +367,7 @@ decode_split_kernel(DecodeArgs a) {
   __syncthreads();
   if (warp >= nh) return;  // no KV head for this warp; nothing below waits for it
   bool ok = true;
-  if constexpr (BIFOCAL) {
+  if constexpr (BIFOCAL && !TWO_FORM) {
     ok = table(0);
     if (ok && n_stage > 1) ok = table(1);
   }
@@ -413,7 +427,8 @@ decode_split_kernel(DecodeArgs a) {
   for (int t = 0; t < n_stage && ok; ++t) {
     const int jt = j_begin + t * P;
     const int n = min(P, j_end - jt);
-    ok = dec_wait(full(slot), phase, abort) && (!BIFOCAL || dec_wait(tready(slot), phase, abort));
+    ok = dec_wait(full(slot), phase, abort) &&
+         (!BIFOCAL || TWO_FORM || dec_wait(tready(slot), phase, abort));
     if (!__all_sync(0xffffffffu, ok)) {
       ok = false;
       break;
@@ -436,16 +451,19 @@ decode_split_kernel(DecodeArgs a) {
         const bool all_remote = p - (jb + 7) > w0eff;
         const bool all_local = p - jb <= w0eff;
         float sc[4] = {0.f, 0.f, 0.f, 0.f};
+        constexpr int kRemoteKind = TWO_FORM ? kKeyF16 : kKeyRotate;
         if (!BIFOCAL) {
-          qk_block<D, false>(sc, qt, krow, cs_row, tq, mat);
+          qk_block<D, kKeyBf16>(sc, qt, krow, cs_row, tq, mat);
         } else if (RO || all_remote) {
-          qk_block<D, true>(sc, qr, krow, cs_row, tq, mat);
+          qk_block<D, kRemoteKind>(sc, qr, krow, cs_row, tq, mat);
         } else if (all_local) {
-          qk_block<D, false>(sc, qt, krow, cs_row, tq, mat);
+          qk_block<D, kKeyBf16>(sc, qt, krow, cs_row, tq, mat);
         } else {  // the block on the window edge: both variants, picked per token
+          // (with TWO_FORM the rows of one variant hold the other's format;
+          // those columns of S are computed but never picked)
           float sl[4] = {0.f, 0.f, 0.f, 0.f};
-          qk_block<D, true>(sc, qr, krow, cs_row, tq, mat);
-          qk_block<D, false>(sl, qt, krow, cs_row, tq, mat);
+          qk_block<D, kRemoteKind>(sc, qr, krow, cs_row, tq, mat);
+          qk_block<D, kKeyBf16>(sl, qt, krow, cs_row, tq, mat);
           if (p - (jb + 2 * tq) <= w0eff) sc[0] = sl[0];
           if (p - (jb + 2 * tq + 1) <= w0eff) sc[1] = sl[1];
         }
@@ -506,7 +524,7 @@ decode_split_kernel(DecodeArgs a) {
     __syncwarp();
     if (lane == 0) mbar_arrive(empty(slot));
     // This warp's rows of the table two stages ahead.
-    if (BIFOCAL && t + 2 < n_stage) ok = table(t + 2);
+    if (BIFOCAL && !TWO_FORM && t + 2 < n_stage) ok = table(t + 2);
     // Warp 0 refills this slot once every warp has released it.
     if (warp == 0 && ok && t + kStages < n_stage) {
       ok = __all_sync(0xffffffffu, dec_wait(empty(slot), phase, abort));
@@ -559,6 +577,49 @@ decode_split_kernel(DecodeArgs a) {
     float *rec = rec0 + gq * rec_stride;
     rec[D] = m_run;
     rec[D + 1] = l_run;
+  }
+}
+
+// Remote form of the key cache, for the two-form decode: for tokens
+// j in [j0, j1) of batch entry blockIdx.y and every KV head,
+//   k_remote[b, j, g, :] = FP16(R(f(j) - j) k_cache[b, j, g, :]),
+// with G from the length L the cache will be read at.  The table rows come
+// from correction_rows and the rotation is the packed sequence of qk_pair,
+// so the decode kernel's tensor-core operands are the same either way.
+// One warp per token, eight tokens per CTA; lane l turns channel pair
+// (2l, 2l + 1) and its RoPE partners.
+template <int D>
+__global__ void __launch_bounds__(kDecThreads)
+remote_cache_kernel(const __nv_bfloat16 *__restrict__ k_cache, __half *__restrict__ k_remote,
+                    int Lcap, int Hkv, int j0, int j1, GroupDivider gdiv, float theta) {
+  using C = DecCfg<D>;
+  constexpr int HALF = D / 2;
+  __shared__ __align__(16) uint8_t tab[kDecWarps * C::CS_ROW];
+  __shared__ uint64_t omega[HALF];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int b = blockIdx.y;
+  const int jt = j0 + blockIdx.x * kDecWarps;
+  const int n = min(kDecWarps, j1 - jt);
+  constexpr double kTurnsQ64 = 0.15915494309189533577 * 18446744073709551616.0;  // 2^64 / (2 pi)
+  for (int i = threadIdx.x; i < HALF; i += kDecThreads)
+    omega[i] = __double2ull_rn(rope_freq(i, D, static_cast<double>(theta)) * kTurnsQ64);
+  __syncthreads();
+  correction_rows<D>(tab, jt, n, gdiv, 0, warp, kDecWarps, lane, omega);  // row `warp`
+  __syncwarp();
+  if (warp >= n || lane >= D / 4) return;
+  const int c = 2 * lane;
+  const float4 cs = *reinterpret_cast<const float4 *>(tab + warp * C::CS_ROW + c * 8);
+  const float2 co = make_float2(cs.x, cs.y), si = make_float2(cs.z, cs.w);
+  const size_t row0 = (static_cast<size_t>(b) * Lcap + jt + warp) * Hkv * D;
+  for (int g = 0; g < Hkv; ++g) {
+    const size_t row = row0 + static_cast<size_t>(g) * D;
+    const uint32_t lo = *reinterpret_cast<const uint32_t *>(k_cache + row + c);
+    const uint32_t hi = *reinterpret_cast<const uint32_t *>(k_cache + row + c + HALF);
+    const float2 xx = make_float2(bf_lo(lo), bf_hi(lo)), yy = make_float2(bf_lo(hi), bf_hi(hi));
+    const float2 l2 = fsub2(fmul2(xx, co), fmul2(yy, si));  // x cos - y sin
+    const float2 h2 = ffma2(yy, co, fmul2(xx, si));         // x sin + y cos
+    *reinterpret_cast<uint32_t *>(k_remote + row + c) = pack_f16(l2.x, l2.y);
+    *reinterpret_cast<uint32_t *>(k_remote + row + c + HALF) = pack_f16(h2.x, h2.y);
   }
 }
 
@@ -658,19 +719,22 @@ decode_combine_kernel(DecodeArgs a) {
   }
 }
 
-template <int D, int GRP, bool BIFOCAL>
+template <int D, int GRP, bool BIFOCAL, bool TWO_FORM>
 cudaError_t launch_split_v(const DecodeArgs &a, cudaStream_t stream) {
   const int smem = DecCfg<D>::BYTES;
-  cudaError_t e = ensure_smem_limit<decode_split_kernel<D, GRP, BIFOCAL>>(smem);
+  cudaError_t e = ensure_smem_limit<decode_split_kernel<D, GRP, BIFOCAL, TWO_FORM>>(smem);
   if (e != cudaSuccess) return e;
   const int n_chunk = (a.Hkv + kDecWarps - 1) / kDecWarps;
-  decode_split_kernel<D, GRP, BIFOCAL><<<dim3(a.n_split, n_chunk, a.B * a.nq), kDecThreads, smem, stream>>>(a);
+  decode_split_kernel<D, GRP, BIFOCAL, TWO_FORM>
+      <<<dim3(a.n_split, n_chunk, a.B * a.nq), kDecThreads, smem, stream>>>(a);
   return cudaGetLastError();
 }
 
 template <int D, int GRP>
 cudaError_t launch_split(const DecodeArgs &a, cudaStream_t stream) {
-  return a.G > 1 ? launch_split_v<D, GRP, true>(a, stream) : launch_split_v<D, GRP, false>(a, stream);
+  if (a.G == 1) return launch_split_v<D, GRP, false, false>(a, stream);
+  return a.k_remote ? launch_split_v<D, GRP, true, true>(a, stream)
+                    : launch_split_v<D, GRP, true, false>(a, stream);
 }
 
 template <int D>
@@ -723,6 +787,19 @@ bool decode_supports_group(int grp) { return grp == 1 || grp == 2 || grp == 4 ||
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t stream) {
   if (a.D == 128) return launch_decode_d<128>(a, stream);
   return launch_decode_d<64>(a, stream);
+}
+
+cudaError_t launch_remote_cache(const __nv_bfloat16 *k_cache, __half *k_remote, int B, int Lcap,
+                                int Hkv, int D, int j0, int j1, int G, float theta,
+                                cudaStream_t stream) {
+  const dim3 grid((j1 - j0 + kDecWarps - 1) / kDecWarps, B);
+  if (D == 128)
+    remote_cache_kernel<128><<<grid, kDecThreads, 0, stream>>>(k_cache, k_remote, Lcap, Hkv, j0,
+                                                                j1, make_group_divider(G), theta);
+  else
+    remote_cache_kernel<64><<<grid, kDecThreads, 0, stream>>>(k_cache, k_remote, Lcap, Hkv, j0,
+                                                               j1, make_group_divider(G), theta);
+  return cudaGetLastError();
 }
 
 }  // namespace jl

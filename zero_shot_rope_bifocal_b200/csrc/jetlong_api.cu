@@ -349,8 +349,9 @@ namespace {
 int check_cache_call(const void *q, const void *k_cache, const void *v_cache, const void *out,
                      const float *lse, int B, int Hq, int Hkv, int nq, int q_pos0, int Lcap, int D,
                      int w_pretrained, int w0, float rope_theta, int out_dtype, int interp,
-                     float ramp_alpha, float ramp_beta, int *L_out) {
+                     float ramp_alpha, float ramp_beta, const void *k_remote, int *L_out) {
   if (!q || !k_cache || !v_cache || !out) return JL_ERR_NULL;
+  if (k_remote && !aligned16(k_remote)) return JL_ERR_ALIGN;
   if (interp && check_ramp(ramp_alpha, ramp_beta) != JL_OK) return JL_ERR_SHAPE;
   if (nq < 1 || q_pos0 < 0) return JL_ERR_SHAPE;
   const long long L_ll = static_cast<long long>(q_pos0) + nq;
@@ -376,11 +377,12 @@ int cache_attention(const void *q, const void *k_cache, const void *v_cache, voi
                     int B, int Hq, int Hkv, int nq, int q_pos0, int Lcap, int D, int w_pretrained,
                     int w0, float rope_theta, int out_dtype, void *workspace,
                     size_t workspace_bytes, jl_stream_t stream, int interp = 0,
-                    float ramp_alpha = 0.f, float ramp_beta = 0.f) {
+                    float ramp_alpha = 0.f, float ramp_beta = 0.f,
+                    const void *k_remote = nullptr) {
   int L = 0;
   int st = check_cache_call(q, k_cache, v_cache, out, lse, B, Hq, Hkv, nq, q_pos0, Lcap, D,
                             w_pretrained, w0, rope_theta, out_dtype, interp, ramp_alpha,
-                            ramp_beta, &L);
+                            ramp_beta, k_remote, &L);
   if (st != JL_OK) return st;
   const size_t need = decode_ws_bytes(B * nq, Hq, Hkv, L, D);
   if (!workspace || workspace_bytes < need) return JL_ERR_WORKSPACE;
@@ -393,6 +395,7 @@ int cache_attention(const void *q, const void *k_cache, const void *v_cache, voi
   a.q = static_cast<const __nv_bfloat16 *>(q);
   a.k_cache = static_cast<const __nv_bfloat16 *>(k_cache);
   a.v_cache = static_cast<const __nv_bfloat16 *>(v_cache);
+  a.k_remote = static_cast<const __half *>(k_remote);
   a.out = out;
   a.lse = lse;
   a.out_f32 = out_dtype == JL_F32;
@@ -468,6 +471,38 @@ int jetlong_prefill_chunk_interp(const void *q, const void *k_cache, const void 
   return cache_attention(q, k_cache, v_cache, out, lse, B, Hq, Hkv, n, P0, Lcap, D,
                          w_pretrained, w0, rope_theta, out_dtype, workspace, workspace_bytes,
                          stream, 1, ramp_alpha, ramp_beta);
+}
+
+int jetlong_remote_cache(const void *k_cache, void *k_remote, int B, int Lcap, int Hkv, int D,
+                         int j0, int j1, int L, int w_pretrained, float rope_theta,
+                         jl_stream_t stream) {
+  if (!k_cache || !k_remote) return JL_ERR_NULL;
+  if (B < 1 || B > 65535 || Hkv < 1 || L < 1 || Lcap < L) return JL_ERR_SHAPE;
+  if (j0 < 0 || j1 < j0 || j1 > L) return JL_ERR_SHAPE;
+  if (D != 64 && D != 128) return JL_ERR_UNSUPPORTED;
+  int st = check_method(w_pretrained, 0, rope_theta);
+  if (st != JL_OK) return st;
+  if (!aligned16(k_cache) || !aligned16(k_remote)) return JL_ERR_ALIGN;
+  if (j0 == j1) return JL_OK;
+  DeviceState *dev = nullptr;
+  if ((st = current_device(&dev)) != JL_OK) return st;
+  if (launch_remote_cache(static_cast<const __nv_bfloat16 *>(k_cache), static_cast<__half *>(k_remote),
+                          B, Lcap, Hkv, D, j0, j1, group_size(L, w_pretrained), rope_theta,
+                          reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return JL_ERR_CUDA;
+  return JL_OK;
+}
+
+int jetlong_decode_two_form(const void *q, const void *k_cache, const void *k_remote,
+                            const void *v_cache, void *out, float *lse, int B, int Hq, int Hkv,
+                            int L, int Lcap, int D, int w_pretrained, int w0, float rope_theta,
+                            int out_dtype, void *workspace, size_t workspace_bytes,
+                            jl_stream_t stream) {
+  if (!k_remote) return JL_ERR_NULL;
+  if (L < 1) return JL_ERR_SHAPE;
+  return cache_attention(q, k_cache, v_cache, out, lse, B, Hq, Hkv, 1, L - 1, Lcap, D,
+                         w_pretrained, w0, rope_theta, out_dtype, workspace, workspace_bytes,
+                         stream, 0, 0.f, 0.f, k_remote);
 }
 
 int jetlong_rope_cache(const void *k, void *k_cache, int B, int n, int Hkv, int D, int pos0,
@@ -571,7 +606,8 @@ extern "C" int jetlong_decode_noalloc(const void *q, const void *k_cache, const 
   if (L < 1) return JL_ERR_SHAPE;
   int L_checked = 0;
   int st = check_cache_call(q, k_cache, v_cache, out, lse, B, Hq, Hkv, 1, L - 1, Lcap, D,
-                            w_pretrained, w0, rope_theta, out_dtype, 0, 0.f, 0.f, &L_checked);
+                            w_pretrained, w0, rope_theta, out_dtype, 0, 0.f, 0.f, nullptr,
+                            &L_checked);
   if (st != JL_OK) return st;
   if (decode_ws_bytes(B, Hq, Hkv, L, D) > kNoAllocScratchBytes) return JL_ERR_WORKSPACE;
   // Then the device (an sm_100 one), and only then the buffer's address.

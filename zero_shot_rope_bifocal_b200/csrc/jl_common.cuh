@@ -157,6 +157,9 @@ cudaError_t launch_three_pass_merge(const float *o_a, const float *o_b, const fl
 
 struct DecodeArgs {
   const __nv_bfloat16 *q, *k_cache, *v_cache;
+  // Remote form of the key cache, FP16 R(f(j) - j) k_cache[j] for the call's
+  // G (same layout as k_cache), or NULL: then remote keys are turned on the fly.
+  const __half *k_remote;
   void *out;
   float *lse;
   int out_f32;
@@ -182,6 +185,11 @@ void decode_plan(int B, int Hkv, int L, int *n_split, int *chunk);
 bool decode_supports_group(int grp);
 
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t stream);
+
+// k_remote[b, j] = FP16(R(f(j) - j) k_cache[b, j]) for j in [j0, j1), all KV heads.
+cudaError_t launch_remote_cache(const __nv_bfloat16 *k_cache, __half *k_remote, int B, int Lcap,
+                                int Hkv, int D, int j0, int j1, int G, float theta,
+                                cudaStream_t stream);
 
 cudaError_t launch_rope_cache(const __nv_bfloat16 *k, __nv_bfloat16 *k_cache, int B, int n,
                               int Hkv, int D, int pos0, int Lcap, float theta,

@@ -62,6 +62,9 @@ SIGNATURES = {
                                    _F, _F, _I, _VP, _SZ, _VP]),
     "jetlong_prefill_chunk_interp": (_I, [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _I,
                                           _I, _I, _F, _F, _F, _I, _VP, _SZ, _VP]),
+    "jetlong_remote_cache": (_I, [_VP, _VP, _I, _I, _I, _I, _I, _I, _I, _I, _F, _VP]),
+    "jetlong_decode_two_form": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _I,
+                                     _I, _F, _I, _VP, _SZ, _VP]),
     "jetlong_rope_cache": (_I, [_VP, _VP, _I, _I, _I, _I, _I, _I, _F, _VP]),
     "jetlong_device_status": (_I, [_VP]),
     "jetlong_check_device_timeout": (_I, [_I, _VP]),
@@ -418,6 +421,52 @@ def jetlong_decode_noalloc(q, k_cache, v_cache, L: int, w_pretrained: int, w0: i
                                       B, Hq, Hkv, int(L), Lcap, D, int(w_pretrained), int(w0),
                                       float(rope_theta), od, _stream_ptr(stream))
     _check("jetlong_decode_noalloc", st)
+    return out, lse
+
+
+def jetlong_remote_cache(k_cache, k_remote, j0: int, j1: int, L: int, w_pretrained: int,
+                         rope_theta: float, *, stream=None):
+    """Write rows [j0, j1) of the FP16 remote form of the key cache for the G
+    of length L: k_remote[:, j] = R(f(j) - j) k_cache[:, j]."""
+    B, Lcap, Hkv, D = k_cache.shape
+    _require(k_cache, "k_cache", (B, Lcap, Hkv, D), torch.bfloat16)
+    _require(k_remote, "k_remote", (B, Lcap, Hkv, D), torch.float16)
+    st = lib().jetlong_remote_cache(_ptr(k_cache), _ptr(k_remote), B, Lcap, Hkv, D, int(j0),
+                                    int(j1), int(L), int(w_pretrained), float(rope_theta),
+                                    _stream_ptr(stream))
+    _check("jetlong_remote_cache", st)
+    return k_remote
+
+
+def jetlong_decode_two_form(q, k_cache, k_remote, v_cache, L: int, w_pretrained: int, w0: int,
+                            rope_theta: float, *, out=None, lse=None, out_dtype=torch.bfloat16,
+                            want_lse: bool = True, workspace=None, stream=None):
+    """jetlong_decode reading remote keys from the remote form of the cache
+    (written by jetlong_remote_cache for the G of this L).  Returns (out, lse)."""
+    if q.dim() != 3 or k_cache.dim() != 4:
+        raise ValueError("q must be [B, Hq, D] and the caches [B, Lcap, Hkv, D]")
+    B, Hq, D = q.shape
+    Lcap, Hkv = k_cache.shape[1], k_cache.shape[2]
+    _require(q, "q", (B, Hq, D), torch.bfloat16)
+    _require(k_cache, "k_cache", (B, Lcap, Hkv, D), torch.bfloat16)
+    _require(k_remote, "k_remote", (B, Lcap, Hkv, D), torch.float16)
+    _require(v_cache, "v_cache", (B, Lcap, Hkv, D), torch.bfloat16)
+    od = _out_dtype(out_dtype if out is None else out.dtype)
+    if out is None:
+        out = torch.empty((B, Hq, D), dtype=torch.bfloat16 if od == JL_BF16 else torch.float32,
+                          device=q.device)
+    _require(out, "out", (B, Hq, D), out.dtype)
+    if lse is None and want_lse:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    if lse is not None:
+        _require(lse, "lse", (B, Hq), torch.float32)
+    workspace, ws_bytes = _workspace(
+        workspace, jetlong_decode_workspace_size(B, Hq, Hkv, int(L), D), q.device)
+    st = lib().jetlong_decode_two_form(_ptr(q), _ptr(k_cache), _ptr(k_remote), _ptr(v_cache),
+                                       _ptr(out), _ptr(lse), B, Hq, Hkv, int(L), Lcap, D,
+                                       int(w_pretrained), int(w0), float(rope_theta), od,
+                                       _ptr(workspace), ws_bytes, _stream_ptr(stream))
+    _check("jetlong_decode_two_form", st)
     return out, lse
 
 
