@@ -107,11 +107,10 @@ JL_API const char *jetlong_version(void);
  * its only device-side storage is static (the error word and the
  * jetlong_decode_noalloc buffer).  Call it when no call of this library is
  * in flight on another thread.
- * Device resets: the library also caches, per process, the device address
- * of the jetlong_decode_noalloc buffer and which kernels already have their
- * shared-memory limit set.  A cudaDeviceReset invalidates both, so do not
- * call this library again in a process after resetting a device it has
- * used.
+ * It also forgets the device address of the jetlong_decode_noalloc buffer
+ * and which kernels already have their shared-memory limit set.  A
+ * cudaDeviceReset invalidates both: after one, call jetlong_shutdown before
+ * the next call of this library.
  */
 JL_API void jetlong_shutdown(void);
 

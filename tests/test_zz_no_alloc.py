@@ -72,3 +72,24 @@ def test_noalloc_rejects_sizes_beyond_its_buffer():
     lse = torch.zeros((w.B, w.Hq), dtype=torch.float32, device="cuda")
     assert _call_noalloc(w, w.L, q, kc, kc, out, lse) == jl.JL_ERR_WORKSPACE
     assert jl.jetlong_device_status() == jl.JL_OK
+
+
+def test_calls_after_shutdown_look_everything_up_again():
+    # jetlong_shutdown forgets the cached buffer address and kernel settings;
+    # the next calls find them again and give the same results
+    w = Workload("noalloc_shutdown", 1, 32, 8, 128, 5000, 1024, 256, 1e6, 79, False, kind="decode")
+    d = decode_inputs(w, device="cuda")
+    kc = torch.empty_like(d.k_raw)
+    jl.jetlong_rope_cache(d.k_raw, kc, 0, w.theta)
+    outs = []
+    for _ in range(2):
+        out = torch.full((w.B, w.Hq, w.D), float("nan"), device="cuda")
+        lse = torch.full((w.B, w.Hq), float("nan"), device="cuda")
+        assert _call_noalloc(w, w.L, d.q, kc, d.v, out, lse) == jl.JL_OK
+        ref = jl.jetlong_decode(d.q, kc, d.v, w.L, w.w_pretrained, w.w0, w.theta,
+                                out_dtype=torch.float32)
+        assert jl.jetlong_device_status() == jl.JL_OK
+        outs.append((out, lse, ref[0]))
+        jl.lib().jetlong_shutdown()
+    assert torch.equal(outs[0][0], outs[1][0]) and torch.equal(outs[0][1], outs[1][1])
+    assert torch.equal(outs[0][2], outs[1][2])

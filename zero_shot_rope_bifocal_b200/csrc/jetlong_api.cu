@@ -17,6 +17,10 @@ namespace jl {
 // device address; host code reaches it through cudaGetSymbolAddress.
 __device__ unsigned int g_device_error;
 
+std::atomic<unsigned> g_state_epoch{0};
+
+void reset_noalloc_cache();  // defined with the jetlong_decode_noalloc buffer below
+
 namespace {
 
 constexpr size_t kAlign = 256;
@@ -145,8 +149,12 @@ const char *jetlong_status_string(int s) {
 const char *jetlong_version(void) { return "0.1.0"; }
 
 void jetlong_shutdown(void) {
-  std::lock_guard<std::mutex> lk(g_mu);
-  for (DeviceState &st : g_dev) st = DeviceState{};
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    for (DeviceState &st : g_dev) st = DeviceState{};
+  }
+  reset_noalloc_cache();
+  g_state_epoch.fetch_add(1, std::memory_order_acq_rel);
 }
 
 int jetlong_group_size(int L, int w_pretrained) {
@@ -595,6 +603,12 @@ int noalloc_scratch(void **out) {
 }
 
 }  // namespace
+
+void reset_noalloc_cache() {
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  for (void *&p : g_noalloc_ptr) p = nullptr;
+}
+
 }  // namespace jl
 
 extern "C" int jetlong_decode_noalloc(const void *q, const void *k_cache, const void *v_cache,

@@ -13,12 +13,22 @@
 
 namespace jl {
 
+// Incremented by jetlong_shutdown: host-side caches made before it are stale.
+extern std::atomic<unsigned> g_state_epoch;
+
 // Sets a kernel's dynamic shared-memory limit once per device (bit `dev` of a
 // per-kernel mask), so later launches make no other CUDA call and can be
-// captured into a CUDA graph.
+// captured into a CUDA graph.  The mask is cleared when jetlong_shutdown has
+// run since it was filled (a device reset drops the attribute).
 template <auto Kernel>
 cudaError_t ensure_smem_limit(int bytes) {
   static std::atomic<unsigned long long> done{0};
+  static std::atomic<unsigned> seen_epoch{0};
+  const unsigned epoch = g_state_epoch.load(std::memory_order_acquire);
+  if (seen_epoch.load(std::memory_order_acquire) != epoch) {
+    done.store(0, std::memory_order_release);
+    seen_epoch.store(epoch, std::memory_order_release);
+  }
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return cudaGetLastError();
   const unsigned long long bit = 1ull << (dev & 63);
