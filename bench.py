@@ -50,15 +50,15 @@ DECODE_WORKLOAD = "decode_8b_128k"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # DRAM bytes (read + write) of one attention-kernel launch at the headline
 # workload, from an ncu capture (dram__bytes_read.sum + dram__bytes_write.sum)
-# of the kernel sources whose SHA-256 is recorded here; the capture and its
-# command are summarised in the profile named below.  The line reports it only
-# while the sources are unchanged, and null otherwise.
+# of the kernel's own sources (its device code and the PTX wrappers it uses),
+# whose SHA-256 is recorded here; the capture and its command are summarised
+# in the profile named below.  The line reports it only while those sources
+# are unchanged, and null otherwise.
 TRAFFIC_RECORD = {"bytes": 6.95e9, "read_bytes": 5.83e9, "write_bytes": 1.12e9,
-                  "sources_sha256": "141800bd62e5fd0e832ce8f7a10900aea6deca9288c007446025643f4de0c9e2",
+                  "sources_sha256": "22a4f68e1b66737134bea386b4dc50ec180e3785a9656bfcc02ee64cab6a10ba",
                   "profile": "profiles/prefill_attention_qwen3_8b_L131072_dram.md"}
 TRAFFIC_SOURCES = ("zero_shot_rope_bifocal_b200/csrc/prefill_sm100.cu",
-                   "zero_shot_rope_bifocal_b200/csrc/sm100_ptx.cuh",
-                   "zero_shot_rope_bifocal_b200/csrc/jl_common.cuh")
+                   "zero_shot_rope_bifocal_b200/csrc/sm100_ptx.cuh")
 NOMINAL = {"hbm_gbs": 8000.0, "bf16_tflops": 2250.0}
 
 
@@ -905,6 +905,7 @@ def run_native(args):
                 "decode_us_per_token": two_us_tok,
                 "achieved_gbs": decode_bytes(wd.B, wd.Hkv, wd.L, wd.D) / (two_us_tok * 1e-6) / 1e9,
                 "vs_rotating_decode": two_us_tok / us_tok,
+                "routing_cost_decode": two_us_tok / ctl_us_tok - 1.0,
                 "rebuild_ms_all_rows": rebuild_ms,
                 "rebuild_every_tokens": wd.w_pretrained},
             "e2e": {"value": e2e_val, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
