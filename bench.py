@@ -718,34 +718,42 @@ def run_native(args):
     if jl.jetlong_device_status() != jl.JL_OK:
         raise RuntimeError("device status not OK after the two-form decode")
 
-    # a 64-token prefill chunk appended at the end of the same 128K cache
-    n_chunk = 64
-    P0 = wd.L - n_chunk
-    cq = torch.randn((wd.B, n_chunk, wd.Hq, wd.D), device=dev).to(torch.bfloat16)
-    cout = torch.empty((wd.B, n_chunk, wd.Hq, wd.D), dtype=torch.bfloat16, device=dev)
-    clse = torch.empty((wd.B, wd.Hq, n_chunk), dtype=torch.float32, device=dev)
-    cws = torch.empty(jl.jetlong_prefill_chunk_workspace_size(wd.B, wd.Hq, wd.Hkv, P0, n_chunk,
-                                                              wd.D),
-                      dtype=torch.uint8, device=dev)
+    # prefill chunks of 16, 64 and 4096 tokens closing the same 128K cache
+    # (below 24 tokens the decode kernels run them, from 24 the prefill kernel)
+    chunks = []
+    for n_chunk in (16, 64, 4096):
+        P0 = wd.L - n_chunk
+        cq = torch.randn((wd.B, n_chunk, wd.Hq, wd.D), device=dev).to(torch.bfloat16)
+        cout = torch.empty((wd.B, n_chunk, wd.Hq, wd.D), dtype=torch.bfloat16, device=dev)
+        clse = torch.empty((wd.B, wd.Hq, n_chunk), dtype=torch.float32, device=dev)
+        cws = torch.empty(jl.jetlong_prefill_chunk_workspace_size(wd.B, wd.Hq, wd.Hkv, P0,
+                                                                  n_chunk, wd.D),
+                          dtype=torch.uint8, device=dev)
 
-    def cstep():
-        jl.jetlong_prefill_chunk(cq, kc, d.v, P0, wd.w_pretrained, wd.w0, wd.theta, out=cout,
-                                 lse=clse, workspace=cws, stream=stream)
+        def cstep():
+            jl.jetlong_prefill_chunk(cq, kc, d.v, P0, wd.w_pretrained, wd.w0, wd.theta,
+                                     out=cout, lse=clse, workspace=cws, stream=stream)
 
-    for _ in range(3):
-        cstep()
-    n_crep = 20
-    barrier()
-    torch.cuda.synchronize(dev)
-    ev0.record(stream)
-    for _ in range(n_crep):
-        cstep()
-    ev1.record(stream)
-    torch.cuda.synchronize(dev)
-    barrier()
-    chunk_ms = reduce_max(ev0.elapsed_time(ev1), world, dev) / n_crep
-    if jl.jetlong_device_status() != jl.JL_OK:
-        raise RuntimeError("device status not OK after the prefill chunk")
+        for _ in range(3):
+            cstep()
+        n_crep = 10
+        barrier()
+        torch.cuda.synchronize(dev)
+        ev0.record(stream)
+        for _ in range(n_crep):
+            cstep()
+        ev1.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier()
+        chunk_ms = reduce_max(ev0.elapsed_time(ev1), world, dev) / n_crep
+        if jl.jetlong_device_status() != jl.JL_OK:
+            raise RuntimeError("device status not OK after the prefill chunk")
+        pairs = n_chunk * P0 + n_chunk * (n_chunk + 1) // 2  # causal (query, key) pairs
+        chunks.append({"n": n_chunk, "P0": P0, "ms": chunk_ms,
+                       "us_per_query": 1e3 * chunk_ms / n_chunk,
+                       "path": "decode kernels" if n_chunk < 24 else "prefill kernel",
+                       "tflops": 4 * wd.B * wd.Hq * wd.D * pairs / (chunk_ms * 1e-3) / 1e12})
+        del cq, cout, clse, cws
 
     # ---- end to end through the public API from pinned host buffers
     hq = x.q.cpu().pin_memory()
@@ -869,13 +877,10 @@ def run_native(args):
                 "decode_us_per_token": ctl_us_tok,
                 "routing_cost_decode": us_tok / ctl_us_tok - 1.0},
             "prefill_chunk": {
-                "what": "64 queries at positions L-64..L-1 appended to the 128K cache "
-                        "(jetlong_prefill_chunk, one G from L), decode kernels over batch x query",
-                "ms": chunk_ms, "us_per_query": 1e3 * chunk_ms / n_chunk,
-                "kv_bytes_per_query": decode_bytes(wd.B, wd.Hkv, wd.L, wd.D),
-                "effective_gbs": n_chunk * decode_bytes(wd.B, wd.Hkv, wd.L, wd.D)
-                / (chunk_ms * 1e-3) / 1e9,
-                "note": "queries share the cache through L2, so effective_gbs can exceed HBM"},
+                "what": "chunks of n queries at positions L-n..L-1 closing the 128K cache "
+                        "(jetlong_prefill_chunk, one G from L); tflops counts 4.Hq.D per causal "
+                        "(query, key) pair",
+                "chunks": chunks},
             "three_pass": {
                 "what": "unfused inclusion-exclusion form: rotate + passes A (remote, causal), "
                         "B (true, band), C (remote, band) + merge kernel, same inputs",

@@ -214,8 +214,19 @@ JL_API int jetlong_prefill_three_pass(const void *q, const void *k, const void *
  * p = P0 + i and sees keys [0, p]: local keys (p - j <= w0) as cached,
  * older keys turned by the correction rotation R(f(j) - j) and scored
  * against RoPE(x_q, f(p)).  With P0 = 0 and n = L this equals jetlong_prefill
- * on the same data.  Runs on the split-KV decode kernels (a chunk is n
- * decode problems over one cache), so its cost grows with n * L.
+ * on the same data.  Two execution paths, chosen by n alone:
+ *   - n < 24: the split-KV decode kernels (a chunk is n decode problems over
+ *     one cache; cost grows with n * L);
+ *   - n >= 24: the tensor-core prefill kernel.  A pass first writes the
+ *     chunk's operands into the workspace (queries rotated to their true and
+ *     remote positions, and the cached keys of [0, P0 + n), as stored and
+ *     turned by R(f(j) - j), with the values, as FP16); 128-row query tiles
+ *     then run the same kernel as jetlong_prefill.  The cost is one pass over
+ *     the cache plus the tensor-core work of n * L pairs; the FP16 range
+ *     contract above applies to this path.
+ * jetlong_prefill_chunk_workspace_size returns the size the chosen path needs
+ * (for n >= 24, 2 x B.Hq.n.D + 3 x B.Hkv.(P0+n).D FP16 values, each array
+ * 256-byte aligned).
  *
  *   q       [B, n, Hq, D] BF16 pre-RoPE queries of the chunk (read)
  *   k_cache [B, Lcap, Hkv, D] BF16, RoPE at true positions, rows [0, P0+n)

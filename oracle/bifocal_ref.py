@@ -323,7 +323,8 @@ def decode(q, k_cache, v_cache, L: int, w_pretrained: int, w0: int, theta: float
 # --------------------------------------------------------------------------
 # Chunked prefill on the true-position cache (§3.1 schedule, §3.2 cache)
 # --------------------------------------------------------------------------
-def prefill_chunk(q, k_cache, v_cache, P0: int, w_pretrained: int, w0: int, theta: float):
+def prefill_chunk(q, k_cache, v_cache, P0: int, w_pretrained: int, w0: int, theta: float,
+                  rows=None):
     """A chunk of n new tokens at positions P0 .. P0+n-1 appended to a prompt.
 
     q: [B, n, Hq, D] pre-RoPE queries of the chunk.  k_cache / v_cache:
@@ -337,7 +338,8 @@ def prefill_chunk(q, k_cache, v_cache, P0: int, w_pretrained: int, w0: int, thet
       remote (p - j >  w0): s = RoPE(x_q, f(p)) . R(f(j) - j) k_cache[j]
 
     scaled by 1/sqrt(D).  Returns (o [B, n, Hq, D], lse [B, Hq, n]), float64.
-    With P0 = 0 and n = L this is the whole-prompt prefill.
+    With P0 = 0 and n = L this is the whole-prompt prefill.  ``rows`` (chunk
+    indices) restricts the work to those queries; the others stay zero.
     """
     q = np.asarray(q, dtype=np.float64)
     kc = np.asarray(k_cache)
@@ -359,7 +361,7 @@ def prefill_chunk(q, k_cache, v_cache, P0: int, w_pretrained: int, w0: int, thet
             v_all = vc[b, :L, g, :].astype(np.float64)
             c_corr_all = correction_rotate(c_all, jpos_all, G, theta)
             heads = np.arange(g * grp, (g + 1) * grp)
-            for i in range(n):
+            for i in (range(n) if rows is None else rows):
                 p = P0 + i
                 c, cc, vv = c_all[: p + 1], c_corr_all[: p + 1], v_all[: p + 1]
                 local = (p - jpos_all[: p + 1]) <= w0
@@ -602,14 +604,15 @@ def correction_rotate_interp(c, kpos, freq_interp, theta: float) -> np.ndarray:
 
 
 def prefill_chunk_interp(q, k_cache, v_cache, P0: int, w_pretrained: int, w0: int,
-                         theta: float, alpha: float = 1.0, beta: float = 32.0):
+                         theta: float, alpha: float = 1.0, beta: float = 32.0, rows=None):
     """Frequency-interpolation variant of ``prefill_chunk``: queries at P0 ..
     P0+n-1 on the true-position cache, one s from L = P0 + n.
 
       local  (p - j <= w0): s = RoPE(x_q, p) . k_cache[j]
       remote (p - j >  w0): s = RoPE'(x_q, p) . R(j (theta' - theta)) k_cache[j]
 
-    Returns (o [B, n, Hq, D], lse [B, Hq, n]) in float64.
+    Returns (o [B, n, Hq, D], lse [B, Hq, n]) in float64.  ``rows`` (chunk
+    indices) restricts the work to those queries; the others stay zero.
     """
     q = np.asarray(q, dtype=np.float64)
     kc = np.asarray(k_cache)
@@ -631,7 +634,7 @@ def prefill_chunk_interp(q, k_cache, v_cache, P0: int, w_pretrained: int, w0: in
             v_all = vc[b, :L, g, :].astype(np.float64)
             cc_all = correction_rotate_interp(c_all, jpos_all, fr, theta)
             heads = np.arange(g * grp, (g + 1) * grp)
-            for i in range(n):
+            for i in (range(n) if rows is None else rows):
                 p = P0 + i
                 local = (p - jpos_all[: p + 1]) <= w0
                 q_true = rope(q[b, i, heads], np.int64(p), theta)

@@ -70,3 +70,36 @@ def test_qwen3_8b_chunk_at_128k():
     out, lse, o_ref, lse_ref = run_chunk(w, 131072 - 64, 64, Lcap_extra=0)
     assert_o(f64(out), o_ref, "8B 128K chunk")
     assert_lse(f64(lse), lse_ref, "8B 128K chunk")
+
+
+def test_qwen3_8b_long_chunk_at_128k_sampled_rows():
+    # A 4096-token chunk closing a 128K prompt runs on the tensor-core prefill
+    # kernel (queries P0.., keys [0, P0 + n) of the cache); sampled queries
+    # against the oracle with the call's G (from P0 + n = 131072).
+    w = Workload("chunk_8b_long", 1, 32, 8, 128, 0, 32768, 4096, 1e6, 43, False, kind="decode")
+    n = 4096
+    P0 = 131072 - n
+    x = generation_inputs(w, P0, n)
+    cache = torch.from_numpy(oracle.rope_cache(f64(x.k_raw), 0, w.theta)).to(torch.bfloat16)
+    q = torch.randn((w.B, n, w.Hq, w.D), generator=torch.Generator().manual_seed(w.seed + 5))
+    q = q.to(torch.bfloat16)
+    out, lse = jl.jetlong_prefill_chunk(q.cuda(), cache.cuda(), x.v.cuda(), P0, w.w_pretrained,
+                                        w.w0, w.theta, out_dtype=torch.float32)
+    assert jl.jetlong_device_status() == jl.JL_OK
+    rows = [0, 1, 127, 128, 2048, n - 2, n - 1] + sorted(
+        torch.randint(2, n - 2, (3,), generator=torch.Generator().manual_seed(7)).tolist())
+    o_ref, lse_ref = oracle.prefill_chunk(f64(q), f64(cache), f64(x.v), P0, w.w_pretrained, w.w0,
+                                          w.theta, rows=rows)
+    assert_o(f64(out[:, rows]), o_ref[:, rows], "8B 128K long chunk")
+    assert_lse(f64(lse[:, :, rows]), lse_ref[:, :, rows], "8B 128K long chunk")
+    assert torch.isfinite(out).all() and torch.isfinite(lse).all()
+
+
+@pytest.mark.parametrize("n", [23, 24])
+def test_chunks_on_both_sides_of_the_path_threshold(n):
+    # 23 queries run on the decode kernels, 24 on the prefill kernel: the same
+    # cache, both against the oracle
+    w = Workload("chunk_thr", 1, 8, 2, 128, 0, 1024, 300, 1e6, 51, True, kind="decode")
+    out, lse, o_ref, lse_ref = run_chunk(w, 5000 - n, n)
+    assert_o(f64(out), o_ref, f"n={n}")
+    assert_lse(f64(lse), lse_ref, f"n={n}")

@@ -194,6 +194,20 @@ def test_chunk_tail_rows_are_the_prefill_rows(P0):
     np.testing.assert_allclose(lc, lse, atol=1e-10)
 
 
+def test_sampled_chunk_rows_are_the_prefill_rows():
+    w, q, k, v = tiny_inputs("tiny")
+    L = q.shape[1]
+    P0 = 200
+    rows = [0, 7, 150, L - P0 - 1]
+    cache = oracle.rope_cache(k, 0, w.theta)
+    oc, lc = oracle.prefill_chunk_interp(q[:, P0:], cache, v, P0, w.w_pretrained, w.w0, w.theta,
+                                         rows=rows)
+    o, lse = oracle.prefill_interp_rows(q, k, v, w.w_pretrained, w.w0, w.theta,
+                                        [P0 + i for i in rows])
+    np.testing.assert_allclose(oc[:, rows], o, atol=1e-10)
+    np.testing.assert_allclose(lc[:, :, rows], lse, atol=1e-10)
+
+
 @pytest.mark.parametrize("L", [129, 300, 512])
 def test_decode_equals_last_prefill_row(L):
     w, q, k, v = tiny_inputs("tiny")

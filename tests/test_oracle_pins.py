@@ -362,6 +362,24 @@ def test_chunk_tail_rows_are_the_prefill_rows(P0):
     np.testing.assert_allclose(lc, lse, atol=1e-10)
 
 
+def test_sampled_chunk_rows_are_the_prefill_rows():
+    # The rows option computes only the listed queries of a chunk, with the
+    # chunk's G (from P0 + n); each equals the direct rule's row, and the
+    # unlisted rows stay zero.
+    w, q, k, v = tiny_inputs("tiny")
+    L = q.shape[1]
+    P0 = 200
+    rows = [0, 5, 111, L - P0 - 1]
+    cache = oracle.rope_cache(k, 0, w.theta)
+    oc, lc = oracle.prefill_chunk(q[:, P0:], cache, v, P0, w.w_pretrained, w.w0, w.theta,
+                                  rows=rows)
+    o, lse = oracle.prefill_rows(q, k, v, w.w_pretrained, w.w0, w.theta, [P0 + i for i in rows])
+    np.testing.assert_allclose(oc[:, rows], o, atol=1e-10)
+    np.testing.assert_allclose(lc[:, :, rows], lse, atol=1e-10)
+    others = [i for i in range(L - P0) if i not in rows]
+    assert not oc[:, others].any() and not lc[:, :, others].any()
+
+
 def test_one_token_chunk_is_a_decode_step():
     w, q, k, v = tiny_inputs("tiny")
     cache = oracle.rope_cache(k, 0, w.theta)

@@ -227,6 +227,8 @@ int prepare_prefill(int stage, const void *q, const void *k, const void *v, void
   a->Hq = Hq;
   a->Hkv = Hkv;
   a->L = L;
+  a->q_off = 0;
+  a->Lq = L;
   a->D = D;
   a->w_pretrained = w_pretrained;
   a->w0 = w0;
@@ -430,6 +432,87 @@ int cache_attention(const void *q, const void *k_cache, const void *v_cache, voi
   return JL_OK;
 }
 
+// A chunk of at least this many queries runs on the tensor-core prefill
+// kernel (operands rotated once, then 128-row query tiles); shorter chunks run
+// on the decode kernels, one split-KV problem per query.
+#ifndef JL_CHUNK_TENSOR_MIN
+#define JL_CHUNK_TENSOR_MIN 24
+#endif
+constexpr int kChunkTensorMin = JL_CHUNK_TENSOR_MIN;
+
+// Workspace of the tensor-core chunk path: the FP16 operands, queries at
+// their true and remote positions [B, Hq, n, D], cached keys in both forms
+// and values [B, Hkv, P0 + n, D].
+size_t chunk_tensor_ws_bytes(int B, int Hq, int Hkv, int P0, int n, int D) {
+  const size_t q = align_up(static_cast<size_t>(B) * Hq * n * D * 2);
+  const size_t k = align_up(static_cast<size_t>(B) * Hkv * (static_cast<size_t>(P0) + n) * D * 2);
+  return 2 * q + 3 * k;
+}
+
+size_t chunk_ws_bytes(int B, int Hq, int Hkv, int P0, int n, int D) {
+  return n >= kChunkTensorMin ? chunk_tensor_ws_bytes(B, Hq, Hkv, P0, n, D)
+                              : decode_ws_bytes(B * n, Hq, Hkv, P0 + n, D);
+}
+
+// A prefill chunk on the tensor-core prefill kernel: the chunk's queries
+// (positions P0 .. P0 + n - 1) against keys [0, P0 + n) of the true-position
+// cache, with the same score rule and one G from P0 + n.
+int chunk_tensor(const void *q, const void *k_cache, const void *v_cache, void *out, float *lse,
+                 int B, int Hq, int Hkv, int P0, int n, int Lcap, int D, int w_pretrained,
+                 int w0, float rope_theta, int out_dtype, void *workspace,
+                 size_t workspace_bytes, jl_stream_t stream, int interp, float ramp_alpha,
+                 float ramp_beta) {
+  int L = 0;
+  int st = check_cache_call(q, k_cache, v_cache, out, lse, B, Hq, Hkv, n, P0, Lcap, D,
+                            w_pretrained, w0, rope_theta, out_dtype, interp, ramp_alpha,
+                            ramp_beta, nullptr, &L);
+  if (st != JL_OK) return st;
+  // grids: (query tiles, KV heads x head pairs, batch) and (positions, batch)
+  if (B > kMaxGridYZ || static_cast<long long>(Hkv) * ((Hq / Hkv + 1) / 2) > kMaxGridYZ)
+    return JL_ERR_SHAPE;
+  const size_t need = chunk_tensor_ws_bytes(B, Hq, Hkv, P0, n, D);
+  if (!workspace || workspace_bytes < need) return JL_ERR_WORKSPACE;
+  if (reinterpret_cast<uintptr_t>(workspace) % kAlign) return JL_ERR_ALIGN;
+  DeviceState *dev = nullptr;
+  if ((st = current_device(&dev)) != JL_OK) return st;
+
+  PrefillArgs a{};
+  a.q = static_cast<const __nv_bfloat16 *>(q);
+  a.out = out;
+  a.lse = lse;
+  a.out_f32 = out_dtype == JL_F32;
+  uint8_t *ws = static_cast<uint8_t *>(workspace);
+  const size_t qb = align_up(static_cast<size_t>(B) * Hq * n * D * 2);
+  const size_t kb = align_up(static_cast<size_t>(B) * Hkv * L * D * 2);
+  a.q_true = reinterpret_cast<__half *>(ws);
+  a.q_remote = reinterpret_cast<__half *>(ws + qb);
+  a.k_true = reinterpret_cast<__half *>(ws + 2 * qb);
+  a.k_remote = reinterpret_cast<__half *>(ws + 2 * qb + kb);
+  a.v_op = reinterpret_cast<__half *>(ws + 2 * qb + 2 * kb);
+  a.B = B;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.L = L;
+  a.D = D;
+  a.w_pretrained = w_pretrained;
+  a.w0 = w0;
+  a.G = group_size(L, w_pretrained);
+  a.theta = rope_theta;
+  a.q_off = P0;
+  a.Lq = n;
+  a.k_cache_in = static_cast<const __nv_bfloat16 *>(k_cache);
+  a.v_cache_in = static_cast<const __nv_bfloat16 *>(v_cache);
+  a.cache_cap = Lcap;
+  a.interp = interp;
+  a.ramp_alpha = ramp_alpha;
+  a.ramp_beta = ramp_beta;
+  a.dev_error = dev->err;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (launch_chunk_operands(a, s) != cudaSuccess) return JL_ERR_CUDA;
+  if (launch_prefill_attention(a, s) != cudaSuccess) return JL_ERR_CUDA;
+  return JL_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -448,13 +531,17 @@ size_t jetlong_prefill_chunk_workspace_size(int B, int Hq, int Hkv, int P0, int 
   if (n < 1 || P0 < 0 || static_cast<long long>(P0) + n > (1ll << 31) - 1) return 0;
   if (check_common(B, Hq, Hkv, P0 + n, D) != JL_OK) return 0;
   if (static_cast<long long>(B) * n > 65535) return 0;
-  return decode_ws_bytes(B * n, Hq, Hkv, P0 + n, D);
+  return chunk_ws_bytes(B, Hq, Hkv, P0, n, D);
 }
 
 int jetlong_prefill_chunk(const void *q, const void *k_cache, const void *v_cache, void *out,
                           float *lse, int B, int Hq, int Hkv, int P0, int n, int Lcap, int D,
                           int w_pretrained, int w0, float rope_theta, int out_dtype,
                           void *workspace, size_t workspace_bytes, jl_stream_t stream) {
+  if (n >= kChunkTensorMin)
+    return chunk_tensor(q, k_cache, v_cache, out, lse, B, Hq, Hkv, P0, n, Lcap, D, w_pretrained,
+                        w0, rope_theta, out_dtype, workspace, workspace_bytes, stream, 0, 0.f,
+                        0.f);
   return cache_attention(q, k_cache, v_cache, out, lse, B, Hq, Hkv, n, P0, Lcap, D,
                          w_pretrained, w0, rope_theta, out_dtype, workspace, workspace_bytes,
                          stream);
@@ -476,6 +563,10 @@ int jetlong_prefill_chunk_interp(const void *q, const void *k_cache, const void 
                                  int Lcap, int D, int w_pretrained, int w0, float rope_theta,
                                  float ramp_alpha, float ramp_beta, int out_dtype, void *workspace,
                                  size_t workspace_bytes, jl_stream_t stream) {
+  if (n >= kChunkTensorMin)
+    return chunk_tensor(q, k_cache, v_cache, out, lse, B, Hq, Hkv, P0, n, Lcap, D, w_pretrained,
+                        w0, rope_theta, out_dtype, workspace, workspace_bytes, stream, 1,
+                        ramp_alpha, ramp_beta);
   return cache_attention(q, k_cache, v_cache, out, lse, B, Hq, Hkv, n, P0, Lcap, D,
                          w_pretrained, w0, rope_theta, out_dtype, workspace, workspace_bytes,
                          stream, 1, ramp_alpha, ramp_beta);

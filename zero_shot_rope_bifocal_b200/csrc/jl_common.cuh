@@ -141,8 +141,15 @@ struct PrefillArgs {
   // MMA operands in the workspace, FP16 head-major [B, H, L, D]: queries and
   // keys rotated to true / remote positions, and the values
   __half *q_true, *q_remote, *k_true, *k_remote, *v_op;
-  // sizes and method parameters
+  // sizes and method parameters; L is the number of keys (positions
+  // [0, L)), the queries are positions [q_off, q_off + Lq) with
+  // q_off + Lq = L (a whole prompt: q_off = 0, Lq = L)
   int B, Hq, Hkv, L, D, w_pretrained, w0, G;
+  int q_off, Lq;
+  // keys and values from the true-position cache [B, cache_cap, Hkv, D]
+  // instead of pre-RoPE k and v (a chunk appended to a cache)
+  const __nv_bfloat16 *k_cache_in, *v_cache_in;
+  int cache_cap;
   float theta;
   int pass;  // PrefillPass
   // remote map: 0 = positions aliased by f (the method), 1 = frequency
@@ -154,6 +161,12 @@ struct PrefillArgs {
 
 // Rotates q and k into the four operand arrays (and the optional cache).
 cudaError_t launch_rope_qk(const PrefillArgs &a, cudaStream_t stream);
+
+// The operands of a chunk appended to a cache: the queries (positions
+// [q_off, L)) rotated to their true and remote positions, and the cached keys
+// and values of positions [0, L) as FP16 operands, the keys also in their
+// remote form (the correction rotation of §3.2 applied).
+cudaError_t launch_chunk_operands(const PrefillArgs &a, cudaStream_t stream);
 
 // The attention kernel proper (tcgen05 / TMEM / TMA).
 cudaError_t launch_prefill_attention(const PrefillArgs &a, cudaStream_t stream);

@@ -90,7 +90,9 @@ struct Layout {
 };
 
 struct Params {
-  int B, Hq, Hkv, L, G, w0eff, n_qt, grp, npair;
+  // query rows are positions [q_off, q_off + Lq) (a whole prompt: q_off = 0,
+  // Lq = L; a chunk appended to a cache: q_off = P0); keys are [0, q_off + Lq)
+  int B, Hq, Hkv, q_off, Lq, G, w0eff, n_qt, grp, npair;
   int pass;  // PrefillPass: the fused rule or one pass of the three-pass merge
   float scale_log2;
   void *out;
@@ -163,8 +165,8 @@ bifocal_prefill_kernel(const __grid_constant__ CUtensorMap tm_qt,
   const int b = blockIdx.z;
   const int head0 = g * prm.grp + 2 * pr;
   const bool has1 = 2 * pr + 1 < prm.grp;
-  const int p0 = qt * BM;
-  const int p1 = min(p0 + BM, prm.L) - 1;
+  const int p0 = prm.q_off + qt * BM;  // position of the tile's first row
+  const int p1 = min(p0 + BM, prm.q_off + prm.Lq) - 1;
   const int w0 = prm.w0eff;
 
   // Visit plan: remote visits of key tiles [kr0, kr0 + n_rem), then local
@@ -247,7 +249,7 @@ bifocal_prefill_kernel(const __grid_constant__ CUtensorMap tm_qt,
         mbar_arrive_expect_tx(bar(LY::kQFull + s), LY::TILE);
         for (int c = 0; c < NBOX; ++c)
           tma_load_3d(sb + LY::Q0 + s * LY::TILE + c * LY::BOX, remote ? &tm_qr : &tm_qt,
-                      bar(LY::kQFull + s), c * 64, p0, b * prm.Hq + head0 + s);
+                      bar(LY::kQFull + s), c * 64, qt * BM, b * prm.Hq + head0 + s);
       };
       load_q(0, n_rem > 0);
       if (has1) load_q(1, n_rem > 0);
@@ -386,7 +388,7 @@ bifocal_prefill_kernel(const __grid_constant__ CUtensorMap tm_qt,
     const int rloc = tid & (BM - 1);     // row inside the tile
     const int row = p0 + rloc;
     const bool active = s == 0 || has1;
-    const bool row_ok = active && row < prm.L;
+    const bool row_ok = active && row < prm.q_off + prm.Lq;
     const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
     float m_used = -INFINITY;  // reference max of this row (base 2)
     float l_sum = 0.f;         // running row sum, relative to m_used
@@ -401,11 +403,14 @@ bifocal_prefill_kernel(const __grid_constant__ CUtensorMap tm_qt,
       }
       tc_fence_after();
       const int k0 = kt * BN;  // key of column 0
-      bool whole;
-      if (remote)
-        whole = row_ok && (row - (k0 + BN - 1) >= dlo) && (row - k0 <= dhi);
-      else
-        whole = row_ok && (k0 + BN - 1 <= row) && (row - k0 <= w0);
+      // Rows past the last query (a partial tile) are never written; their
+      // scores are finite (their query rows were zero-filled), so they skip
+      // the mask like rows whose every pair is kept.
+      bool whole = !row_ok;
+      if (row_ok && remote)
+        whole = (row - (k0 + BN - 1) >= dlo) && (row - k0 <= dhi);
+      else if (row_ok)
+        whole = (k0 + BN - 1 <= row) && (row - k0 <= w0);
       // The row's raw scores (the scale is positive and applied later), one
       // TMEM read of all 128 columns, then the mask on edge tiles only.
       float x[BN];
@@ -499,7 +504,7 @@ bifocal_prefill_kernel(const __grid_constant__ CUtensorMap tm_qt,
       tc_fence_after();
       const float inv_l = row_ok ? 1.f / l_sum : 0.f;
       const int head = head0 + s;
-      const size_t obase = ((static_cast<size_t>(b) * prm.L + row) * prm.Hq + head) * D;
+      const size_t obase = ((static_cast<size_t>(b) * prm.Lq + qt * BM + rloc) * prm.Hq + head) * D;
 #pragma unroll 1
       for (int c = 0; c < D / 32; ++c) {
         uint32_t rr[32];
@@ -530,7 +535,7 @@ bifocal_prefill_kernel(const __grid_constant__ CUtensorMap tm_qt,
         }
       }
       if (row_ok && prm.lse)
-        prm.lse[(static_cast<size_t>(b) * prm.Hq + head) * prm.L + row] =
+        prm.lse[(static_cast<size_t>(b) * prm.Hq + head) * prm.Lq + qt * BM + rloc] =
             (m_used + log2f(l_sum)) * 0.69314718055994531f;
     }
   }
@@ -578,8 +583,8 @@ cudaError_t launch_d(const PrefillArgs &a, cudaStream_t stream) {
   if (!encode_fn()) return cudaErrorNotSupported;
   CUtensorMap tqt, tqr, tkt, tkr, tv;
   const bool two = a.G > 1;
-  if (!encode_head_major(&tqt, a.q_true, a.B * a.Hq, a.L, D) ||
-      !encode_head_major(&tqr, two ? a.q_remote : a.q_true, a.B * a.Hq, a.L, D) ||
+  if (!encode_head_major(&tqt, a.q_true, a.B * a.Hq, a.Lq, D) ||
+      !encode_head_major(&tqr, two ? a.q_remote : a.q_true, a.B * a.Hq, a.Lq, D) ||
       !encode_head_major(&tkt, a.k_true, a.B * a.Hkv, a.L, D) ||
       !encode_head_major(&tkr, two ? a.k_remote : a.k_true, a.B * a.Hkv, a.L, D) ||
       !encode_head_major(&tv, a.v_op, a.B * a.Hkv, a.L, D))
@@ -588,13 +593,14 @@ cudaError_t launch_d(const PrefillArgs &a, cudaStream_t stream) {
   prm.B = a.B;
   prm.Hq = a.Hq;
   prm.Hkv = a.Hkv;
-  prm.L = a.L;
+  prm.q_off = a.q_off;
+  prm.Lq = a.Lq;
   prm.G = a.G;
   // The fused rule with G = 1 is plain causal attention; a pass of the
   // three-pass merge keeps its band whatever G is.
   prm.w0eff = (a.G == 1 && a.pass == kPassFused) ? INT_MAX : a.w0;
   prm.pass = a.pass;
-  prm.n_qt = (a.L + BM - 1) / BM;
+  prm.n_qt = (a.Lq + BM - 1) / BM;
   prm.grp = a.Hq / a.Hkv;
   prm.npair = (prm.grp + 1) / 2;
   prm.scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(D));

@@ -21,6 +21,11 @@
 // With the frequency-interpolation remote map (the §4.7 ablation) the remote
 // arrays hold RoPE'(x, i): true position, interpolated frequencies theta'_t.
 //
+// Chunk operands (a chunk of queries appended to a cache, §3.1, §3.2): the
+// queries as above at their positions P0 + t, and the keys and values read
+// from the true-position cache; the remote keys are the cached ones turned by
+// the correction rotation R(f(j) - j).
+//
 // Cache writer (§3.2): k_cache[b, pos0 + t] = RoPE(k[b, t], pos0 + t).
 //
 // Each CTA forms the frequencies once, evaluates cos/sin once per (position,
@@ -144,6 +149,117 @@ rope_qk_kernel(PrefillArgs a) {
   if (!in_range) atomicOr(a.dev_error, kDevRange);
 }
 
+// Chunk operands, queries: for t < Lq, position pos = q_off + t,
+//   q_true[b,h,t] = RoPE(x_q[b,t,h], pos),  q_remote[b,h,t] = RoPE(x_q[b,t,h], f(pos))
+// (RoPE'(x_q, pos) under the frequency-interpolation map), FP16 head-major
+// [B, Hq, Lq, D]; G and the interpolation factor come from L = q_off + Lq.
+__global__ void __launch_bounds__(kRopeThreads)
+chunk_q_kernel(PrefillArgs a) {
+  extern __shared__ float2 cs_smem[];  // [2][kPosPerCta][D/2] (cos, sin), then 2 x [D/2] freq
+  const int half = a.D / 2;
+  const int b = blockIdx.y;
+  const int t_begin = blockIdx.x * kPosPerCta;
+  const int npos = min(kPosPerCta, a.Lq - t_begin);
+  const bool two = a.G > 1;
+  float2 *cs_true = cs_smem;
+  float2 *cs_remote = cs_smem + kPosPerCta * half;
+  double *freq = reinterpret_cast<double *>(cs_smem + 2 * kPosPerCta * half);
+  double *freq_remote = freq + half;
+  const double theta = static_cast<double>(a.theta);
+  for (int i = threadIdx.x; i < half; i += blockDim.x) {
+    const double f = rope_freq(i, a.D, theta);
+    freq[i] = f;
+    freq_remote[i] =
+        a.interp ? f * interp_factor(f, a.L, a.w_pretrained, a.ramp_alpha, a.ramp_beta) : f;
+  }
+  __syncthreads();
+  for (int idx = threadIdx.x; idx < npos * half * (two ? 2 : 1); idx += blockDim.x) {
+    const int var = idx / (npos * half);
+    const int rem = idx - var * npos * half;
+    const int t = rem / half, i = rem - t * half;
+    const int pos = a.q_off + t_begin + t;
+    const long long ppos = (var == 0 || a.interp) ? pos : remap(pos, a.G);
+    float c, s;
+    rope_cos_sin(ppos, var == 0 ? freq[i] : freq_remote[i], c, s);
+    (var == 0 ? cs_true : cs_remote)[t * half + i] = make_float2(c, s);
+  }
+  __syncthreads();
+  bool in_range = true;
+  const int quarter = a.D / 4;
+  for (int idx = threadIdx.x; idx < npos * a.Hq * quarter; idx += blockDim.x) {
+    const int t = idx / (a.Hq * quarter);
+    const int rem = idx - t * a.Hq * quarter;
+    const int h = rem / quarter;
+    const int i = (rem - h * quarter) * 2;
+    const __nv_bfloat16 *src =
+        a.q + ((static_cast<size_t>(b) * a.Lq + t_begin + t) * a.Hq + h) * a.D;
+    const size_t drow = ((static_cast<size_t>(b) * a.Hq + h) * a.Lq + t_begin + t) * a.D;
+    in_range &= store_f16(a.q_true + drow, i, half,
+                          rotate2(src, i, half, cs_true[t * half + i], cs_true[t * half + i + 1]));
+    if (two)
+      in_range &= store_f16(a.q_remote + drow, i, half,
+                            rotate2(src, i, half, cs_remote[t * half + i],
+                                    cs_remote[t * half + i + 1]));
+  }
+  if (!in_range) atomicOr(a.dev_error, kDevRange);
+}
+
+// Chunk operands, keys and values from the true-position cache (§3.2): for
+// j < L,
+//   k_true[b,g,j] = k_cache[b,j,g],  k_remote[b,g,j] = R(f(j) - j) k_cache[b,j,g],
+//   v_op[b,g,j] = v_cache[b,j,g],
+// FP16 head-major [B, Hkv, L, D].  R(Delta) turns channel pair (i, i + D/2) by
+// Delta * theta_i; under the frequency-interpolation map the remote form is
+// RoPE'(x_k, j), i.e. the cached key turned by j * (theta'_i - theta_i).
+__global__ void __launch_bounds__(kRopeThreads)
+cache_kv_kernel(PrefillArgs a) {
+  extern __shared__ float2 cs_smem[];  // [kPosPerCta][D/2] (cos, sin), then [D/2] freq
+  const int half = a.D / 2;
+  const int b = blockIdx.y;
+  const int j_begin = blockIdx.x * kPosPerCta;
+  const int npos = min(kPosPerCta, a.L - j_begin);
+  const bool two = a.G > 1;
+  double *freq = reinterpret_cast<double *>(cs_smem + kPosPerCta * half);
+  const double theta = static_cast<double>(a.theta);
+  for (int i = threadIdx.x; i < half; i += blockDim.x) {
+    const double f = rope_freq(i, a.D, theta);
+    // the correction's angle per unit of Delta: theta_i, or theta'_i - theta_i
+    freq[i] = a.interp ? f * (interp_factor(f, a.L, a.w_pretrained, a.ramp_alpha, a.ramp_beta) - 1.0)
+                       : f;
+  }
+  __syncthreads();
+  if (two) {
+    for (int idx = threadIdx.x; idx < npos * half; idx += blockDim.x) {
+      const int t = idx / half, i = idx - t * half;
+      const int j = j_begin + t;
+      const long long delta = a.interp ? j : static_cast<long long>(remap(j, a.G)) - j;
+      float c, s;
+      rope_cos_sin(delta, freq[i], c, s);
+      cs_smem[t * half + i] = make_float2(c, s);
+    }
+  }
+  __syncthreads();
+  bool in_range = true;
+  const int quarter = a.D / 4;
+  const float2 one = make_float2(1.f, 0.f);
+  for (int idx = threadIdx.x; idx < npos * a.Hkv * quarter; idx += blockDim.x) {
+    const int t = idx / (a.Hkv * quarter);
+    const int rem = idx - t * a.Hkv * quarter;
+    const int g = rem / quarter;
+    const int i = (rem - g * quarter) * 2;
+    const int j = j_begin + t;
+    const size_t srow = ((static_cast<size_t>(b) * a.cache_cap + j) * a.Hkv + g) * a.D;
+    const size_t drow = ((static_cast<size_t>(b) * a.Hkv + g) * a.L + j) * a.D;
+    const __nv_bfloat16 *kc = a.k_cache_in + srow;
+    in_range &= store_f16(a.k_true + drow, i, half, rotate2(kc, i, half, one, one));
+    if (two)
+      in_range &= store_f16(a.k_remote + drow, i, half,
+                            rotate2(kc, i, half, cs_smem[t * half + i], cs_smem[t * half + i + 1]));
+    in_range &= store_f16(a.v_op + drow, i, half, rotate2(a.v_cache_in + srow, i, half, one, one));
+  }
+  if (!in_range) atomicOr(a.dev_error, kDevRange);
+}
+
 __global__ void __launch_bounds__(kRopeThreads)
 rope_cache_kernel(const __nv_bfloat16 *__restrict__ k, __nv_bfloat16 *__restrict__ k_cache, int n,
                   int Hkv, int D, int pos0, int Lcap, float theta_f) {
@@ -182,6 +298,16 @@ cudaError_t launch_rope_qk(const PrefillArgs &a, cudaStream_t stream) {
   const dim3 grid((a.L + kPosPerCta - 1) / kPosPerCta, a.B);
   const size_t smem = 2 * kPosPerCta * (a.D / 2) * sizeof(float2) + 2 * (a.D / 2) * sizeof(double);
   rope_qk_kernel<<<grid, kRopeThreads, smem, stream>>>(a);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_chunk_operands(const PrefillArgs &a, cudaStream_t stream) {
+  const size_t smem_q = 2 * kPosPerCta * (a.D / 2) * sizeof(float2) + 2 * (a.D / 2) * sizeof(double);
+  chunk_q_kernel<<<dim3((a.Lq + kPosPerCta - 1) / kPosPerCta, a.B), kRopeThreads, smem_q, stream>>>(a);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const size_t smem_k = kPosPerCta * (a.D / 2) * sizeof(float2) + (a.D / 2) * sizeof(double);
+  cache_kv_kernel<<<dim3((a.L + kPosPerCta - 1) / kPosPerCta, a.B), kRopeThreads, smem_k, stream>>>(a);
   return cudaGetLastError();
 }
 
