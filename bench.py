@@ -343,10 +343,11 @@ def sweep_prefill(jl, torch, dev, stream, name: str, w0: int | None = None, reps
     flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
 
     def rotate():
-        jl.jetlong_prefill_rotate(x.q, x.k, x.v, w.w_pretrained, w.theta, ws, stream=stream)
+        jl.jetlong_prefill_rotate(x.k, x.v, w.w_pretrained, w.theta, ws, stream=stream)
 
     def attend():
-        jl.jetlong_prefill_attend(out, lse, Hkv, w.w_pretrained, w.w0, ws, stream=stream)
+        jl.jetlong_prefill_attend(x.q, out, lse, Hkv, w.w_pretrained, w.w0, w.theta, ws,
+                                  stream=stream)
 
     for _ in range(2):
         rotate()
@@ -457,10 +458,11 @@ def run_native(args):
     stream = torch.cuda.current_stream(dev)
 
     def step(ev_mid=None, ev_end=None):
-        jl.jetlong_prefill_rotate(x.q, x.k, x.v, w.w_pretrained, w.theta, ws, stream=stream)
+        jl.jetlong_prefill_rotate(x.k, x.v, w.w_pretrained, w.theta, ws, stream=stream)
         if ev_mid is not None:
             ev_mid.record(stream)
-        jl.jetlong_prefill_attend(out, lse, Hkv, w.w_pretrained, w.w0, ws, stream=stream)
+        jl.jetlong_prefill_attend(x.q, out, lse, Hkv, w.w_pretrained, w.w0, w.theta, ws,
+                                  stream=stream)
         if ev_end is not None:
             ev_end.record(stream)
 
@@ -496,10 +498,10 @@ def run_native(args):
     # (w_pretrained = L, so G = 1: plain causal RoPE at true positions), on the
     # same inputs; it prices the routing (remote visits, edge tiles, rotation).
     def ctl_step(ev_mid=None, ev_end=None):
-        jl.jetlong_prefill_rotate(x.q, x.k, x.v, L, w.theta, ws, stream=stream)
+        jl.jetlong_prefill_rotate(x.k, x.v, L, w.theta, ws, stream=stream)
         if ev_mid is not None:
             ev_mid.record(stream)
-        jl.jetlong_prefill_attend(out, lse, Hkv, L, w.w0, ws, stream=stream)
+        jl.jetlong_prefill_attend(x.q, out, lse, Hkv, L, w.w0, w.theta, ws, stream=stream)
         if ev_end is not None:
             ev_end.record(stream)
 

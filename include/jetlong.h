@@ -160,24 +160,27 @@ JL_API int jetlong_prefill(const void *q, const void *k, const void *v, void *ou
  * several times).  jetlong_prefill == jetlong_prefill_rotate followed by
  * jetlong_prefill_attend on the same workspace and stream.
  *
- * jetlong_prefill_rotate: RoPE in the Q/K load path.  Reads q, k, v (layouts
- *   as for jetlong_prefill) and writes the tensor-core operands into the
- *   workspace: queries and keys rotated to true positions i, j and, when
- *   G > 1, to remote positions f(i), f(j), plus the values, all FP16
- *   head-major; if k_cache_out is not NULL it also writes the BF16
- *   true-position cache rows [0, L) (§3.2).
- * jetlong_prefill_attend: the attention kernel.  Reads the operands a
- *   preceding jetlong_prefill_rotate with the same B, Hq, Hkv, L, D,
- *   w_pretrained left in `workspace`; writes out and lse (lse may be NULL).
+ * jetlong_prefill_rotate: the key side of RoPE.  Reads k and v (layouts as
+ *   for jetlong_prefill) and writes the key operands into the workspace: keys
+ *   rotated to true positions j and, when G > 1, to remote positions f(j),
+ *   plus the values, all FP16 head-major [B, Hkv, L, D]; if k_cache_out is
+ *   not NULL it also writes the BF16 true-position cache rows [0, L) (§3.2).
+ * jetlong_prefill_attend: the attention kernel.  Reads q (pre-RoPE, layout as
+ *   for jetlong_prefill: its query side of RoPE runs in the kernel's load
+ *   path, rotating each query row to f(i) and to i as the tile is staged)
+ *   and the operands a preceding jetlong_prefill_rotate with the same B, Hkv,
+ *   L, D, w_pretrained and rope_theta left in `workspace`; writes out and lse
+ *   (lse may be NULL).
  */
-JL_API int jetlong_prefill_rotate(const void *q, const void *k, const void *v, int B, int Hq,
-                                  int Hkv, int L, int D, int w_pretrained, float rope_theta,
-                                  void *k_cache_out, int k_cache_capacity, void *workspace,
-                                  size_t workspace_bytes, jl_stream_t stream);
+JL_API int jetlong_prefill_rotate(const void *k, const void *v, int B, int Hkv, int L, int D,
+                                  int w_pretrained, float rope_theta, void *k_cache_out,
+                                  int k_cache_capacity, void *workspace, size_t workspace_bytes,
+                                  jl_stream_t stream);
 
-JL_API int jetlong_prefill_attend(void *out, float *lse, int B, int Hq, int Hkv, int L, int D,
-                                  int w_pretrained, int w0, int out_dtype, const void *workspace,
-                                  size_t workspace_bytes, jl_stream_t stream);
+JL_API int jetlong_prefill_attend(const void *q, void *out, float *lse, int B, int Hq, int Hkv,
+                                  int L, int D, int w_pretrained, int w0, float rope_theta,
+                                  int out_dtype, const void *workspace, size_t workspace_bytes,
+                                  jl_stream_t stream);
 
 /*
  * The unfused three-pass form of the same result (Jet-Long paper, §3.3

@@ -56,7 +56,7 @@ def test_group_size_agrees_with_oracle(lib):
 
 def test_workspace_sizes(lib):
     n = jl.jetlong_prefill_workspace_size(1, 32, 8, 131072, 128)
-    assert n >= 2 * (2 * 32 + 3 * 8) * 131072 * 128
+    assert n >= 2 * 3 * 8 * 131072 * 128
     assert jl.jetlong_prefill_workspace_size(1, 3, 2, 100, 128) == 0  # Hq % Hkv != 0
     assert jl.jetlong_prefill_workspace_size(1, 2, 1, 100, 96) == 0   # unsupported D
     prev = 0
@@ -225,18 +225,30 @@ def test_rope_cache_rejects_bad_arguments(lib, args, status):
 
 
 def test_stage_entry_points_check_their_own_buffers(lib):
-    # rotate needs q, k, v; attend needs out; neither accepts a short workspace
-    rot = lambda q=P, k=P, v=P, ws=P, wsb=1 << 40: lib.jetlong_prefill_rotate(
-        q, k, v, 1, 2, 1, 512, 64, 128, 1e4, None, 0, ws, wsb, None)
-    att = lambda out=P, lse=None, ws=P, wsb=1 << 40: lib.jetlong_prefill_attend(
-        out, lse, 1, 2, 1, 512, 64, 128, 32, 0, ws, wsb, None)
+    # rotate needs k, v; attend needs q (rotated in its load path) and out;
+    # neither accepts a short workspace
+    rot = lambda k=P, v=P, ws=P, wsb=1 << 40: lib.jetlong_prefill_rotate(
+        k, v, 1, 1, 512, 64, 128, 1e4, None, 0, ws, wsb, None)
+    att = lambda q=P, out=P, lse=None, ws=P, wsb=1 << 40: lib.jetlong_prefill_attend(
+        q, out, lse, 1, 2, 1, 512, 64, 128, 32, 1e4, 0, ws, wsb, None)
     assert rot(v=None) == jl.JL_ERR_NULL
     assert rot(k=None) == jl.JL_ERR_NULL
     assert rot(v=ctypes.c_void_p(264)) == jl.JL_ERR_ALIGN
     assert rot(wsb=100) == jl.JL_ERR_WORKSPACE
+    assert att(q=None) == jl.JL_ERR_NULL
     assert att(out=None) == jl.JL_ERR_NULL
+    assert att(q=ctypes.c_void_p(264)) == jl.JL_ERR_ALIGN
     assert att(lse=ctypes.c_void_p(260)) == jl.JL_ERR_ALIGN
     assert att(ws=None) == jl.JL_ERR_WORKSPACE
+
+
+def test_prefill_workspace_holds_only_the_key_operands():
+    # the queries are rotated in the attention kernel's load path, so the
+    # workspace holds k_true, k_remote and v: 3 x B.Hkv.L.D FP16 values
+    for B, Hq, Hkv, L, D in ((1, 32, 8, 131072, 128), (2, 4, 2, 1000, 64)):
+        n = jl.jetlong_prefill_workspace_size(B, Hq, Hkv, L, D)
+        one = -(-(B * Hkv * L * D * 2) // 256) * 256
+        assert n == 3 * one
 
 
 # ---------------------------------------------------------------- frequency-interpolation map

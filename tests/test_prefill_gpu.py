@@ -154,8 +154,8 @@ def test_staged_calls_equal_the_fused_call():
                      dtype=torch.uint8, device="cuda")
     out2 = torch.empty_like(out1)
     lse2 = torch.empty_like(lse1)
-    jl.jetlong_prefill_rotate(q, k, v, w.w_pretrained, w.theta, ws)
-    jl.jetlong_prefill_attend(out2, lse2, w.Hkv, w.w_pretrained, w.w0, ws)
+    jl.jetlong_prefill_rotate(k, v, w.w_pretrained, w.theta, ws)
+    jl.jetlong_prefill_attend(q, out2, lse2, w.Hkv, w.w_pretrained, w.w0, w.theta, ws)
     assert jl.jetlong_device_status() == jl.JL_OK
     assert torch.equal(out1, out2) and torch.equal(lse1, lse2)
 

@@ -103,10 +103,11 @@ int check_ramp(float alpha, float beta) {
   return JL_OK;
 }
 
-size_t prefill_ws_bytes(int B, int Hq, int Hkv, int L, int D) {
-  const size_t q = static_cast<size_t>(B) * Hq * L * D * 2;
+// The key operands of a prefill: k_true, k_remote, v (FP16 [B, Hkv, L, D]).
+// The queries need none: the attention kernel rotates them as it loads them.
+size_t prefill_ws_bytes(int B, int /*Hq*/, int Hkv, int L, int D) {
   const size_t k = static_cast<size_t>(B) * Hkv * L * D * 2;
-  return 2 * align_up(q) + 3 * align_up(k);  // q_true, q_remote, k_true, k_remote, v
+  return 3 * align_up(k);
 }
 
 // Three-pass workspace: the prefill operands, then O_A, O_B, O_C (fp32
@@ -183,8 +184,8 @@ int prepare_prefill(int stage, const void *q, const void *k, const void *v, void
                     void *workspace, size_t workspace_bytes, PrefillArgs *a,
                     bool three_pass = false) {
   const bool rot = stage & kStageRotate, att = stage & kStageAttend;
-  if (rot && (!q || !k || !v)) return JL_ERR_NULL;
-  if (att && !out) return JL_ERR_NULL;
+  if (rot && (!k || !v)) return JL_ERR_NULL;
+  if (att && (!q || !out)) return JL_ERR_NULL;
   int st = check_common(B, Hq, Hkv, L, D);
   if (st != JL_OK) return st;
   // grids: (positions, batch) for the operand pass, (query tiles, KV heads x
@@ -194,10 +195,9 @@ int prepare_prefill(int stage, const void *q, const void *k, const void *v, void
   if ((st = check_method(w_pretrained, w0, rope_theta)) != JL_OK) return st;
   if (att && out_dtype != JL_BF16 && out_dtype != JL_F32) return JL_ERR_UNSUPPORTED;
   if (rot && k_cache_out && k_cache_capacity < L) return JL_ERR_SHAPE;
-  if (rot && (!aligned16(q) || !aligned16(k) || !aligned16(v) ||
-              (k_cache_out && !aligned16(k_cache_out))))
+  if (rot && (!aligned16(k) || !aligned16(v) || (k_cache_out && !aligned16(k_cache_out))))
     return JL_ERR_ALIGN;
-  if (att && (!aligned16(out) || (lse && !aligned16(lse)))) return JL_ERR_ALIGN;
+  if (att && (!aligned16(q) || !aligned16(out) || (lse && !aligned16(lse)))) return JL_ERR_ALIGN;
   const size_t need = three_pass ? three_pass_ws_bytes(B, Hq, Hkv, L, D)
                                  : prefill_ws_bytes(B, Hq, Hkv, L, D);
   if (!workspace || workspace_bytes < need) return JL_ERR_WORKSPACE;
@@ -207,7 +207,7 @@ int prepare_prefill(int stage, const void *q, const void *k, const void *v, void
   if ((st = current_device(&dev)) != JL_OK) return st;
 
   *a = PrefillArgs{};
-  a->q = rot ? static_cast<const __nv_bfloat16 *>(q) : nullptr;
+  a->q = att ? static_cast<const __nv_bfloat16 *>(q) : nullptr;
   a->k = rot ? static_cast<const __nv_bfloat16 *>(k) : nullptr;
   a->v = rot ? static_cast<const __nv_bfloat16 *>(v) : nullptr;
   a->out = att ? out : nullptr;
@@ -216,13 +216,10 @@ int prepare_prefill(int stage, const void *q, const void *k, const void *v, void
   a->k_cache_out = rot ? static_cast<__nv_bfloat16 *>(k_cache_out) : nullptr;
   a->k_cache_capacity = a->k_cache_out ? k_cache_capacity : 0;
   uint8_t *ws = static_cast<uint8_t *>(workspace);
-  const size_t qb = align_up(static_cast<size_t>(B) * Hq * L * D * 2);
   const size_t kb = align_up(static_cast<size_t>(B) * Hkv * L * D * 2);
-  a->q_true = reinterpret_cast<__half *>(ws);
-  a->q_remote = reinterpret_cast<__half *>(ws + qb);
-  a->k_true = reinterpret_cast<__half *>(ws + 2 * qb);
-  a->k_remote = reinterpret_cast<__half *>(ws + 2 * qb + kb);
-  a->v_op = reinterpret_cast<__half *>(ws + 2 * qb + 2 * kb);
+  a->k_true = reinterpret_cast<__half *>(ws);
+  a->k_remote = reinterpret_cast<__half *>(ws + kb);
+  a->v_op = reinterpret_cast<__half *>(ws + 2 * kb);
   a->B = B;
   a->Hq = Hq;
   a->Hkv = Hkv;
@@ -252,7 +249,7 @@ int jetlong_prefill(const void *q, const void *k, const void *v, void *out, floa
                                  workspace, workspace_bytes, &a);
   if (st != JL_OK) return st;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (launch_rope_qk(a, s) != cudaSuccess) return JL_ERR_CUDA;
+  if (launch_rope_kv(a, s) != cudaSuccess) return JL_ERR_CUDA;
   if (launch_prefill_attention(a, s) != cudaSuccess) return JL_ERR_CUDA;
   return JL_OK;
 }
@@ -272,30 +269,30 @@ int jetlong_prefill_interp(const void *q, const void *k, const void *v, void *ou
   a.ramp_alpha = ramp_alpha;
   a.ramp_beta = ramp_beta;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (launch_rope_qk(a, s) != cudaSuccess) return JL_ERR_CUDA;
+  if (launch_rope_kv(a, s) != cudaSuccess) return JL_ERR_CUDA;
   if (launch_prefill_attention(a, s) != cudaSuccess) return JL_ERR_CUDA;
   return JL_OK;
 }
 
-int jetlong_prefill_rotate(const void *q, const void *k, const void *v, int B, int Hq, int Hkv,
-                           int L, int D, int w_pretrained, float rope_theta, void *k_cache_out,
+int jetlong_prefill_rotate(const void *k, const void *v, int B, int Hkv, int L, int D,
+                           int w_pretrained, float rope_theta, void *k_cache_out,
                            int k_cache_capacity, void *workspace, size_t workspace_bytes,
                            jl_stream_t stream) {
   PrefillArgs a;
-  const int st = prepare_prefill(kStageRotate, q, k, v, nullptr, nullptr, B, Hq, Hkv, L, D,
+  const int st = prepare_prefill(kStageRotate, nullptr, k, v, nullptr, nullptr, B, Hkv, Hkv, L, D,
                                  w_pretrained, 0, rope_theta, JL_BF16, k_cache_out,
                                  k_cache_capacity, workspace, workspace_bytes, &a);
   if (st != JL_OK) return st;
-  if (launch_rope_qk(a, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return JL_ERR_CUDA;
+  if (launch_rope_kv(a, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return JL_ERR_CUDA;
   return JL_OK;
 }
 
-int jetlong_prefill_attend(void *out, float *lse, int B, int Hq, int Hkv, int L, int D,
-                           int w_pretrained, int w0, int out_dtype, const void *workspace,
-                           size_t workspace_bytes, jl_stream_t stream) {
+int jetlong_prefill_attend(const void *q, void *out, float *lse, int B, int Hq, int Hkv, int L,
+                           int D, int w_pretrained, int w0, float rope_theta, int out_dtype,
+                           const void *workspace, size_t workspace_bytes, jl_stream_t stream) {
   PrefillArgs a;
-  const int st = prepare_prefill(kStageAttend, nullptr, nullptr, nullptr, out, lse, B, Hq, Hkv, L,
-                                 D, w_pretrained, w0, 1.0f, out_dtype, nullptr, 0,
+  const int st = prepare_prefill(kStageAttend, q, nullptr, nullptr, out, lse, B, Hq, Hkv, L, D,
+                                 w_pretrained, w0, rope_theta, out_dtype, nullptr, 0,
                                  const_cast<void *>(workspace), workspace_bytes, &a);
   if (st != JL_OK) return st;
   if (launch_prefill_attention(a, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
@@ -326,7 +323,7 @@ int jetlong_prefill_three_pass(const void *q, const void *k, const void *v, void
     o_pass[i] = reinterpret_cast<float *>(ws + i * ob);
     l_pass[i] = reinterpret_cast<float *>(ws + 3 * ob + i * lb);
   }
-  if (launch_rope_qk(a, s) != cudaSuccess) return JL_ERR_CUDA;
+  if (launch_rope_kv(a, s) != cudaSuccess) return JL_ERR_CUDA;
   const PrefillPass passes[3] = {kPassRemoteCausal, kPassLocalBand, kPassRemoteBand};
   for (int i = 0; i < 3; ++i) {
     PrefillArgs p = a;
@@ -440,17 +437,16 @@ int cache_attention(const void *q, const void *k_cache, const void *v_cache, voi
 #endif
 constexpr int kChunkTensorMin = JL_CHUNK_TENSOR_MIN;
 
-// Workspace of the tensor-core chunk path: the FP16 operands, queries at
-// their true and remote positions [B, Hq, n, D], cached keys in both forms
-// and values [B, Hkv, P0 + n, D].
-size_t chunk_tensor_ws_bytes(int B, int Hq, int Hkv, int P0, int n, int D) {
-  const size_t q = align_up(static_cast<size_t>(B) * Hq * n * D * 2);
+// Workspace of the tensor-core chunk path: the FP16 key operands, cached
+// keys in both forms and values [B, Hkv, P0 + n, D] (the kernel rotates the
+// chunk's queries as it loads them).
+size_t chunk_tensor_ws_bytes(int B, int Hkv, int P0, int n, int D) {
   const size_t k = align_up(static_cast<size_t>(B) * Hkv * (static_cast<size_t>(P0) + n) * D * 2);
-  return 2 * q + 3 * k;
+  return 3 * k;
 }
 
 size_t chunk_ws_bytes(int B, int Hq, int Hkv, int P0, int n, int D) {
-  return n >= kChunkTensorMin ? chunk_tensor_ws_bytes(B, Hq, Hkv, P0, n, D)
+  return n >= kChunkTensorMin ? chunk_tensor_ws_bytes(B, Hkv, P0, n, D)
                               : decode_ws_bytes(B * n, Hq, Hkv, P0 + n, D);
 }
 
@@ -470,7 +466,7 @@ int chunk_tensor(const void *q, const void *k_cache, const void *v_cache, void *
   // grids: (query tiles, KV heads x head pairs, batch) and (positions, batch)
   if (B > kMaxGridYZ || static_cast<long long>(Hkv) * ((Hq / Hkv + 1) / 2) > kMaxGridYZ)
     return JL_ERR_SHAPE;
-  const size_t need = chunk_tensor_ws_bytes(B, Hq, Hkv, P0, n, D);
+  const size_t need = chunk_tensor_ws_bytes(B, Hkv, P0, n, D);
   if (!workspace || workspace_bytes < need) return JL_ERR_WORKSPACE;
   if (reinterpret_cast<uintptr_t>(workspace) % kAlign) return JL_ERR_ALIGN;
   DeviceState *dev = nullptr;
@@ -482,13 +478,10 @@ int chunk_tensor(const void *q, const void *k_cache, const void *v_cache, void *
   a.lse = lse;
   a.out_f32 = out_dtype == JL_F32;
   uint8_t *ws = static_cast<uint8_t *>(workspace);
-  const size_t qb = align_up(static_cast<size_t>(B) * Hq * n * D * 2);
   const size_t kb = align_up(static_cast<size_t>(B) * Hkv * L * D * 2);
-  a.q_true = reinterpret_cast<__half *>(ws);
-  a.q_remote = reinterpret_cast<__half *>(ws + qb);
-  a.k_true = reinterpret_cast<__half *>(ws + 2 * qb);
-  a.k_remote = reinterpret_cast<__half *>(ws + 2 * qb + kb);
-  a.v_op = reinterpret_cast<__half *>(ws + 2 * qb + 2 * kb);
+  a.k_true = reinterpret_cast<__half *>(ws);
+  a.k_remote = reinterpret_cast<__half *>(ws + kb);
+  a.v_op = reinterpret_cast<__half *>(ws + 2 * kb);
   a.B = B;
   a.Hq = Hq;
   a.Hkv = Hkv;

@@ -110,7 +110,7 @@ __device__ __forceinline__ void rope_cos_sin(long long pos, double freq, float &
 // r_t = w_pretrained * theta_t / (2 pi) that frequency t makes within the
 // pretrained window, and s = max(1, L / w_pretrained), the continuous dynamic
 // factor of §3.1.  Returns theta'_t / theta_t.
-__device__ __forceinline__ double interp_factor(double freq, int L, int w_pretrained,
+__host__ __device__ __forceinline__ double interp_factor(double freq, int L, int w_pretrained,
                                                 double alpha, double beta) {
   const double s = fmax(1.0, static_cast<double>(L) / static_cast<double>(w_pretrained));
   const double turns = static_cast<double>(w_pretrained) * freq * 0.15915494309189533577;
@@ -138,9 +138,10 @@ struct PrefillArgs {
   int out_f32;
   __nv_bfloat16 *k_cache_out;
   int k_cache_capacity;
-  // MMA operands in the workspace, FP16 head-major [B, H, L, D]: queries and
-  // keys rotated to true / remote positions, and the values
-  __half *q_true, *q_remote, *k_true, *k_remote, *v_op;
+  // key operands in the workspace, FP16 head-major [B, Hkv, L, D]: keys
+  // rotated to true / remote positions, and the values (the queries are
+  // rotated by the attention kernel from q)
+  __half *k_true, *k_remote, *v_op;
   // sizes and method parameters; L is the number of keys (positions
   // [0, L)), the queries are positions [q_off, q_off + Lq) with
   // q_off + Lq = L (a whole prompt: q_off = 0, Lq = L)
@@ -159,13 +160,13 @@ struct PrefillArgs {
   unsigned int *dev_error;
 };
 
-// Rotates q and k into the four operand arrays (and the optional cache).
-cudaError_t launch_rope_qk(const PrefillArgs &a, cudaStream_t stream);
+// Rotates k into the two key operand arrays, copies v to its operand array
+// (and writes the optional cache).
+cudaError_t launch_rope_kv(const PrefillArgs &a, cudaStream_t stream);
 
-// The operands of a chunk appended to a cache: the queries (positions
-// [q_off, L)) rotated to their true and remote positions, and the cached keys
-// and values of positions [0, L) as FP16 operands, the keys also in their
-// remote form (the correction rotation of §3.2 applied).
+// The key operands of a chunk appended to a cache: the cached keys and values
+// of positions [0, L) as FP16 operands, the keys also in their remote form
+// (the correction rotation of §3.2 applied).
 cudaError_t launch_chunk_operands(const PrefillArgs &a, cudaStream_t stream);
 
 // The attention kernel proper (tcgen05 / TMEM / TMA).

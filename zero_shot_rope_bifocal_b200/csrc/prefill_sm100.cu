@@ -77,7 +77,7 @@ struct Layout {
   static constexpr int RING = 2 * TILE;
   static constexpr int BAR = RING + NS * TILE;
   // barrier indices (8 bytes each)
-  static constexpr int kQFull = 0, kQEmpty = 2, kKvFull = 4, kKvEmpty = 4 + NS,
+  static constexpr int kQFull = 0, kKvFull = 4, kKvEmpty = 4 + NS,
                        kSFull = 4 + 2 * NS, kPFull = 6 + 2 * NS, kOFull = 8 + 2 * NS,
                        kDrain = 10 + 2 * NS, kNumBars = 11 + 2 * NS;
   static constexpr int TMEM_SLOT = BAR + 8 * kNumBars;
@@ -95,6 +95,14 @@ struct Params {
   int B, Hq, Hkv, q_off, Lq, G, w0eff, n_qt, grp, npair;
   int pass;  // PrefillPass: the fused rule or one pass of the three-pass merge
   float scale_log2;
+  // Queries, pre-RoPE BF16 [B, Lq, Hq, D]: the softmax threads rotate their
+  // rows into the FP16 operand tiles.  omega[i] = theta_i / (2 pi), turns per
+  // position as a 64-bit binary fraction; omega_remote[i] is the remote
+  // map's (theta_i, or theta'_i under the frequency interpolation, where the
+  // remote position is the true one).
+  const __nv_bfloat16 *q_raw;
+  int remote_interp;
+  uint64_t omega[64], omega_remote[64];
   void *out;
   float *lse;
   int out_f32;
@@ -142,13 +150,76 @@ __device__ __forceinline__ bool wait_or_abort(uint32_t bar, uint32_t parity,
   }
 }
 
+// RoPE in the Q load path: one softmax thread turns its row of the query
+// into the FP16 operand tile of its query tile, at the remote position
+// (f(row), or row with the remote map's frequencies) or at the true
+// position.  The tile is 128-byte swizzled as the MMA descriptors expect:
+// row r of a 64-channel box is 128 bytes, its 16-byte chunk k stored at chunk
+// k ^ (r % 8).  Rows past the last query are zero.  The angle pos * theta_i
+// is exact modulo one turn: the wrapping 64-bit product with theta_i / (2 pi)
+// (a 64-bit binary fraction) has the signed phase in its top 32 bits, so the
+// sine/cosine only sees [-pi, pi).  The generic-proxy writes are fenced for
+// the async proxy before the caller's arrival on the tile's barrier.  Kept out
+// of line: it runs twice per CTA and its registers stay out of the visit loop.
+template <int D>
+__device__ __noinline__ void build_q_row(uint8_t *tile, int rloc, int row, bool row_ok, int b,
+                                         int head, bool remote_var, const Params &prm) {
+  constexpr int BOX = 128 * 128;
+  auto store16 = [&](int c, uint4 v) {  // channels [c, c + 8)
+    uint8_t *box = tile + (c >> 6) * BOX + rloc * 128;
+    *reinterpret_cast<uint4 *>(box + ((((c & 63) >> 3) ^ (rloc & 7)) << 4)) = v;
+  };
+  bool in_range = true;
+  if (row_ok) {
+    const uint64_t pos =
+        static_cast<uint64_t>((!remote_var || prm.remote_interp) ? row : remap(row, prm.G));
+    const uint64_t *om = remote_var ? prm.omega_remote : prm.omega;
+    constexpr float kTurnToRad = 1.4629180792671596e-09f;  // 2 pi / 2^32
+    auto cos_sin = [&](int i, float &cv, float &sv) {
+      const int32_t ph = static_cast<int32_t>((pos * om[i]) >> 32);
+      __sincosf(static_cast<float>(ph) * kTurnToRad, &sv, &cv);
+    };
+    const uint4 *src = reinterpret_cast<const uint4 *>(
+        prm.q_raw + ((static_cast<size_t>(b) * prm.Lq + (row - prm.q_off)) * prm.Hq + head) * D);
+    uint4 raw[D / 8];  // the whole row, all loads in flight at once
+#pragma unroll
+    for (int k = 0; k < D / 8; ++k) raw[k] = __ldg(src + k);
+#pragma unroll
+    for (int c = 0; c < D / 2; c += 8) {  // channels c.. and their partners c + D/2..
+      const uint4 xa = raw[c / 8], xb = raw[(c + D / 2) / 8];
+      const uint32_t wa[4] = {xa.x, xa.y, xa.z, xa.w}, wb[4] = {xb.x, xb.y, xb.z, xb.w};
+      uint32_t oa[4], ob[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        float c0, s0, c1, s1;
+        cos_sin(c + 2 * e, c0, s0);
+        cos_sin(c + 2 * e + 1, c1, s1);
+        const float x0 = __uint_as_float(wa[e] << 16), x1 = __uint_as_float(wa[e] & 0xffff0000u);
+        const float y0 = __uint_as_float(wb[e] << 16), y1 = __uint_as_float(wb[e] & 0xffff0000u);
+        const __half2 lo = __floats2half2_rn(x0 * c0 - y0 * s0, x1 * c1 - y1 * s1);
+        const __half2 hi = __floats2half2_rn(x0 * s0 + y0 * c0, x1 * s1 + y1 * c1);
+        in_range &= !(__hisinf(__low2half(lo)) | __hisinf(__high2half(lo)) |
+                      __hisinf(__low2half(hi)) | __hisinf(__high2half(hi)));
+        oa[e] = *reinterpret_cast<const uint32_t *>(&lo);
+        ob[e] = *reinterpret_cast<const uint32_t *>(&hi);
+      }
+      store16(c, make_uint4(oa[0], oa[1], oa[2], oa[3]));
+      store16(c + D / 2, make_uint4(ob[0], ob[1], ob[2], ob[3]));
+    }
+  } else {
+#pragma unroll
+    for (int c = 0; c < D; c += 8) store16(c, make_uint4(0u, 0u, 0u, 0u));
+  }
+  if (!in_range) atomicOr(prm.dev_error, kDevRange);
+  fence_proxy_async_smem();
+}
+
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
-bifocal_prefill_kernel(const __grid_constant__ CUtensorMap tm_qt,
-                       const __grid_constant__ CUtensorMap tm_qr,
-                       const __grid_constant__ CUtensorMap tm_kt,
+bifocal_prefill_kernel(const __grid_constant__ CUtensorMap tm_kt,
                        const __grid_constant__ CUtensorMap tm_kr,
-                       const __grid_constant__ CUtensorMap tm_v, const Params prm) {
+                       const __grid_constant__ CUtensorMap tm_v,
+                       const __grid_constant__ Params prm) {
   using LY = Layout<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
@@ -211,16 +282,17 @@ bifocal_prefill_kernel(const __grid_constant__ CUtensorMap tm_qt,
   if (*skip != kDevOk) return;
 
   if (tid == 0) {
-    // P-ready barriers take one arrival from every softmax thread of the
-    // tile (one per row); all others one arrival (plus transaction bytes for
-    // TMA).
+    // Q-ready and P-ready barriers take one arrival from every softmax
+    // thread of the tile (one per row); all others one arrival (plus
+    // transaction bytes for TMA).
     for (int i = 0; i < LY::kNumBars; ++i)
-      mbar_init(bar(i), (i == LY::kPFull || i == LY::kPFull + 1) ? BM : 1);
+      mbar_init(bar(i), (i == LY::kPFull || i == LY::kPFull + 1 || i == LY::kQFull ||
+                         i == LY::kQFull + 1)
+                            ? BM
+                            : 1);
     fence_mbar_init();
   }
   if (warp == kProducerWarp && lane == 0) {
-    prefetch_tmap(&tm_qt);
-    prefetch_tmap(&tm_qr);
     prefetch_tmap(&tm_kt);
     prefetch_tmap(&tm_kr);
     prefetch_tmap(&tm_v);
@@ -245,14 +317,6 @@ bifocal_prefill_kernel(const __grid_constant__ CUtensorMap tm_qt,
   if (warp >= kSoftmaxWarps) {
     if (warp == kProducerWarp && lane == 0) {
       // ---------------------------------------------------------- producer
-      auto load_q = [&](int s, bool remote) {
-        mbar_arrive_expect_tx(bar(LY::kQFull + s), LY::TILE);
-        for (int c = 0; c < NBOX; ++c)
-          tma_load_3d(sb + LY::Q0 + s * LY::TILE + c * LY::BOX, remote ? &tm_qr : &tm_qt,
-                      bar(LY::kQFull + s), c * 64, qt * BM, b * prm.Hq + head0 + s);
-      };
-      load_q(0, n_rem > 0);
-      if (has1) load_q(1, n_rem > 0);
       int r = 0;
       bool ok = true;
       uint32_t issued[NS] = {0, 0, 0, 0};  // uses issued per slot
@@ -271,14 +335,6 @@ bifocal_prefill_kernel(const __grid_constant__ CUtensorMap tm_qt,
             tma_load_3d(dst + c * LY::BOX, tm, bar(LY::kKvFull + slot), c * 64, kt * BN,
                         b * prm.Hkv + g);
           issued[slot] = use + 1;
-        }
-        if (ok && switch_q && j == n_rem - 1) {
-          ok = wait_or_abort(bar(LY::kQEmpty + 0), 0u, abort);
-          if (ok) load_q(0, false);
-          if (ok && has1) {
-            ok = wait_or_abort(bar(LY::kQEmpty + 1), 0u, abort);
-            if (ok) load_q(1, false);
-          }
         }
       }
       if (!ok) {
@@ -321,11 +377,7 @@ bifocal_prefill_kernel(const __grid_constant__ CUtensorMap tm_qt,
       if (ok) {
         tc_fence_after();
         qk(0, kslot);
-        if (switch_q && n_rem == 1) mma_commit(bar(LY::kQEmpty + 0));
-        if (has1) {
-          qk(1, kslot);
-          if (switch_q && n_rem == 1) mma_commit(bar(LY::kQEmpty + 1));
-        }
+        if (has1) qk(1, kslot);
         mma_commit(bar(LY::kKvEmpty + kslot));
       }
       for (int j = 0; j < nv && ok; ++j) {
@@ -347,7 +399,6 @@ bifocal_prefill_kernel(const __grid_constant__ CUtensorMap tm_qt,
           if (!ok) break;
           tc_fence_after();
           qk(0, kslot);
-          if (switch_q && j + 2 == n_rem) mma_commit(bar(LY::kQEmpty + 0));
         }
         // tile 1: O1 += P1(j) V(j), then S1(j+1)
         if (has1) {
@@ -363,7 +414,6 @@ bifocal_prefill_kernel(const __grid_constant__ CUtensorMap tm_qt,
             if (!ok) break;
             tc_fence_after();
             qk(1, kslot);
-            if (switch_q && j + 2 == n_rem) mma_commit(bar(LY::kQEmpty + 1));
           }
           mma_commit(bar(LY::kKvEmpty + kslot));
         }
@@ -390,6 +440,15 @@ bifocal_prefill_kernel(const __grid_constant__ CUtensorMap tm_qt,
     const bool active = s == 0 || has1;
     const bool row_ok = active && row < prm.q_off + prm.Lq;
     const uint32_t lane_base = static_cast<uint32_t>(wq * 32) << 16;
+    // RoPE in the Q load path (build_q_row): at the remote position first
+    // (if the tile has remote visits), at the true position after the switch.
+    auto build_q = [&](bool remote_var) {
+      build_q_row<D>(smem + Layout<D>::Q0 + s * Layout<D>::TILE, rloc, row, row_ok, b, head0 + s,
+                     remote_var, prm);
+      mbar_arrive(bar(LY::kQFull + s));
+    };
+    if (active) build_q(n_rem > 0);
+
     float m_used = -INFINITY;  // reference max of this row (base 2)
     float l_sum = 0.f;         // running row sum, relative to m_used
     bool ok = active;
@@ -497,6 +556,9 @@ bifocal_prefill_kernel(const __grid_constant__ CUtensorMap tm_qt,
       }
       tc_fence_before();
       mbar_arrive(bar(LY::kPFull + s));
+      // After the last remote visit the query tile switches to true
+      // positions: S(j) was read, so QK(j) is done with the tile.
+      if (switch_q && j == n_rem - 1) build_q(false);
     }
     // ---- epilogue: O / l and the log-sum-exp of this row
     if (ok) ok = wait_or_abort(bar(LY::kOFull + s), 0u, abort);
@@ -581,11 +643,9 @@ bool encode_head_major(CUtensorMap *tm, const void *base, int BH, int L, int D) 
 template <int D>
 cudaError_t launch_d(const PrefillArgs &a, cudaStream_t stream) {
   if (!encode_fn()) return cudaErrorNotSupported;
-  CUtensorMap tqt, tqr, tkt, tkr, tv;
+  CUtensorMap tkt, tkr, tv;
   const bool two = a.G > 1;
-  if (!encode_head_major(&tqt, a.q_true, a.B * a.Hq, a.Lq, D) ||
-      !encode_head_major(&tqr, two ? a.q_remote : a.q_true, a.B * a.Hq, a.Lq, D) ||
-      !encode_head_major(&tkt, a.k_true, a.B * a.Hkv, a.L, D) ||
+  if (!encode_head_major(&tkt, a.k_true, a.B * a.Hkv, a.L, D) ||
       !encode_head_major(&tkr, two ? a.k_remote : a.k_true, a.B * a.Hkv, a.L, D) ||
       !encode_head_major(&tv, a.v_op, a.B * a.Hkv, a.L, D))
     return cudaErrorInvalidValue;
@@ -608,11 +668,22 @@ cudaError_t launch_d(const PrefillArgs &a, cudaStream_t stream) {
   prm.lse = a.lse;
   prm.out_f32 = a.out_f32;
   prm.dev_error = a.dev_error;
+  prm.q_raw = a.q;
+  prm.remote_interp = a.interp;
+  const double log_theta = std::log(static_cast<double>(a.theta));
+  const double turns_q64 = 0.15915494309189533577 * 18446744073709551616.0;  // 2^64 / (2 pi)
+  for (int i = 0; i < D / 2; ++i) {
+    const double f = std::exp(-2.0 * static_cast<double>(i) / static_cast<double>(D) * log_theta);
+    const double fr =
+        a.interp ? f * interp_factor(f, a.L, a.w_pretrained, a.ramp_alpha, a.ramp_beta) : f;
+    prm.omega[i] = static_cast<uint64_t>(std::llround(f * turns_q64));  // < 2^62
+    prm.omega_remote[i] = static_cast<uint64_t>(std::llround(fr * turns_q64));
+  }
   const int smem = Layout<D>::ALLOC;
   cudaError_t e = ensure_smem_limit<bifocal_prefill_kernel<D>>(smem);
   if (e != cudaSuccess) return e;
   const dim3 grid(prm.n_qt, a.Hkv * prm.npair, a.B);
-  bifocal_prefill_kernel<D><<<grid, kThreads, smem, stream>>>(tqt, tqr, tkt, tkr, tv, prm);
+  bifocal_prefill_kernel<D><<<grid, kThreads, smem, stream>>>(tkt, tkr, tv, prm);
   return cudaGetLastError();
 }
 

@@ -1,37 +1,38 @@
-// rope_kernels.cu -- RoPE in the Q/K load path of the bifocal attention.
+// rope_kernels.cu -- the key side of RoPE for the bifocal attention (the
+// queries are rotated in the attention kernel's load path, see
+// prefill_sm100.cu).
 //
-// Prefill operand pass (Jet-Long paper, §3 score rule and §3.2): for every
-// token the queries are rotated to the true position i and to the remote
-// position f(i), the keys to j and to f(j):
+// Prefill key operands (Jet-Long paper, §3 score rule and §3.2): every key
+// is rotated to its true position j and to its remote position f(j):
 //
-//   q_true[b,h,i]  = RoPE(x_q, i)      q_remote[b,h,i] = RoPE(x_q, f(i))
 //   k_true[b,g,j]  = RoPE(x_k, j)      k_remote[b,g,j] = RoPE(x_k, f(j))
 //
 // k_true is exactly the true-position KV cache of §3.2, and k_remote equals
 // the correction rotation by Delta j = f(j) - j applied to it.  The outputs
 // (and a copy of v) are the tensor-core operands: FP16, head-major
-// [B, H, L, D], so that the attention kernel's TMA fetches each 128-token tile
-// as one contiguous block.  FP16 holds the rotated values with three more
-// mantissa bits than BF16; a value beyond the FP16 range (|x| > 65504) is
-// reported through the device error word.  The optional cache output keeps
-// the caller's BF16 format.  When G == 1 (L <= w_pretrained,
-// the native-window case of Appendix H) f is the identity and only the
-// true-position arrays are written.
+// [B, Hkv, L, D], so that the attention kernel's TMA fetches each 128-token
+// tile as one contiguous block.  Every key tile is read by every query tile
+// of its KV head, so the keys are rotated once here rather than in each
+// CTA.  FP16 holds the rotated values with three more mantissa bits than
+// BF16; a value beyond the FP16 range (|x| > 65504) is reported through the
+// device error word.  The optional cache output keeps the caller's BF16
+// format.  When G == 1 (L <= w_pretrained, the native-window case of
+// Appendix H) f is the identity and only the true-position arrays are
+// written.
 //
 // With the frequency-interpolation remote map (the §4.7 ablation) the remote
-// arrays hold RoPE'(x, i): true position, interpolated frequencies theta'_t.
+// arrays hold RoPE'(x, j): true position, interpolated frequencies theta'_t.
 //
 // Chunk operands (a chunk of queries appended to a cache, §3.1, §3.2): the
-// queries as above at their positions P0 + t, and the keys and values read
-// from the true-position cache; the remote keys are the cached ones turned by
-// the correction rotation R(f(j) - j).
+// keys and values read from the true-position cache; the remote keys are the
+// cached ones turned by the correction rotation R(f(j) - j).
 //
 // Cache writer (§3.2): k_cache[b, pos0 + t] = RoPE(k[b, t], pos0 + t).
 //
 // Each CTA forms the frequencies once, evaluates cos/sin once per (position,
 // frequency) into shared memory and applies it to every head of that
-// position; channel pairs are
-// (i, i + D/2), processed two pairs per thread with BF16x2 loads and stores.
+// position; channel pairs are (i, i + D/2), processed two pairs per thread
+// with BF16x2 loads and FP16x2 stores.
 #include "jl_common.cuh"
 
 namespace jl {
@@ -73,7 +74,7 @@ __device__ __forceinline__ bool store_f16(__half *dst, int i, int half, const Ro
 }
 
 __global__ void __launch_bounds__(kRopeThreads)
-rope_qk_kernel(PrefillArgs a) {
+rope_kv_kernel(PrefillArgs a) {
   extern __shared__ float2 cs_smem[];  // [2][kPosPerCta][D/2] (cos, sin), then 2 x [D/2] freq
   const int half = a.D / 2;
   const int b = blockIdx.y;
@@ -107,22 +108,6 @@ rope_qk_kernel(PrefillArgs a) {
 
   bool in_range = true;
   const int quarter = a.D / 4;  // pairs of channel pairs per head row
-  // queries
-  for (int idx = threadIdx.x; idx < npos * a.Hq * quarter; idx += blockDim.x) {
-    const int t = idx / (a.Hq * quarter);
-    const int rem = idx - t * a.Hq * quarter;
-    const int h = rem / quarter;
-    const int i = (rem - h * quarter) * 2;
-    const int pos = p_begin + t;
-    const __nv_bfloat16 *src = a.q + ((static_cast<size_t>(b) * a.L + pos) * a.Hq + h) * a.D;
-    const size_t drow = ((static_cast<size_t>(b) * a.Hq + h) * a.L + pos) * a.D;
-    in_range &= store_f16(a.q_true + drow, i, half,
-                          rotate2(src, i, half, cs_true[t * half + i], cs_true[t * half + i + 1]));
-    if (two)
-      in_range &= store_f16(a.q_remote + drow, i, half,
-                            rotate2(src, i, half, cs_remote[t * half + i],
-                                    cs_remote[t * half + i + 1]));
-  }
   // keys (+ optional true-position cache) and values
   for (int idx = threadIdx.x; idx < npos * a.Hkv * quarter; idx += blockDim.x) {
     const int t = idx / (a.Hkv * quarter);
@@ -145,61 +130,6 @@ rope_qk_kernel(PrefillArgs a) {
     // values: the identity rotation, i.e. a BF16 -> FP16 copy into head-major order
     in_range &= store_f16(a.v_op + drow, i, half,
                           rotate2(a.v + srow, i, half, make_float2(1.f, 0.f), make_float2(1.f, 0.f)));
-  }
-  if (!in_range) atomicOr(a.dev_error, kDevRange);
-}
-
-// Chunk operands, queries: for t < Lq, position pos = q_off + t,
-//   q_true[b,h,t] = RoPE(x_q[b,t,h], pos),  q_remote[b,h,t] = RoPE(x_q[b,t,h], f(pos))
-// (RoPE'(x_q, pos) under the frequency-interpolation map), FP16 head-major
-// [B, Hq, Lq, D]; G and the interpolation factor come from L = q_off + Lq.
-__global__ void __launch_bounds__(kRopeThreads)
-chunk_q_kernel(PrefillArgs a) {
-  extern __shared__ float2 cs_smem[];  // [2][kPosPerCta][D/2] (cos, sin), then 2 x [D/2] freq
-  const int half = a.D / 2;
-  const int b = blockIdx.y;
-  const int t_begin = blockIdx.x * kPosPerCta;
-  const int npos = min(kPosPerCta, a.Lq - t_begin);
-  const bool two = a.G > 1;
-  float2 *cs_true = cs_smem;
-  float2 *cs_remote = cs_smem + kPosPerCta * half;
-  double *freq = reinterpret_cast<double *>(cs_smem + 2 * kPosPerCta * half);
-  double *freq_remote = freq + half;
-  const double theta = static_cast<double>(a.theta);
-  for (int i = threadIdx.x; i < half; i += blockDim.x) {
-    const double f = rope_freq(i, a.D, theta);
-    freq[i] = f;
-    freq_remote[i] =
-        a.interp ? f * interp_factor(f, a.L, a.w_pretrained, a.ramp_alpha, a.ramp_beta) : f;
-  }
-  __syncthreads();
-  for (int idx = threadIdx.x; idx < npos * half * (two ? 2 : 1); idx += blockDim.x) {
-    const int var = idx / (npos * half);
-    const int rem = idx - var * npos * half;
-    const int t = rem / half, i = rem - t * half;
-    const int pos = a.q_off + t_begin + t;
-    const long long ppos = (var == 0 || a.interp) ? pos : remap(pos, a.G);
-    float c, s;
-    rope_cos_sin(ppos, var == 0 ? freq[i] : freq_remote[i], c, s);
-    (var == 0 ? cs_true : cs_remote)[t * half + i] = make_float2(c, s);
-  }
-  __syncthreads();
-  bool in_range = true;
-  const int quarter = a.D / 4;
-  for (int idx = threadIdx.x; idx < npos * a.Hq * quarter; idx += blockDim.x) {
-    const int t = idx / (a.Hq * quarter);
-    const int rem = idx - t * a.Hq * quarter;
-    const int h = rem / quarter;
-    const int i = (rem - h * quarter) * 2;
-    const __nv_bfloat16 *src =
-        a.q + ((static_cast<size_t>(b) * a.Lq + t_begin + t) * a.Hq + h) * a.D;
-    const size_t drow = ((static_cast<size_t>(b) * a.Hq + h) * a.Lq + t_begin + t) * a.D;
-    in_range &= store_f16(a.q_true + drow, i, half,
-                          rotate2(src, i, half, cs_true[t * half + i], cs_true[t * half + i + 1]));
-    if (two)
-      in_range &= store_f16(a.q_remote + drow, i, half,
-                            rotate2(src, i, half, cs_remote[t * half + i],
-                                    cs_remote[t * half + i + 1]));
   }
   if (!in_range) atomicOr(a.dev_error, kDevRange);
 }
@@ -294,18 +224,14 @@ rope_cache_kernel(const __nv_bfloat16 *__restrict__ k, __nv_bfloat16 *__restrict
 
 }  // namespace
 
-cudaError_t launch_rope_qk(const PrefillArgs &a, cudaStream_t stream) {
+cudaError_t launch_rope_kv(const PrefillArgs &a, cudaStream_t stream) {
   const dim3 grid((a.L + kPosPerCta - 1) / kPosPerCta, a.B);
   const size_t smem = 2 * kPosPerCta * (a.D / 2) * sizeof(float2) + 2 * (a.D / 2) * sizeof(double);
-  rope_qk_kernel<<<grid, kRopeThreads, smem, stream>>>(a);
+  rope_kv_kernel<<<grid, kRopeThreads, smem, stream>>>(a);
   return cudaGetLastError();
 }
 
 cudaError_t launch_chunk_operands(const PrefillArgs &a, cudaStream_t stream) {
-  const size_t smem_q = 2 * kPosPerCta * (a.D / 2) * sizeof(float2) + 2 * (a.D / 2) * sizeof(double);
-  chunk_q_kernel<<<dim3((a.Lq + kPosPerCta - 1) / kPosPerCta, a.B), kRopeThreads, smem_q, stream>>>(a);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
   const size_t smem_k = kPosPerCta * (a.D / 2) * sizeof(float2) + (a.D / 2) * sizeof(double);
   cache_kv_kernel<<<dim3((a.L + kPosPerCta - 1) / kPosPerCta, a.B), kRopeThreads, smem_k, stream>>>(a);
   return cudaGetLastError();

@@ -42,9 +42,9 @@ SIGNATURES = {
     "jetlong_prefill_workspace_size": (_SZ, [_I, _I, _I, _I, _I]),
     "jetlong_prefill": (_I, [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _I, _F, _I,
                              _VP, _I, _VP, _SZ, _VP]),
-    "jetlong_prefill_rotate": (_I, [_VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _F, _VP, _I, _VP, _SZ,
+    "jetlong_prefill_rotate": (_I, [_VP, _VP, _I, _I, _I, _I, _I, _F, _VP, _I, _VP, _SZ, _VP]),
+    "jetlong_prefill_attend": (_I, [_VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _I, _F, _I, _VP, _SZ,
                                     _VP]),
-    "jetlong_prefill_attend": (_I, [_VP, _VP, _I, _I, _I, _I, _I, _I, _I, _I, _VP, _SZ, _VP]),
     "jetlong_prefill_three_pass_workspace_size": (_SZ, [_I, _I, _I, _I, _I]),
     "jetlong_prefill_three_pass": (_I, [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _I, _F,
                                         _I, _VP, _SZ, _VP]),
@@ -241,38 +241,40 @@ def _prefill(fn, q, k, v, w_pretrained, w0, method, out, lse, out_dtype, want_ls
     return out, lse
 
 
-def jetlong_prefill_rotate(q, k, v, w_pretrained: int, rope_theta: float, workspace, *,
+def jetlong_prefill_rotate(k, v, w_pretrained: int, rope_theta: float, workspace, *,
                            k_cache_out=None, stream=None):
-    """Stage 1 of jetlong_prefill: the FP16 tensor-core operands into ``workspace``."""
-    B, L, Hq, D = q.shape
-    Hkv = k.shape[2]
-    _require(q, "q", (B, L, Hq, D), torch.bfloat16)
+    """Stage 1 of jetlong_prefill: the FP16 key operands into ``workspace``."""
+    if k.dim() != 4:
+        raise ValueError("k and v must be [B, L, Hkv, D]")
+    B, L, Hkv, D = k.shape
     _require(k, "k", (B, L, Hkv, D), torch.bfloat16)
     _require(v, "v", (B, L, Hkv, D), torch.bfloat16)
     cap = 0 if k_cache_out is None else k_cache_out.shape[1]
     if k_cache_out is not None:
         _require(k_cache_out, "k_cache_out", (B, cap, Hkv, D), torch.bfloat16)
-    workspace, ws_bytes = _workspace(workspace, 0, q.device)
-    st = lib().jetlong_prefill_rotate(_ptr(q), _ptr(k), _ptr(v), B, Hq, Hkv, L, D,
-                                      int(w_pretrained), float(rope_theta), _ptr(k_cache_out), cap,
-                                      _ptr(workspace), ws_bytes, _stream_ptr(stream))
+    workspace, ws_bytes = _workspace(workspace, 0, k.device)
+    st = lib().jetlong_prefill_rotate(_ptr(k), _ptr(v), B, Hkv, L, D, int(w_pretrained),
+                                      float(rope_theta), _ptr(k_cache_out), cap, _ptr(workspace),
+                                      ws_bytes, _stream_ptr(stream))
     _check("jetlong_prefill_rotate", st)
 
 
-def jetlong_prefill_attend(out, lse, Hkv: int, w_pretrained: int, w0: int, workspace, *,
-                           stream=None):
-    """Stage 2 of jetlong_prefill: the attention kernel on the operands in ``workspace``."""
+def jetlong_prefill_attend(q, out, lse, Hkv: int, w_pretrained: int, w0: int, rope_theta: float,
+                           workspace, *, stream=None):
+    """Stage 2 of jetlong_prefill: the attention kernel (queries rotated as
+    they are loaded) on the key operands in ``workspace``."""
     od = _out_code(out, None)
-    if out.dim() != 4:
-        raise ValueError("out must be [B, L, Hq, D]")
-    B, L, Hq, D = out.shape
+    if q.dim() != 4 or out.dim() != 4:
+        raise ValueError("q and out must be [B, L, Hq, D]")
+    B, L, Hq, D = q.shape
+    _require(q, "q", (B, L, Hq, D), torch.bfloat16)
     _require(out, "out", (B, L, Hq, D), out.dtype)
     if lse is not None:
         _require(lse, "lse", (B, Hq, L), torch.float32)
     workspace, ws_bytes = _workspace(workspace, 0, out.device)
-    st = lib().jetlong_prefill_attend(_ptr(out), _ptr(lse), B, Hq, int(Hkv), L, D,
-                                      int(w_pretrained), int(w0), od, _ptr(workspace), ws_bytes,
-                                      _stream_ptr(stream))
+    st = lib().jetlong_prefill_attend(_ptr(q), _ptr(out), _ptr(lse), B, Hq, int(Hkv), L, D,
+                                      int(w_pretrained), int(w0), float(rope_theta), od,
+                                      _ptr(workspace), ws_bytes, _stream_ptr(stream))
     _check("jetlong_prefill_attend", st)
 
 

@@ -44,10 +44,10 @@ def main(argv=None) -> int:
         lse = torch.empty((w.B, w.Hq, w.L), dtype=torch.float32, device=dev)
         ws = torch.empty(jl.jetlong_prefill_workspace_size(w.B, w.Hq, w.Hkv, w.L, w.D),
                          dtype=torch.uint8, device=dev)
-        jl.jetlong_prefill_rotate(x.q, x.k, x.v, w.w_pretrained, w.theta, ws)
+        jl.jetlong_prefill_rotate(x.k, x.v, w.w_pretrained, w.theta, ws)
 
         def call():
-            jl.jetlong_prefill_attend(out, lse, w.Hkv, w.w_pretrained, w.w0, ws)
+            jl.jetlong_prefill_attend(x.q, out, lse, w.Hkv, w.w_pretrained, w.w0, w.theta, ws)
     else:
         d = decode_inputs(w, device=dev)
         kc = torch.empty_like(d.k_raw)
