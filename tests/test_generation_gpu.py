@@ -9,8 +9,8 @@ fp64 oracle).
   consecutive steps while the cache itself is never rewritten (§3.2).  The
   oracle builds its own cache from the raw keys; nothing it reads comes from
   the GPU.
-* Decode at 256K, 512K and 1M tokens (G = 8, 16, 32) and a prefill at 256K
-  (G = 8): the schedule far past the 4x extension of the headline layer.
+* Decode and prefill at 256K, 512K and 1M tokens (G = 8, 16, 32): the
+  schedule far past the 4x extension of the headline layer.
 """
 import numpy as np
 import pytest
@@ -78,8 +78,10 @@ def test_long_context_decode(L):
     assert_lse(f64(lse), lse_ref, f"L={L}")
 
 
-def test_long_context_prefill_256k_sampled_rows():
-    w = Workload("long_pf", 1, 8, 2, 128, 262144, 32768, 4096, 1e6, 91, True)
+@pytest.mark.parametrize("L", [262144, 524288, 1048576])
+def test_long_context_prefill_sampled_rows(L):
+    # G = 8, 16, 32: remote positions f(i) = i // G stay below w_pretrained
+    w = Workload("long_pf", 1, 8, 2, 128, L, 32768, 4096, 1e6, 91, True)
     x = prefill_inputs(w, device="cuda")
     out, lse = jl.jetlong_prefill(x.q, x.k, x.v, w.w_pretrained, w.w0, w.theta,
                                   out_dtype=torch.float32)
@@ -88,6 +90,7 @@ def test_long_context_prefill_256k_sampled_rows():
     ridx = torch.tensor(rows, device="cuda")
     o_ref, lse_ref = oracle.prefill_rows(f64(x.q.index_select(1, ridx)), f64(x.k), f64(x.v),
                                          w.w_pretrained, w.w0, w.theta, rows, q_holds_rows=True)
-    assert_o(f64(out.index_select(1, ridx)), o_ref, "256K")
-    assert_lse(f64(lse.index_select(2, ridx)), lse_ref, "256K")
+    assert jl.jetlong_group_size(L, w.w_pretrained) == L // 32768
+    assert_o(f64(out.index_select(1, ridx)), o_ref, f"L={L}")
+    assert_lse(f64(lse.index_select(2, ridx)), lse_ref, f"L={L}")
     assert torch.isfinite(out).all() and torch.isfinite(lse).all()
