@@ -54,8 +54,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # whose SHA-256 is recorded here; the capture and its command are summarised
 # in the profile named below.  The line reports it only while those sources
 # are unchanged, and null otherwise.
-TRAFFIC_RECORD = {"bytes": 6.95e9, "read_bytes": 5.83e9, "write_bytes": 1.12e9,
-                  "sources_sha256": "22a4f68e1b66737134bea386b4dc50ec180e3785a9656bfcc02ee64cab6a10ba",
+TRAFFIC_RECORD = {"bytes": 6.12e9, "read_bytes": 4.98e9, "write_bytes": 1.14e9,
+                  "sources_sha256": "833d188279f620c457fc1f51348fa4b0e03d886edc149d74a3243e0aa8f88447",
                   "profile": "profiles/prefill_attention_qwen3_8b_L131072_dram.md"}
 TRAFFIC_SOURCES = ("zero_shot_rope_bifocal_b200/csrc/prefill_sm100.cu",
                    "zero_shot_rope_bifocal_b200/csrc/sm100_ptx.cuh")
@@ -69,10 +69,10 @@ def prefill_flops(B: int, Hq: int, L: int, D: int) -> int:
 
 
 def prefill_operand_bytes(B: int, Hq: int, Hkv: int, L: int, D: int) -> int:
-    """Bytes the attention kernel must move at least: the FP16 operands read
-    once (q at true and remote positions, k at true and remote positions, v)
-    and the BF16 output written once."""
-    return (2 * B * Hq * L * D + 3 * B * Hkv * L * D) * 2 + B * L * Hq * D * 2
+    """Bytes the attention kernel must move at least: q read once (BF16; the
+    kernel rotates it as it loads it), the FP16 key operands read once (k at
+    true and remote positions, v) and the BF16 output written once."""
+    return B * L * Hq * D * 2 + 3 * B * Hkv * L * D * 2 + B * L * Hq * D * 2
 
 
 def row_flops(Hq: int, D: int, rows) -> int:
