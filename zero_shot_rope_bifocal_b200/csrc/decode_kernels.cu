@@ -260,7 +260,7 @@ __device__ __forceinline__ bool dec_wait(uint32_t bar, uint32_t parity, volatile
 // correction table either.
 template <int D, int GRP, bool BIFOCAL, bool TWO_FORM = false>
 __global__ void __launch_bounds__(kDecThreads, kCtasPerSm)
-decode_split_kernel(DecodeArgs a) {
+decode_split_kernel(const __grid_constant__ DecodeArgs a) {
   using C = DecCfg<D>;
   constexpr int P = C::P, NBLK = C::NBLK, KB = C::KB, HALF = D / 2, MB = D / 16;
 
@@ -342,26 +342,19 @@ decode_split_kernel(DecodeArgs a) {
     // The first copies go out before the RoPE tables are computed.
     for (int u = 0; u < kStages && u < n_stage; ++u) issue(u);
   }
-  constexpr double kTurnsQ64 = 0.15915494309189533577 * 18446744073709551616.0;  // 2^64 / (2 pi)
-  for (int i = tid; i < HALF; i += kDecThreads) {
-    const double f = rope_freq(i, D, static_cast<double>(a.theta));
-    // interpolation: (theta' - theta) / (2 pi) lies in (-1/(2 pi), 0], inside int64 once scaled
-    omega[i] = a.interp
-                   ? static_cast<uint64_t>(__double2ll_rn(
-                         f * (interp_factor(f, a.L, a.w_pretrained, a.ramp_alpha, a.ramp_beta) - 1.0) *
-                         kTurnsQ64))
-                   : __double2ull_rn(f * kTurnsQ64);
-  }
+  // The turn fractions per position come with the call (formed once on the
+  // host); the query's angles are exact modulo one turn like the table's.
+  constexpr float kTurnToRad = 1.4629180792671596e-09f;  // 2 pi / 2^32
+  for (int i = tid; i < HALF; i += kDecThreads) omega[i] = a.omega_corr[i];
+  const uint64_t pos_r = static_cast<uint64_t>(a.interp ? p : remap_fast(p, a.gdiv));
   for (int idx = tid; idx < 2 * HALF; idx += kDecThreads) {
     const int i = idx < HALF ? idx : idx - HALF;
-    const double f = rope_freq(i, D, static_cast<double>(a.theta));
+    // RoPE(x_q, p), and the remote query: RoPE(x_q, f(p)), or RoPE'(x_q, p)
+    // (true position, interpolated frequency)
+    const uint64_t turns = idx < HALF ? static_cast<uint64_t>(p) * a.omega_qt[i]
+                                      : pos_r * a.omega_qr[i];
     float c, sn;
-    if (idx < HALF)
-      rope_cos_sin(p, f, c, sn);
-    else if (a.interp)  // RoPE'(x_q, p): true position, interpolated frequency
-      rope_cos_sin(p, f * interp_factor(f, a.L, a.w_pretrained, a.ramp_alpha, a.ramp_beta), c, sn);
-    else
-      rope_cos_sin(remap(p, G), f, c, sn);
+    __sincosf(static_cast<float>(static_cast<int32_t>(turns >> 32)) * kTurnToRad, &sn, &c);
     qcs[idx] = make_float2(c, sn);
   }
   __syncthreads();
@@ -638,7 +631,7 @@ static_assert(kMaxSplit <= 2 * kCombineThreads, "two splits per thread in the ma
 
 template <int D>
 __global__ void __launch_bounds__(kCombineThreads)
-decode_combine_kernel(DecodeArgs a) {
+decode_combine_kernel(const __grid_constant__ DecodeArgs a) {
   asm volatile("griddepcontrol.wait;" ::: "memory");
   __shared__ float wsh[kMaxSplit];
   __shared__ float red[kCombineWarps][32];

@@ -351,6 +351,23 @@ namespace {
 // Queries at positions q_pos0 .. q_pos0 + nq - 1 (per batch entry) against the
 // true-position cache, each over keys [0, its position], with one G from the
 // longest range L = q_pos0 + nq: a decode step (nq = 1) or a prefill chunk.
+// The decode kernels' turn fractions (theta_i / (2 pi) as 64-bit binary
+// fractions) for the call's theta, map and length.
+void fill_decode_turns(DecodeArgs *a) {
+  const double turns_q64 = 0.15915494309189533577 * 18446744073709551616.0;  // 2^64 / (2 pi)
+  const double log_theta = std::log(static_cast<double>(a->theta));
+  for (int i = 0; i < a->D / 2; ++i) {
+    const double f = std::exp(-2.0 * static_cast<double>(i) / static_cast<double>(a->D) * log_theta);
+    const double factor =
+        a->interp ? interp_factor(f, a->L, a->w_pretrained, a->ramp_alpha, a->ramp_beta) : 1.0;
+    a->omega_qt[i] = static_cast<uint64_t>(std::llround(f * turns_q64));  // < 2^62
+    a->omega_qr[i] = static_cast<uint64_t>(std::llround(f * factor * turns_q64));
+    // (theta' - theta) / (2 pi) lies in (-1/(2 pi), 0]: inside int64 once scaled
+    a->omega_corr[i] = a->interp ? static_cast<uint64_t>(std::llround(f * (factor - 1.0) * turns_q64))
+                                 : a->omega_qt[i];
+  }
+}
+
 // Every host check of such a call except the workspace's; sets *L_out to the
 // key range q_pos0 + nq.  Makes no CUDA call.
 int check_cache_call(const void *q, const void *k_cache, const void *v_cache, const void *out,
@@ -424,6 +441,7 @@ int cache_attention(const void *q, const void *k_cache, const void *v_cache, voi
   a.ramp_alpha = ramp_alpha;
   a.ramp_beta = ramp_beta;
   decode_plan(B * nq, Hkv, L, &a.n_split, &a.chunk);
+  fill_decode_turns(&a);
   a.dev_error = dev->err;
   if (launch_decode(a, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return JL_ERR_CUDA;
   return JL_OK;

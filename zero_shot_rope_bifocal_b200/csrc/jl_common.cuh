@@ -199,6 +199,12 @@ struct DecodeArgs {
   int interp;  // remote map, as in PrefillArgs
   float ramp_alpha, ramp_beta;
   GroupDivider gdiv;  // floor(x / G) by multiplication
+  // Turns per position as 64-bit binary fractions (theta_i / (2 pi)), formed
+  // on the host: of the true query (omega_qt), of the remote query (at f(p)
+  // with theta_i, or at p with theta'_i under the interpolation map), and of
+  // the correction rotation per unit of Delta (theta_i, or theta'_i - theta_i,
+  // negative, in two's complement).
+  uint64_t omega_qt[64], omega_qr[64], omega_corr[64];
   unsigned int *dev_error;
 };
 
