@@ -277,7 +277,6 @@ decode_split_kernel(const __grid_constant__ DecodeArgs a) {
   const int g0 = chunk_id * kDecWarps;
   const int nh = min(kDecWarps, a.Hkv - g0);  // KV heads of this CTA = working warps
   const int p = a.q_pos0 + (bq - b * a.nq);  // this query's position; keys [0, p]
-  const int G = a.G;
   const int w0eff = BIFOCAL ? a.w0 : INT_MAX;
   const int j_begin = s * a.chunk;
   const int j_end = min(p + 1, j_begin + a.chunk);  // may be <= j_begin: an empty split

@@ -158,6 +158,12 @@ struct PrefillArgs {
   int interp;
   float ramp_alpha, ramp_beta;
   unsigned int *dev_error;
+  // Turns per position as 64-bit binary fractions, formed on the host by the
+  // key-pass launchers: theta_i / (2 pi) (omega_true), the remote map's
+  // (theta_i, or theta'_i under the interpolation map), and the correction
+  // rotation's per unit of Delta (theta_i, or theta'_i - theta_i, negative,
+  // in two's complement).
+  uint64_t omega_true[64], omega_remote[64], omega_corr[64];
 };
 
 // Rotates k into the two key operand arrays, copies v to its operand array

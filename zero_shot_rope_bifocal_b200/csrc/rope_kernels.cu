@@ -33,6 +33,8 @@
 // frequency) into shared memory and applies it to every head of that
 // position; channel pairs are (i, i + D/2), processed two pairs per thread
 // with BF16x2 loads and FP16x2 stores.
+#include <cmath>
+
 #include "jl_common.cuh"
 
 namespace jl {
@@ -63,35 +65,92 @@ __device__ __forceinline__ void store_bf16(__nv_bfloat16 *dst, int i, int half, 
   *reinterpret_cast<__nv_bfloat162 *>(dst + i + half) = __floats2bfloat162_rn(v.s0, v.s1);
 }
 
-// FP16 MMA operand; returns false if a value left the FP16 range.
-__device__ __forceinline__ bool store_f16(__half *dst, int i, int half, const Rot2 &v) {
-  const __half2 lo = __floats2half2_rn(v.r0, v.r1);
-  const __half2 hi = __floats2half2_rn(v.s0, v.s1);
-  *reinterpret_cast<__half2 *>(dst + i) = lo;
-  *reinterpret_cast<__half2 *>(dst + i + half) = hi;
-  return !(__hisinf(__low2half(lo)) | __hisinf(__high2half(lo)) | __hisinf(__low2half(hi)) |
-           __hisinf(__high2half(hi)));
+// Positions per CTA of the key passes; every position's (cos, sin) is formed
+// once and used by every KV head.
+constexpr int kKvPos = 16;
+constexpr float kTurnToRad = 1.4629180792671596e-09f;  // 2 pi / 2^32
+
+// cos / sin of the angle whose turns are (pos * omega) mod 1, exact in
+// 64-bit fixed point: the wrapping product's top 32 bits are the signed
+// phase, so the sine/cosine only sees [-pi, pi).
+__device__ __forceinline__ float2 turn_cos_sin(uint64_t pos, uint64_t omega) {
+  const int32_t ph = static_cast<int32_t>((pos * omega) >> 32);
+  float c, s;
+  __sincosf(static_cast<float>(ph) * kTurnToRad, &s, &c);
+  return make_float2(c, s);
 }
 
+// Eight channel pairs (c .. c+7 with partners c+D/2 ..) of a BF16 row,
+// loaded as two 16-byte vectors, turned by their (cos, sin) and returned as
+// FP32 (lo = channels c.., hi = partners).
+struct Rot8 {
+  float lo[8], hi[8];
+};
+__device__ __forceinline__ Rot8 rotate8(uint4 xa, uint4 xb, const float2 *cs) {
+  const uint32_t wa[4] = {xa.x, xa.y, xa.z, xa.w}, wb[4] = {xb.x, xb.y, xb.z, xb.w};
+  Rot8 r;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    const uint32_t ua = wa[e >> 1], ub = wb[e >> 1];
+    const float x = __uint_as_float((e & 1) ? (ua & 0xffff0000u) : (ua << 16));
+    const float y = __uint_as_float((e & 1) ? (ub & 0xffff0000u) : (ub << 16));
+    r.lo[e] = x * cs[e].x - y * cs[e].y;
+    r.hi[e] = x * cs[e].y + y * cs[e].x;
+  }
+  return r;
+}
+
+// Stores 8 values as FP16 (16 bytes); returns false if one left the FP16 range.
+__device__ __forceinline__ bool store8_f16(__half *dst, const float (&v)[8]) {
+  uint32_t w[4];
+  bool ok = true;
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const __half2 h = __floats2half2_rn(v[2 * e], v[2 * e + 1]);
+    ok &= !(__hisinf(__low2half(h)) | __hisinf(__high2half(h)));
+    w[e] = *reinterpret_cast<const uint32_t *>(&h);
+  }
+  *reinterpret_cast<uint4 *>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
+  return ok;
+}
+
+__device__ __forceinline__ void store8_bf16(__nv_bfloat16 *dst, const float (&v)[8]) {
+  uint32_t w[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(v[2 * e], v[2 * e + 1]);
+    w[e] = *reinterpret_cast<const uint32_t *>(&h);
+  }
+  *reinterpret_cast<uint4 *>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+// BF16 -> FP16 copy of 8 values (the values' operand); false if out of range.
+__device__ __forceinline__ bool copy8_f16(__half *dst, uint4 x) {
+  const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+  float v[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e)
+    v[e] = __uint_as_float((e & 1) ? (w[e >> 1] & 0xffff0000u) : (w[e >> 1] << 16));
+  return store8_f16(dst, v);
+}
+
+// Prefill key operands: for each position j of [16 blockIdx.x, +16) and KV
+// head g, k_true = RoPE(x_k, j), k_remote = RoPE(x_k, f(j)) (RoPE'(x_k, j)
+// under the interpolation map), v copied, all FP16 head-major, plus the
+// optional BF16 true-position cache.  Work item = (position, head, group of
+// 8 channels and their partners): 16-byte loads and stores.
 __global__ void __launch_bounds__(kRopeThreads)
-rope_kv_kernel(PrefillArgs a) {
-  extern __shared__ float2 cs_smem[];  // [2][kPosPerCta][D/2] (cos, sin), then 2 x [D/2] freq
+rope_kv_kernel(const __grid_constant__ PrefillArgs a) {
+  __shared__ float2 cs[2][kKvPos][64];  // (cos, sin): true, remote
+  __shared__ uint64_t om[2][64];
   const int half = a.D / 2;
   const int b = blockIdx.y;
-  const int p_begin = blockIdx.x * kPosPerCta;
-  const int npos = min(kPosPerCta, a.L - p_begin);
+  const int p_begin = blockIdx.x * kKvPos;
+  const int npos = min(kKvPos, a.L - p_begin);
   const bool two = a.G > 1;
-  float2 *cs_true = cs_smem;
-  float2 *cs_remote = cs_smem + kPosPerCta * half;
-
-  double *freq = reinterpret_cast<double *>(cs_smem + 2 * kPosPerCta * half);
-  double *freq_remote = freq + half;  // theta'_t (interpolation) or theta_t
-  const double theta = static_cast<double>(a.theta);
-  for (int i = threadIdx.x; i < half; i += blockDim.x) {
-    const double f = rope_freq(i, a.D, theta);
-    freq[i] = f;
-    freq_remote[i] =
-        a.interp ? f * interp_factor(f, a.L, a.w_pretrained, a.ramp_alpha, a.ramp_beta) : f;
+  if (threadIdx.x < half) {
+    om[0][threadIdx.x] = a.omega_true[threadIdx.x];
+    om[1][threadIdx.x] = a.omega_remote[threadIdx.x];
   }
   __syncthreads();
   for (int idx = threadIdx.x; idx < npos * half * (two ? 2 : 1); idx += blockDim.x) {
@@ -99,37 +158,39 @@ rope_kv_kernel(PrefillArgs a) {
     const int rem = idx - var * npos * half;
     const int t = rem / half, i = rem - t * half;
     const int pos = p_begin + t;
-    const long long ppos = (var == 0 || a.interp) ? pos : remap(pos, a.G);
-    float c, s;
-    rope_cos_sin(ppos, var == 0 ? freq[i] : freq_remote[i], c, s);
-    (var == 0 ? cs_true : cs_remote)[t * half + i] = make_float2(c, s);
+    const uint64_t pp = (var == 0 || a.interp) ? pos : remap(pos, a.G);
+    cs[var][t][i] = turn_cos_sin(pp, om[var][i]);
   }
   __syncthreads();
-
   bool in_range = true;
-  const int quarter = a.D / 4;  // pairs of channel pairs per head row
-  // keys (+ optional true-position cache) and values
-  for (int idx = threadIdx.x; idx < npos * a.Hkv * quarter; idx += blockDim.x) {
-    const int t = idx / (a.Hkv * quarter);
-    const int rem = idx - t * a.Hkv * quarter;
-    const int g = rem / quarter;
-    const int i = (rem - g * quarter) * 2;
+  const int c8n = a.D / 16;  // groups of 8 channel pairs per head row
+  for (int idx = threadIdx.x; idx < npos * a.Hkv * c8n; idx += blockDim.x) {
+    const int t = idx / (a.Hkv * c8n);
+    const int rem = idx - t * a.Hkv * c8n;
+    const int g = rem / c8n;
+    const int c = (rem - g * c8n) * 8;
     const int pos = p_begin + t;
     const size_t srow = ((static_cast<size_t>(b) * a.L + pos) * a.Hkv + g) * a.D;
-    const __nv_bfloat16 *src = a.k + srow;
     const size_t drow = ((static_cast<size_t>(b) * a.Hkv + g) * a.L + pos) * a.D;
-    const Rot2 kt = rotate2(src, i, half, cs_true[t * half + i], cs_true[t * half + i + 1]);
-    in_range &= store_f16(a.k_true + drow, i, half, kt);
-    if (two)
-      in_range &= store_f16(a.k_remote + drow, i, half,
-                            rotate2(src, i, half, cs_remote[t * half + i],
-                                    cs_remote[t * half + i + 1]));
-    if (a.k_cache_out)
-      store_bf16(a.k_cache_out + ((static_cast<size_t>(b) * a.k_cache_capacity + pos) * a.Hkv + g) * a.D,
-                 i, half, kt);
-    // values: the identity rotation, i.e. a BF16 -> FP16 copy into head-major order
-    in_range &= store_f16(a.v_op + drow, i, half,
-                          rotate2(a.v + srow, i, half, make_float2(1.f, 0.f), make_float2(1.f, 0.f)));
+    const uint4 ka = __ldg(reinterpret_cast<const uint4 *>(a.k + srow + c));
+    const uint4 kb = __ldg(reinterpret_cast<const uint4 *>(a.k + srow + c + half));
+    const Rot8 kt = rotate8(ka, kb, &cs[0][t][c]);
+    in_range &= store8_f16(a.k_true + drow + c, kt.lo);
+    in_range &= store8_f16(a.k_true + drow + c + half, kt.hi);
+    if (two) {
+      const Rot8 kr = rotate8(ka, kb, &cs[1][t][c]);
+      in_range &= store8_f16(a.k_remote + drow + c, kr.lo);
+      in_range &= store8_f16(a.k_remote + drow + c + half, kr.hi);
+    }
+    if (a.k_cache_out) {
+      __nv_bfloat16 *crow =
+          a.k_cache_out + ((static_cast<size_t>(b) * a.k_cache_capacity + pos) * a.Hkv + g) * a.D;
+      store8_bf16(crow + c, kt.lo);
+      store8_bf16(crow + c + half, kt.hi);
+    }
+    in_range &= copy8_f16(a.v_op + drow + c, __ldg(reinterpret_cast<const uint4 *>(a.v + srow + c)));
+    in_range &= copy8_f16(a.v_op + drow + c + half,
+                          __ldg(reinterpret_cast<const uint4 *>(a.v + srow + c + half)));
   }
   if (!in_range) atomicOr(a.dev_error, kDevRange);
 }
@@ -142,50 +203,52 @@ rope_kv_kernel(PrefillArgs a) {
 // Delta * theta_i; under the frequency-interpolation map the remote form is
 // RoPE'(x_k, j), i.e. the cached key turned by j * (theta'_i - theta_i).
 __global__ void __launch_bounds__(kRopeThreads)
-cache_kv_kernel(PrefillArgs a) {
-  extern __shared__ float2 cs_smem[];  // [kPosPerCta][D/2] (cos, sin), then [D/2] freq
+cache_kv_kernel(const __grid_constant__ PrefillArgs a) {
+  __shared__ float2 cs[kKvPos][64];  // (cos, sin) of the correction
+  __shared__ uint64_t om[64];
   const int half = a.D / 2;
   const int b = blockIdx.y;
-  const int j_begin = blockIdx.x * kPosPerCta;
-  const int npos = min(kPosPerCta, a.L - j_begin);
+  const int j_begin = blockIdx.x * kKvPos;
+  const int npos = min(kKvPos, a.L - j_begin);
   const bool two = a.G > 1;
-  double *freq = reinterpret_cast<double *>(cs_smem + kPosPerCta * half);
-  const double theta = static_cast<double>(a.theta);
-  for (int i = threadIdx.x; i < half; i += blockDim.x) {
-    const double f = rope_freq(i, a.D, theta);
-    // the correction's angle per unit of Delta: theta_i, or theta'_i - theta_i
-    freq[i] = a.interp ? f * (interp_factor(f, a.L, a.w_pretrained, a.ramp_alpha, a.ramp_beta) - 1.0)
-                       : f;
-  }
+  if (threadIdx.x < half) om[threadIdx.x] = a.omega_corr[threadIdx.x];
   __syncthreads();
   if (two) {
     for (int idx = threadIdx.x; idx < npos * half; idx += blockDim.x) {
       const int t = idx / half, i = idx - t * half;
       const int j = j_begin + t;
       const long long delta = a.interp ? j : static_cast<long long>(remap(j, a.G)) - j;
-      float c, s;
-      rope_cos_sin(delta, freq[i], c, s);
-      cs_smem[t * half + i] = make_float2(c, s);
+      cs[t][i] = turn_cos_sin(static_cast<uint64_t>(delta), om[i]);
     }
   }
   __syncthreads();
   bool in_range = true;
-  const int quarter = a.D / 4;
-  const float2 one = make_float2(1.f, 0.f);
-  for (int idx = threadIdx.x; idx < npos * a.Hkv * quarter; idx += blockDim.x) {
-    const int t = idx / (a.Hkv * quarter);
-    const int rem = idx - t * a.Hkv * quarter;
-    const int g = rem / quarter;
-    const int i = (rem - g * quarter) * 2;
+  const int c8n = a.D / 16;
+  const float2 one[8] = {make_float2(1.f, 0.f), make_float2(1.f, 0.f), make_float2(1.f, 0.f),
+                         make_float2(1.f, 0.f), make_float2(1.f, 0.f), make_float2(1.f, 0.f),
+                         make_float2(1.f, 0.f), make_float2(1.f, 0.f)};
+  for (int idx = threadIdx.x; idx < npos * a.Hkv * c8n; idx += blockDim.x) {
+    const int t = idx / (a.Hkv * c8n);
+    const int rem = idx - t * a.Hkv * c8n;
+    const int g = rem / c8n;
+    const int c = (rem - g * c8n) * 8;
     const int j = j_begin + t;
     const size_t srow = ((static_cast<size_t>(b) * a.cache_cap + j) * a.Hkv + g) * a.D;
     const size_t drow = ((static_cast<size_t>(b) * a.Hkv + g) * a.L + j) * a.D;
-    const __nv_bfloat16 *kc = a.k_cache_in + srow;
-    in_range &= store_f16(a.k_true + drow, i, half, rotate2(kc, i, half, one, one));
-    if (two)
-      in_range &= store_f16(a.k_remote + drow, i, half,
-                            rotate2(kc, i, half, cs_smem[t * half + i], cs_smem[t * half + i + 1]));
-    in_range &= store_f16(a.v_op + drow, i, half, rotate2(a.v_cache_in + srow, i, half, one, one));
+    const uint4 ka = __ldg(reinterpret_cast<const uint4 *>(a.k_cache_in + srow + c));
+    const uint4 kb = __ldg(reinterpret_cast<const uint4 *>(a.k_cache_in + srow + c + half));
+    const Rot8 kt = rotate8(ka, kb, one);
+    in_range &= store8_f16(a.k_true + drow + c, kt.lo);
+    in_range &= store8_f16(a.k_true + drow + c + half, kt.hi);
+    if (two) {
+      const Rot8 kr = rotate8(ka, kb, &cs[t][c]);
+      in_range &= store8_f16(a.k_remote + drow + c, kr.lo);
+      in_range &= store8_f16(a.k_remote + drow + c + half, kr.hi);
+    }
+    in_range &= copy8_f16(a.v_op + drow + c,
+                          __ldg(reinterpret_cast<const uint4 *>(a.v_cache_in + srow + c)));
+    in_range &= copy8_f16(a.v_op + drow + c + half,
+                          __ldg(reinterpret_cast<const uint4 *>(a.v_cache_in + srow + c + half)));
   }
   if (!in_range) atomicOr(a.dev_error, kDevRange);
 }
@@ -224,16 +287,33 @@ rope_cache_kernel(const __nv_bfloat16 *__restrict__ k, __nv_bfloat16 *__restrict
 
 }  // namespace
 
+// The key passes' turn fractions for the call's theta, map and length.
+static PrefillArgs with_turns(const PrefillArgs &a) {
+  PrefillArgs t = a;
+  const double turns_q64 = 0.15915494309189533577 * 18446744073709551616.0;  // 2^64 / (2 pi)
+  const double log_theta = std::log(static_cast<double>(a.theta));
+  for (int i = 0; i < a.D / 2; ++i) {
+    const double f = std::exp(-2.0 * static_cast<double>(i) / static_cast<double>(a.D) * log_theta);
+    const double factor =
+        a.interp ? interp_factor(f, a.L, a.w_pretrained, a.ramp_alpha, a.ramp_beta) : 1.0;
+    t.omega_true[i] = static_cast<uint64_t>(std::llround(f * turns_q64));  // < 2^62
+    t.omega_remote[i] = static_cast<uint64_t>(std::llround(f * factor * turns_q64));
+    // (theta' - theta) / (2 pi) lies in (-1/(2 pi), 0]: inside int64 once scaled
+    t.omega_corr[i] = a.interp ? static_cast<uint64_t>(std::llround(f * (factor - 1.0) * turns_q64))
+                               : t.omega_true[i];
+  }
+  return t;
+}
+
 cudaError_t launch_rope_kv(const PrefillArgs &a, cudaStream_t stream) {
-  const dim3 grid((a.L + kPosPerCta - 1) / kPosPerCta, a.B);
-  const size_t smem = 2 * kPosPerCta * (a.D / 2) * sizeof(float2) + 2 * (a.D / 2) * sizeof(double);
-  rope_kv_kernel<<<grid, kRopeThreads, smem, stream>>>(a);
+  const dim3 grid((a.L + kKvPos - 1) / kKvPos, a.B);
+  rope_kv_kernel<<<grid, kRopeThreads, 0, stream>>>(with_turns(a));
   return cudaGetLastError();
 }
 
 cudaError_t launch_chunk_operands(const PrefillArgs &a, cudaStream_t stream) {
-  const size_t smem_k = kPosPerCta * (a.D / 2) * sizeof(float2) + (a.D / 2) * sizeof(double);
-  cache_kv_kernel<<<dim3((a.L + kPosPerCta - 1) / kPosPerCta, a.B), kRopeThreads, smem_k, stream>>>(a);
+  const dim3 grid((a.L + kKvPos - 1) / kKvPos, a.B);
+  cache_kv_kernel<<<grid, kRopeThreads, 0, stream>>>(with_turns(a));
   return cudaGetLastError();
 }
 
