@@ -1,4 +1,5 @@
-// prefill_sm100.cu -- bifocal causal attention for a whole prompt on sm_100a.
+// prefill_sm100.cu -- bifocal causal attention for a whole prompt (or a chunk
+// of queries appended to a cache) on sm_100a.
 //
 // Method (Jet-Long paper): score rule of §3 (local pairs i - j <= w0 at true
 // positions, older pairs at the remapped positions f(i), f(j)), schedule of
@@ -7,38 +8,41 @@
 // picked by the rule; this kernel runs that single online softmax, visiting
 // each key tile with the operand variant(s) its pairs need:
 //
-//   * a "remote" visit of key tile kt uses (q_remote, k_remote) and keeps only
-//     the pairs with i - j > w0;
-//   * a "local" visit uses (q_true, k_true) and keeps pairs with
-//     0 <= i - j <= w0 (causal).
+//   * a "remote" visit of key tile kt uses the query tile rotated to remote
+//     positions and k_remote, and keeps only the pairs with i - j > w0;
+//   * a "local" visit uses the query tile at true positions and k_true, and
+//     keeps pairs with 0 <= i - j <= w0 (causal).
 //
 // Tiles that straddle the window edge are visited twice, once per variant,
 // each with its complementary mask, so every pair is counted exactly once and
 // nothing is subtracted (no cancellation).  For one 128-row query tile the
 // remote visits form a prefix of the key tiles and the local visits a suffix,
-// so the query operand switches from q_remote to q_true exactly once.  With
-// G == 1 (L <= w_pretrained) f is the identity and every tile is a plain
+// so the query tile switches from remote to true positions exactly once.
+// With G == 1 (L <= w_pretrained) f is the identity and every tile is a plain
 // causal "local" visit: the native-window case of Appendix H.
 //
-// Operands: the RoPE pass leaves q/k (both variants) and v in the workspace as
-// FP16, head-major [B, H, L, D].  FP16 keeps three more mantissa bits than
-// BF16 for the rotated values the tensor core must consume in 16 bits.
+// Operands: RoPE runs in the Q load path -- the softmax threads turn the
+// BF16 queries into the FP16 query tile in shared memory (build_q_row) -- and
+// the key pass leaves k at true and remote positions and v in the workspace
+// as FP16, head-major [B, Hkv, L, D], since every key tile is read by every
+// query tile of its head.  FP16 keeps three more mantissa bits than BF16 for
+// the rotated values the tensor core must consume in 16 bits.
 //
 // CTA = two 128-row query tiles of the same 128 positions, for two query
 // heads of one KV group (GQA packing: each K/V tile staged in shared memory
 // serves 256 query rows).  Warp-specialised, 10 warps:
 //   * warps 0-3 / 4-7: softmax for query tile 0 / 1, one thread per row (a
-//     TMEM lane).  A thread holds its row's 128 scores in registers: one TMEM
-//     read, the row max, the exponentials, P stored back, with no exchange
-//     between threads; it rescales its O row when the max grows and runs the
-//     epilogue of its row;
-//   * warp 8: TMA producer (queries once per variant, K and V tiles through
-//     a four-slot ring);
+//     TMEM lane).  A thread builds its row of the query tile, holds its row's
+//     128 scores in registers: one TMEM read, the row max, the exponentials,
+//     P stored back, with no exchange between threads; it rescales its O row
+//     when the max grows and runs the epilogue of its row;
+//   * warp 8: TMA producer of the K and V tiles through a four-slot ring;
 //   * warp 9: tcgen05.mma issuer, in the order
 //       S0(j+1) = Q0 K(j+1)^T after O0 += P0(j) V(j), and likewise for tile 1,
 //     so the tensor core works on one tile while the other tile's softmax
 //     runs.
-// Ten warps leave up to 200 registers per thread, which holds a whole row.
+// Ten warps put three on two of the four SM sub-partitions, whose register
+// files then allow 168 registers per thread: enough for a whole row.
 // TMEM (512 columns): S0 | S1 | O0 | O1; a row's P (packed FP16) is written
 // over the first 64 columns of its S once the scores are in registers.
 // Each wait is bounded in time (jl::kWaitLimitNs) and also gives up when
