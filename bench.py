@@ -51,11 +51,11 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # DRAM bytes (read + write) of one attention-kernel launch at the headline
 # workload, from an ncu capture (dram__bytes_read.sum + dram__bytes_write.sum)
 # of the kernel's own sources (its device code and the PTX wrappers it uses),
-# whose SHA-256 is recorded here; the capture and its command are summarised
+# whose code lines' SHA-256 is recorded here; the capture and its command are summarised
 # in the profile named below.  The line reports it only while those sources
 # are unchanged, and null otherwise.
 TRAFFIC_RECORD = {"bytes": 6.12e9, "read_bytes": 4.98e9, "write_bytes": 1.14e9,
-                  "sources_sha256": "833d188279f620c457fc1f51348fa4b0e03d886edc149d74a3243e0aa8f88447",
+                  "sources_sha256": "be874d6a4e54b063be8a6c5edb7649ae723aa5d0461a3f55db0d7837e40b85b1",
                   "profile": "profiles/prefill_attention_qwen3_8b_L131072_dram.md"}
 TRAFFIC_SOURCES = ("zero_shot_rope_bifocal_b200/csrc/prefill_sm100.cu",
                    "zero_shot_rope_bifocal_b200/csrc/sm100_ptx.cuh")
@@ -85,11 +85,16 @@ def decode_bytes(B: int, Hkv: int, L: int, D: int) -> int:
 
 
 def kernel_sources_sha256() -> str:
+    """SHA-256 of the kernel sources' code lines (comment-only lines and
+    blank lines left out, so that a comment edit keeps the record)."""
     import hashlib
     h = hashlib.sha256()
     for rel in TRAFFIC_SOURCES:
-        with open(os.path.join(ROOT, rel), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, rel), encoding="utf-8") as fh:
+            for line in fh:
+                t = line.strip()
+                if t and not t.startswith("//"):
+                    h.update(t.encode() + b"\n")
     return h.hexdigest()
 
 
