@@ -128,3 +128,20 @@ def test_oracle_rate_extras():
     x = bench.oracle_rate_extras(w, full / 1000.0, 2.0, [5, 6, 7, 8])
     assert x["rows_per_s"] == 2.0
     assert abs(x["extrapolated_full_prefill_s"] - 2000.0) < 1e-6
+
+
+def test_traffic_record_follows_the_kernel_code_not_its_comments(tmp_path, monkeypatch):
+    import bench
+    src = tmp_path / "k.cu"
+    src.write_text("// a comment\n__global__ void k() {}\n")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    monkeypatch.setattr(bench, "TRAFFIC_SOURCES", ("k.cu",))
+    sha = bench.kernel_sources_sha256()
+    monkeypatch.setattr(bench, "TRAFFIC_RECORD", {"bytes": 5.0, "sources_sha256": sha,
+                                                  "profile": "p.md"})
+    assert bench.measured_traffic() == (5.0, "p.md")
+    src.write_text("// another comment\n\n__global__ void k() {}\n")  # comments only
+    assert bench.measured_traffic() == (5.0, "p.md")
+    src.write_text("// a comment\n__global__ void k() { int x = 1; }\n")  # code changed
+    assert bench.measured_traffic()[0] is None
+
