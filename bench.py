@@ -55,7 +55,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # in the profile named below.  The line reports it only while those sources
 # are unchanged, and null otherwise.
 TRAFFIC_RECORD = {"bytes": 6.12e9, "read_bytes": 4.98e9, "write_bytes": 1.14e9,
-                  "sources_sha256": "be874d6a4e54b063be8a6c5edb7649ae723aa5d0461a3f55db0d7837e40b85b1",
+                  "sources_sha256": "f79d1e483ed80ccdc36ef9456c9571bc1f72921f63c5943ae50a9ef765d06e52",
                   "profile": "profiles/prefill_attention_qwen3_8b_L131072_dram.md"}
 TRAFFIC_SOURCES = ("zero_shot_rope_bifocal_b200/csrc/prefill_sm100.cu",
                    "zero_shot_rope_bifocal_b200/csrc/sm100_ptx.cuh")

@@ -36,7 +36,9 @@
 //     128 scores in registers: one TMEM read, the row max, the exponentials,
 //     P stored back, with no exchange between threads; it rescales its O row
 //     when the max grows and runs the epilogue of its row;
-//   * warp 8: TMA producer of the K and V tiles through a four-slot ring;
+//   * warp 8: TMA producer of the K and V tiles through a ring of two
+//     two-tile units, unit u holding V(u-1) and K(u): the pair the MMA
+//     issuer uses in the same visit, so one wait and one release per visit;
 //   * warp 9: tcgen05.mma issuer, in the order
 //       S0(j+1) = Q0 K(j+1)^T after O0 += P0(j) V(j), and likewise for tile 1,
 //     so the tensor core works on one tile while the other tile's softmax
@@ -58,7 +60,7 @@ namespace {
 
 constexpr int BM = 128;  // query rows per tile (= TMEM lanes)
 constexpr int BN = 128;  // keys per tile
-constexpr int NS = 4;    // K/V ring slots (one K or V tile each)
+constexpr int NU = 2;    // K/V ring units of two tiles: unit u = V(u-1), K(u)
 constexpr int kSoftmaxWarps = 8;  // 2 warpgroups: one per query tile
 constexpr int kWarps = 10;
 constexpr int kThreads = kWarps * 32;
@@ -79,11 +81,11 @@ struct Layout {
   static constexpr int BOX = 128 * 128;    // bytes of one 128-row x 64-col swizzled box
   static constexpr int Q0 = 0;
   static constexpr int RING = 2 * TILE;
-  static constexpr int BAR = RING + NS * TILE;
+  static constexpr int BAR = RING + 2 * NU * TILE;
   // barrier indices (8 bytes each)
-  static constexpr int kQFull = 0, kKvFull = 4, kKvEmpty = 4 + NS,
-                       kSFull = 4 + 2 * NS, kPFull = 6 + 2 * NS, kOFull = 8 + 2 * NS,
-                       kDrain = 10 + 2 * NS, kNumBars = 11 + 2 * NS;
+  static constexpr int kQFull = 0, kKvFull = 4, kKvEmpty = 4 + NU,
+                       kSFull = 4 + 2 * NU, kPFull = 6 + 2 * NU, kOFull = 8 + 2 * NU,
+                       kDrain = 10 + 2 * NU, kNumBars = 11 + 2 * NU;
   static constexpr int TMEM_SLOT = BAR + 8 * kNumBars;
   static constexpr int ABORT = TMEM_SLOT + 4;
   static constexpr int SKIP = TMEM_SLOT + 8;
@@ -321,38 +323,46 @@ bifocal_prefill_kernel(const __grid_constant__ CUtensorMap tm_kt,
   if (warp >= kSoftmaxWarps) {
     if (warp == kProducerWarp && lane == 0) {
       // ---------------------------------------------------------- producer
-      int r = 0;
+      // Unit u holds V(u-1) in its first tile and K(u) in its second (unit 0
+      // only K(0), unit nv only V(nv-1)): the pair the MMA issuer uses
+      // together in visit u-1 (O += P V(u-1), then S = Q K(u)^T).
       bool ok = true;
-      uint32_t issued[NS] = {0, 0, 0, 0};  // uses issued per slot
-      for (int j = 0; j < nv && ok; ++j) {
-        const bool remote = j < n_rem;
-        const int kt = remote ? kr0 + j : kl0 + (j - n_rem);
-        for (int part = 0; part < 2 && ok; ++part, ++r) {
-          const int slot = r % NS;
-          const uint32_t use = static_cast<uint32_t>(r / NS);
-          ok = wait_or_abort(bar(LY::kKvEmpty + slot), (use & 1u) ^ 1u, abort);
-          if (!ok) break;
-          const uint32_t dst = sb + LY::RING + slot * LY::TILE;
-          mbar_arrive_expect_tx(bar(LY::kKvFull + slot), LY::TILE);
-          const CUtensorMap *tm = part == 0 ? (remote ? &tm_kr : &tm_kt) : &tm_v;
+      uint32_t issued[NU] = {0, 0};  // uses issued per unit slot
+      for (int u = 0; u <= nv && ok; ++u) {
+        const int slot = u % NU;
+        const uint32_t use = static_cast<uint32_t>(u / NU);
+        ok = wait_or_abort(bar(LY::kKvEmpty + slot), (use & 1u) ^ 1u, abort);
+        if (!ok) break;
+        const uint32_t dst = sb + LY::RING + slot * 2 * LY::TILE;
+        const bool has_v = u > 0, has_k = u < nv;
+        mbar_arrive_expect_tx(bar(LY::kKvFull + slot), (has_v + has_k) * LY::TILE);
+        auto kt_of = [&](int visit) {
+          return visit < n_rem ? kr0 + visit : kl0 + (visit - n_rem);
+        };
+        if (has_v)
           for (int c = 0; c < NBOX; ++c)
-            tma_load_3d(dst + c * LY::BOX, tm, bar(LY::kKvFull + slot), c * 64, kt * BN,
-                        b * prm.Hkv + g);
-          issued[slot] = use + 1;
+            tma_load_3d(dst + c * LY::BOX, &tm_v, bar(LY::kKvFull + slot), c * 64,
+                        kt_of(u - 1) * BN, b * prm.Hkv + g);
+        if (has_k) {
+          const CUtensorMap *tm = u < n_rem ? &tm_kr : &tm_kt;
+          for (int c = 0; c < NBOX; ++c)
+            tma_load_3d(dst + LY::TILE + c * LY::BOX, tm, bar(LY::kKvFull + slot), c * 64,
+                        kt_of(u) * BN, b * prm.Hkv + g);
         }
+        issued[slot] = use + 1;
       }
       if (!ok) {
         // Let copies already in flight land before the CTA exits (bounded).
-        for (int s = 0; s < NS; ++s)
+        for (int s = 0; s < NU; ++s)
           if (issued[s] > 0) mbar_wait_bounded(bar(LY::kKvFull + s), (issued[s] - 1u) & 1u, kWaitLimitNs);
       }
     } else if (warp == kMmaWarp && lane == 0) {
       // ---------------------------------------------------------- MMA issuer
-      auto qk = [&](int s, uint32_t kslot) {
+      auto qk = [&](int s, uint32_t kaddr) {
         // descriptors of k-step 0; step kk moves the start address by off(kk)
         // (the address field holds addr >> 4 in its low bits)
         const uint64_t dq = smem_desc_sw128(sb + LY::Q0 + s * LY::TILE, 16, 1024);
-        const uint64_t dk = smem_desc_sw128(sb + LY::RING + kslot * LY::TILE, 16, 1024);
+        const uint64_t dk = smem_desc_sw128(kaddr, 16, 1024);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint64_t off = static_cast<uint64_t>(((kk >> 2) * LY::BOX + (kk & 3) * 32) >> 4);
@@ -360,67 +370,59 @@ bifocal_prefill_kernel(const __grid_constant__ CUtensorMap tm_kt,
         }
         mma_commit(bar(LY::kSFull + s));
       };
-      auto pv = [&](int s, uint32_t vslot, bool acc) {
-        const uint64_t dv = smem_desc_sw128(sb + LY::RING + vslot * LY::TILE, LY::BOX, 1024);
+      auto pv = [&](int s, uint32_t vaddr, bool acc) {
+        const uint64_t dv = smem_desc_sw128(vaddr, LY::BOX, 1024);
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk)  // P of keys [16kk, 16kk+16): columns [8kk, 8kk+8)
           mma_f16kind_ts(tO(s), tS(s) + kk * 8,
                          dv + static_cast<uint64_t>((kk * 16 * 128) >> 4), IDESC_PV,
                          (acc || kk > 0) ? 1u : 0u);
       };
+      auto unit_addr = [&](int u) { return sb + LY::RING + (u % NU) * 2 * LY::TILE; };
+      auto unit_wait = [&](int u) {
+        return wait_or_abort(bar(LY::kKvFull + u % NU), static_cast<uint32_t>(u / NU) & 1u, abort);
+      };
       bool ok = wait_or_abort(bar(LY::kQFull + 0), 0u, abort);
       if (ok && has1) ok = wait_or_abort(bar(LY::kQFull + 1), 0u, abort);
-      int r = 0;
-      // visit 0: S0, S1
-      int kslot = 0;
-      if (ok) {
-        kslot = r % NS;
-        ok = wait_or_abort(bar(LY::kKvFull + kslot), static_cast<uint32_t>(r / NS) & 1u, abort);
-        ++r;
-      }
+      // visit 0: S0, S1 from unit 0 (K(0))
+      if (ok) ok = unit_wait(0);
       if (ok) {
         tc_fence_after();
-        qk(0, kslot);
-        if (has1) qk(1, kslot);
-        mma_commit(bar(LY::kKvEmpty + kslot));
+        qk(0, unit_addr(0) + LY::TILE);
+        if (has1) qk(1, unit_addr(0) + LY::TILE);
+        mma_commit(bar(LY::kKvEmpty + 0));
       }
       for (int j = 0; j < nv && ok; ++j) {
-        const int vslot = r % NS;
-        ok = wait_or_abort(bar(LY::kKvFull + vslot), static_cast<uint32_t>(r / NS) & 1u, abort);
-        ++r;
+        // unit j+1: V(j) and (if more) K(j+1)
+        ok = unit_wait(j + 1);
         if (!ok) break;
+        const uint32_t va = unit_addr(j + 1), ka = va + LY::TILE;
         // tile 0: O0 += P0(j) V(j), then S0(j+1)
         ok = wait_or_abort(bar(LY::kPFull + 0), static_cast<uint32_t>(j) & 1u, abort);
         if (!ok) break;
         tc_fence_after();
-        pv(0, vslot, j > 0);
+        pv(0, va, j > 0);
         const bool more = j + 1 < nv;
         if (more) {
-          kslot = r % NS;
-          ok = wait_or_abort(bar(LY::kKvFull + kslot), static_cast<uint32_t>(r / NS) & 1u, abort);
-          ++r;
-          if (ok && switch_q && j + 1 == n_rem) ok = wait_or_abort(bar(LY::kQFull + 0), 1u, abort);
+          if (switch_q && j + 1 == n_rem) ok = wait_or_abort(bar(LY::kQFull + 0), 1u, abort);
           if (!ok) break;
           tc_fence_after();
-          qk(0, kslot);
+          qk(0, ka);
         }
         // tile 1: O1 += P1(j) V(j), then S1(j+1)
         if (has1) {
           ok = wait_or_abort(bar(LY::kPFull + 1), static_cast<uint32_t>(j) & 1u, abort);
           if (!ok) break;
           tc_fence_after();
-          pv(1, vslot, j > 0);
-        }
-        mma_commit(bar(LY::kKvEmpty + vslot));
-        if (more) {
-          if (has1) {
+          pv(1, va, j > 0);
+          if (more) {
             if (switch_q && j + 1 == n_rem) ok = wait_or_abort(bar(LY::kQFull + 1), 1u, abort);
             if (!ok) break;
             tc_fence_after();
-            qk(1, kslot);
+            qk(1, ka);
           }
-          mma_commit(bar(LY::kKvEmpty + kslot));
         }
+        mma_commit(bar(LY::kKvEmpty + (j + 1) % NU));
       }
       if (ok) {
         mma_commit(bar(LY::kOFull + 0));
