@@ -725,10 +725,11 @@ def run_native(args):
     if jl.jetlong_device_status() != jl.JL_OK:
         raise RuntimeError("device status not OK after the two-form decode")
 
-    # prefill chunks of 16, 64 and 4096 tokens closing the same 128K cache
-    # (below 24 tokens the decode kernels run them, from 24 the prefill kernel)
+    # prefill chunks of 4 to 4096 tokens closing the same 128K cache (below
+    # CHUNK_TENSOR_MIN tokens the decode kernels run them, from there on the
+    # prefill kernel, its keys split across CTAs while the query tiles are few)
     chunks = []
-    for n_chunk in (16, 64, 4096):
+    for n_chunk in (4, 16, 64, 1024, 4096):
         P0 = wd.L - n_chunk
         cq = torch.randn((wd.B, n_chunk, wd.Hq, wd.D), device=dev).to(torch.bfloat16)
         cout = torch.empty((wd.B, n_chunk, wd.Hq, wd.D), dtype=torch.bfloat16, device=dev)
@@ -758,7 +759,7 @@ def run_native(args):
         pairs = n_chunk * P0 + n_chunk * (n_chunk + 1) // 2  # causal (query, key) pairs
         chunks.append({"n": n_chunk, "P0": P0, "ms": chunk_ms,
                        "us_per_query": 1e3 * chunk_ms / n_chunk,
-                       "path": "decode kernels" if n_chunk < 24 else "prefill kernel",
+                       "path": "decode kernels" if n_chunk < jl.CHUNK_TENSOR_MIN else "prefill kernel",
                        "tflops": 4 * wd.B * wd.Hq * wd.D * pairs / (chunk_ms * 1e-3) / 1e12})
         del cq, cout, clse, cws
 

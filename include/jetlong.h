@@ -93,6 +93,12 @@ typedef enum {
 
 typedef enum { JL_BF16 = 0, JL_F32 = 1 } jl_dtype;
 
+/* A prefill chunk of at least this many queries runs on the tensor-core
+ * prefill kernel, a shorter one on the decode kernels (jetlong_prefill_chunk). */
+#ifndef JL_CHUNK_TENSOR_MIN
+#define JL_CHUNK_TENSOR_MIN 6
+#endif
+
 /* Human-readable name of a status code (static string, never NULL). */
 JL_API const char *jetlong_status_string(int status);
 
@@ -217,19 +223,24 @@ JL_API int jetlong_prefill_three_pass(const void *q, const void *k, const void *
  * p = P0 + i and sees keys [0, p]: local keys (p - j <= w0) as cached,
  * older keys turned by the correction rotation R(f(j) - j) and scored
  * against RoPE(x_q, f(p)).  With P0 = 0 and n = L this equals jetlong_prefill
- * on the same data.  Two execution paths, chosen by n alone:
- *   - n < 24: the split-KV decode kernels (a chunk is n decode problems over
- *     one cache; cost grows with n * L);
- *   - n >= 24: the tensor-core prefill kernel.  A pass first writes the
- *     chunk's operands into the workspace (queries rotated to their true and
- *     remote positions, and the cached keys of [0, P0 + n), as stored and
- *     turned by R(f(j) - j), with the values, as FP16); 128-row query tiles
- *     then run the same kernel as jetlong_prefill.  The cost is one pass over
- *     the cache plus the tensor-core work of n * L pairs; the FP16 range
- *     contract above applies to this path.
+ * on the same data.  Two execution paths, chosen by n alone
+ * (JL_CHUNK_TENSOR_MIN, above):
+ *   - n < JL_CHUNK_TENSOR_MIN: the split-KV decode kernels (a chunk is n
+ *     decode problems over one cache; cost grows with n * L);
+ *   - n >= JL_CHUNK_TENSOR_MIN: the tensor-core prefill kernel.  A pass first writes the
+ *     cached keys of [0, P0 + n), as stored and turned by R(f(j) - j), and
+ *     the values into the workspace as FP16; 128-row query tiles then run
+ *     the same kernel as jetlong_prefill, which rotates the chunk's queries
+ *     as it loads them.  When the chunk has too few query tiles to fill the
+ *     GPU (fewer than 75 tile x head-pair units), each tile's key tiles are
+ *     split into up to 148 / units contiguous ranges, one CTA each, whose
+ *     partial results a log-sum-exp merge combines.  The cost is one pass
+ *     over the cache plus the tensor-core work of n * L pairs; the FP16
+ *     range contract above applies to this path.
  * jetlong_prefill_chunk_workspace_size returns the size the chosen path needs
- * (for n >= 24, 2 x B.Hq.n.D + 3 x B.Hkv.(P0+n).D FP16 values, each array
- * 256-byte aligned).
+ * (tensor-core path: 3 x B.Hkv.(P0+n).D FP16 values, plus, when the keys are
+ * split into S > 1 ranges, B.n.Hq.S.(D + 2) float32 partial records; each
+ * array 256-byte aligned).
  *
  *   q       [B, n, Hq, D] BF16 pre-RoPE queries of the chunk (read)
  *   k_cache [B, Lcap, Hkv, D] BF16, RoPE at true positions, rows [0, P0+n)

@@ -186,6 +186,32 @@ def test_chunk_workspace_covers_a_decode_step():
     assert jl.jetlong_prefill_chunk_workspace_size(1, 32, 8, 0, 0, 128) == 0
 
 
+def test_chunk_threshold_matches_the_header():
+    m = re.search(r"#define JL_CHUNK_TENSOR_MIN (\d+)", open(HEADER).read())
+    assert m and int(m.group(1)) == jl.CHUNK_TENSOR_MIN
+
+
+def test_chunk_workspace_holds_the_split_records():
+    # tensor-core chunk path: the three FP16 key-operand arrays, then fp32
+    # partial records [B, n, Hq, S, D + 2] when the keys are split into S
+    # ranges (fewer than 75 query-tile x head-pair units; S = 148 / units,
+    # at most the first tile's key tiles and 65535 / B), each 256-byte aligned
+    al = lambda x: -(-x // 256) * 256
+    for B, Hq, Hkv, P0, n, D in ((1, 32, 8, 131008, 64, 128), (1, 32, 8, 126976, 4096, 128),
+                                 (1, 4, 1, 1000, 30, 64), (2, 16, 8, 300, 6, 128),
+                                 (1, 8, 8, 0, 6, 64)):
+        units = -(-n // 128) * Hkv * ((Hq // Hkv + 1) // 2) * B
+        S = 1 if 2 * units > 148 else min(148 // units, (min(P0 + 128, P0 + n) - 1) // 128 + 1,
+                                          65535 // B)
+        rec = al(B * n * Hq * S * (D + 2) * 4) if S > 1 else 0
+        want = 3 * al(B * Hkv * (P0 + n) * D * 2) + rec
+        assert jl.jetlong_prefill_chunk_workspace_size(B, Hq, Hkv, P0, n, D) == want, (B, P0, n)
+    # below the threshold a chunk is n decode problems: the decode plan's records
+    n = jl.CHUNK_TENSOR_MIN - 1
+    assert (jl.jetlong_prefill_chunk_workspace_size(1, 32, 8, 5000, n, 128) ==
+            jl.jetlong_decode_workspace_size(n, 32, 8, 5000 + n, 128))
+
+
 def decode_call(lib, **kw):
     a = dict(q=P, kc=P, vc=P, out=P, lse=None, B=1, Hq=32, Hkv=8, L=1000, Lcap=1000, D=128,
              wp=32768, w0=4096, theta=1e6, od=0, ws=P, wsb=1 << 40, stream=None)

@@ -54,6 +54,24 @@ def test_chunk_shapes(B, Hq, Hkv, D, wp, w0, P0, n):
     assert_lse(f64(lse), lse_ref, "chunk shapes")
 
 
+@pytest.mark.parametrize("Hq,Hkv,D,wp,w0,P0,n", [
+    (4, 1, 64, 1024, 300, 2900, 100),   # G = 3: 24 splits of ~27 visits; splits remote-only,
+                                        # local-only, and across the remote-to-local switch
+    (4, 2, 128, 4096, 200, 2000, 129),  # G = 1 (plain causal), two query tiles, ragged tail
+    (2, 2, 64, 512, 0, 1800, 7),        # w0 = 0, a chunk just above the path threshold
+    (8, 2, 128, 256, 1000, 1500, 40),   # w0 beyond most of the chunk's keys: few remote tiles
+])
+def test_chunk_key_split_every_row(Hq, Hkv, D, wp, w0, P0, n):
+    # Short chunks on the tensor path split each query tile's key visits
+    # into ranges (one CTA each) merged by log-sum-exp; every row against the
+    # oracle.
+    assert n >= jl.CHUNK_TENSOR_MIN
+    w = Workload("chunk_split", 1, Hq, Hkv, D, 0, wp, w0, 1e6, 61 + n, False, kind="decode")
+    out, lse, o_ref, lse_ref = run_chunk(w, P0, n)
+    assert_o(f64(out), o_ref, "key split")
+    assert_lse(f64(lse), lse_ref, "key split")
+
+
 def test_chunk_across_the_appendix_e_boundary_uses_one_group_size():
     # P0 + n = 98,308: G = 4 for every query of the chunk, although a
     # token-by-token decode would use G = 3 for the first four of them.
@@ -95,9 +113,10 @@ def test_qwen3_8b_long_chunk_at_128k_sampled_rows():
     assert torch.isfinite(out).all() and torch.isfinite(lse).all()
 
 
-@pytest.mark.parametrize("n", [23, 24])
+@pytest.mark.parametrize("n", [jl.CHUNK_TENSOR_MIN - 1, jl.CHUNK_TENSOR_MIN, 23, 24])
 def test_chunks_on_both_sides_of_the_path_threshold(n):
-    # 23 queries run on the decode kernels, 24 on the prefill kernel: the same
+    # n below the threshold runs on the decode kernels, n at or above it on the
+    # prefill kernel (with the keys split: one query tile here): the same
     # cache, both against the oracle
     w = Workload("chunk_thr", 1, 8, 2, 128, 0, 1024, 300, 1e6, 51, True, kind="decode")
     out, lse, o_ref, lse_ref = run_chunk(w, 5000 - n, n)

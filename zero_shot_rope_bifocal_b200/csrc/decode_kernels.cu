@@ -781,6 +781,28 @@ cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t stream) {
   return launch_decode_d<64>(a, stream);
 }
 
+cudaError_t launch_split_merge(const float *partial, int n_split, void *out, int out_f32,
+                               float *lse, int B, int nq, int Hq, int D, cudaStream_t stream) {
+  if (n_split < 1 || n_split > kMaxSplit) return cudaErrorInvalidValue;
+  DecodeArgs a{};
+  a.partial = const_cast<float *>(partial);
+  a.n_split = n_split;
+  a.out = out;
+  a.out_f32 = out_f32;
+  a.lse = lse;
+  a.B = B;
+  a.nq = nq;
+  a.Hq = Hq;
+  a.D = D;
+  // a plain launch: the dependency wait at the top of the merge returns at once
+  const dim3 grid(static_cast<unsigned>(B * nq * Hq), D / 32);
+  if (D == 128)
+    decode_combine_kernel<128><<<grid, kCombineThreads, 0, stream>>>(a);
+  else
+    decode_combine_kernel<64><<<grid, kCombineThreads, 0, stream>>>(a);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_remote_cache(const __nv_bfloat16 *k_cache, __half *k_remote, int B, int Lcap,
                                 int Hkv, int D, int j0, int j1, int G, float theta,
                                 cudaStream_t stream) {

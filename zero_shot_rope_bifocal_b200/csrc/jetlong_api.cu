@@ -4,6 +4,7 @@
 // Every check runs on the host before the first CUDA call, so an invalid call
 // returns its status without touching the device (and works on a machine with
 // no GPU at all).
+#include <algorithm>
 #include <cmath>
 #include <mutex>
 
@@ -447,24 +448,42 @@ int cache_attention(const void *q, const void *k_cache, const void *v_cache, voi
   return JL_OK;
 }
 
-// A chunk of at least this many queries runs on the tensor-core prefill
-// kernel (operands rotated once, then 128-row query tiles); shorter chunks run
-// on the decode kernels, one split-KV problem per query.
-#ifndef JL_CHUNK_TENSOR_MIN
-#define JL_CHUNK_TENSOR_MIN 24
-#endif
+// A chunk of at least JL_CHUNK_TENSOR_MIN queries (include/jetlong.h) runs on
+// the tensor-core prefill kernel (key operands converted once, 128-row query
+// tiles, the keys split when the tiles are few); shorter chunks run on the
+// decode kernels, one split-KV problem per query, whose cost is n passes over
+// the cache: on a 128K cache the two meet at about 5 queries.
 constexpr int kChunkTensorMin = JL_CHUNK_TENSOR_MIN;
+
+// Key split of the tensor-core chunk path: a chunk of few query tiles would
+// leave most SMs idle (one CTA per SM, each walking all of its tile's key
+// tiles), so each tile's visits are split into ranges, one CTA each, up to one
+// wave of 148 CTAs, and merged by log-sum-exp.  Every split keeps at least one
+// visit: the first query tile visits at least (its last position) / 128 + 1
+// key tiles under the fused rule.
+int chunk_split_count(int B, int Hq, int Hkv, int P0, int n) {
+  constexpr int kSms = 148;
+  const long long ctas = static_cast<long long>((n + 127) / 128) * Hkv * ((Hq / Hkv + 1) / 2) * B;
+  if (ctas * 2 > kSms) return 1;
+  int ns = static_cast<int>(kSms / ctas);
+  ns = std::min(ns, (std::min(P0 + 128, P0 + n) - 1) / 128 + 1);
+  ns = std::min(ns, static_cast<int>(kMaxGridYZ / B));
+  return std::max(ns, 1);
+}
 
 // Workspace of the tensor-core chunk path: the FP16 key operands, cached
 // keys in both forms and values [B, Hkv, P0 + n, D] (the kernel rotates the
-// chunk's queries as it loads them).
-size_t chunk_tensor_ws_bytes(int B, int Hkv, int P0, int n, int D) {
+// chunk's queries as it loads them), then the split records
+// [B, n, Hq, n_split, D + 2] fp32 when the keys are split.
+size_t chunk_tensor_ws_bytes(int B, int Hq, int Hkv, int P0, int n, int D) {
   const size_t k = align_up(static_cast<size_t>(B) * Hkv * (static_cast<size_t>(P0) + n) * D * 2);
-  return 3 * k;
+  const int ns = chunk_split_count(B, Hq, Hkv, P0, n);
+  const size_t rec = ns > 1 ? align_up(static_cast<size_t>(B) * n * Hq * ns * (D + 2) * 4) : 0;
+  return 3 * k + rec;
 }
 
 size_t chunk_ws_bytes(int B, int Hq, int Hkv, int P0, int n, int D) {
-  return n >= kChunkTensorMin ? chunk_tensor_ws_bytes(B, Hkv, P0, n, D)
+  return n >= kChunkTensorMin ? chunk_tensor_ws_bytes(B, Hq, Hkv, P0, n, D)
                               : decode_ws_bytes(B * n, Hq, Hkv, P0 + n, D);
 }
 
@@ -484,7 +503,7 @@ int chunk_tensor(const void *q, const void *k_cache, const void *v_cache, void *
   // grids: (query tiles, KV heads x head pairs, batch) and (positions, batch)
   if (B > kMaxGridYZ || static_cast<long long>(Hkv) * ((Hq / Hkv + 1) / 2) > kMaxGridYZ)
     return JL_ERR_SHAPE;
-  const size_t need = chunk_tensor_ws_bytes(B, Hkv, P0, n, D);
+  const size_t need = chunk_tensor_ws_bytes(B, Hq, Hkv, P0, n, D);
   if (!workspace || workspace_bytes < need) return JL_ERR_WORKSPACE;
   if (reinterpret_cast<uintptr_t>(workspace) % kAlign) return JL_ERR_ALIGN;
   DeviceState *dev = nullptr;
@@ -500,6 +519,8 @@ int chunk_tensor(const void *q, const void *k_cache, const void *v_cache, void *
   a.k_true = reinterpret_cast<__half *>(ws);
   a.k_remote = reinterpret_cast<__half *>(ws + kb);
   a.v_op = reinterpret_cast<__half *>(ws + 2 * kb);
+  a.n_split = chunk_split_count(B, Hq, Hkv, P0, n);
+  a.partial = a.n_split > 1 ? reinterpret_cast<float *>(ws + 3 * kb) : nullptr;
   a.B = B;
   a.Hq = Hq;
   a.Hkv = Hkv;

@@ -158,6 +158,13 @@ struct PrefillArgs {
   int interp;
   float ramp_alpha, ramp_beta;
   unsigned int *dev_error;
+  // Key split (a chunk with few query tiles): n_split > 1 splits each query
+  // tile's key visits into n_split contiguous ranges, one CTA each, which
+  // write unnormalised partial records [B, Lq, Hq, n_split, D + 2] (O, the
+  // base-2 max, the sum) to `partial`; launch_split_merge then forms out and
+  // lse.  n_split = 1: the kernel writes out and lse itself.
+  int n_split;
+  float *partial;
   // Turns per position as 64-bit binary fractions, formed on the host by the
   // key-pass launchers: theta_i / (2 pi) (omega_true), the remote map's
   // (theta_i, or theta'_i under the interpolation map), and the correction
@@ -221,6 +228,12 @@ void decode_plan(int B, int Hkv, int L, int *n_split, int *chunk);
 bool decode_supports_group(int grp);
 
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t stream);
+
+// Log-sum-exp merge of split partial records [B, nq, Hq, n_split, D + 2]
+// (unnormalised O, base-2 max, sum) into out [B, nq, Hq, D] and lse
+// [B, Hq, nq] (lse may be NULL); n_split <= 296.
+cudaError_t launch_split_merge(const float *partial, int n_split, void *out, int out_f32,
+                               float *lse, int B, int nq, int Hq, int D, cudaStream_t stream);
 
 // k_remote[b, j] = FP16(R(f(j) - j) k_cache[b, j]) for j in [j0, j1), all KV heads.
 cudaError_t launch_remote_cache(const __nv_bfloat16 *k_cache, __half *k_remote, int B, int Lcap,

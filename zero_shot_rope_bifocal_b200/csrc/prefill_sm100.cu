@@ -113,6 +113,11 @@ struct Params {
   float *lse;
   int out_f32;
   unsigned int *dev_error;
+  // key split: blockIdx.z = b * n_split + split; with n_split > 1 each CTA
+  // takes a contiguous share of its tile's visits and writes partial
+  // records [B, Lq, Hq, n_split, D + 2] (O unnormalised, m in base 2, l)
+  int n_split;
+  float *partial;
 };
 
 __device__ __forceinline__ float u2f(uint32_t u) { return __uint_as_float(u); }
@@ -239,7 +244,8 @@ bifocal_prefill_kernel(const __grid_constant__ CUtensorMap tm_kt,
   const int qt = prm.n_qt - 1 - static_cast<int>(blockIdx.x);  // longest rows first
   const int g = static_cast<int>(blockIdx.y) / prm.npair;
   const int pr = static_cast<int>(blockIdx.y) - g * prm.npair;
-  const int b = blockIdx.z;
+  const int split = static_cast<int>(blockIdx.z) % prm.n_split;
+  const int b = static_cast<int>(blockIdx.z) / prm.n_split;
   const int head0 = g * prm.grp + 2 * pr;
   const bool has1 = 2 * pr + 1 < prm.grp;
   const int p0 = prm.q_off + qt * BM;  // position of the tile's first row
@@ -275,7 +281,21 @@ bifocal_prefill_kernel(const __grid_constant__ CUtensorMap tm_kt,
     dlo = 0;
     dhi = w0;
   }
-  const int nv = n_rem + (n_kt - kl0);
+  int nv = n_rem + (n_kt - kl0);
+  if (prm.n_split > 1) {
+    // This split's share [v0, v1) of the visits: a remote part (if it
+    // starts before the local visits) and a local part, in the same order.
+    const int v0 = static_cast<int>(static_cast<long long>(nv) * split / prm.n_split);
+    const int v1 = static_cast<int>(static_cast<long long>(nv) * (split + 1) / prm.n_split);
+    if (v0 < n_rem) {
+      kr0 += v0;
+      n_rem = min(n_rem, v1) - v0;
+    } else {
+      kl0 += v0 - n_rem;
+      n_rem = 0;
+    }
+    nv = v1 - v0;
+  }
   const bool switch_q = n_rem > 0 && n_rem < nv;
 
   // A launch that already recorded a failure ends quickly: thread 0 reads the
@@ -566,13 +586,17 @@ bifocal_prefill_kernel(const __grid_constant__ CUtensorMap tm_kt,
       // positions: S(j) was read, so QK(j) is done with the tile.
       if (switch_q && j == n_rem - 1) build_q(false);
     }
-    // ---- epilogue: O / l and the log-sum-exp of this row
+    // ---- epilogue: O / l and the log-sum-exp of this row, or (key split)
+    // the row's partial record
     if (ok) ok = wait_or_abort(bar(LY::kOFull + s), 0u, abort);
     if (__all_sync(0xffffffffu, ok)) {
       tc_fence_after();
       const float inv_l = row_ok ? 1.f / l_sum : 0.f;
       const int head = head0 + s;
-      const size_t obase = ((static_cast<size_t>(b) * prm.Lq + qt * BM + rloc) * prm.Hq + head) * D;
+      const size_t row_head = (static_cast<size_t>(b) * prm.Lq + qt * BM + rloc) * prm.Hq + head;
+      const size_t obase = row_head * D;
+      const bool split_rec = prm.n_split > 1;
+      float *rec = split_rec ? prm.partial + (row_head * prm.n_split + split) * (D + 2) : nullptr;
 #pragma unroll 1
       for (int c = 0; c < D / 32; ++c) {
         uint32_t rr[32];
@@ -581,7 +605,13 @@ bifocal_prefill_kernel(const __grid_constant__ CUtensorMap tm_kt,
         tmem_wait_ld();
         reg_fence(rr);
         if (!row_ok) continue;
-        if (prm.out_f32) {
+        if (split_rec) {
+          // a split without visits (never planned) has no O in TMEM: zeros
+          float2 *dst = reinterpret_cast<float2 *>(rec + c * 32);
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            dst[e] = nv > 0 ? make_float2(u2f(rr[2 * e]), u2f(rr[2 * e + 1])) : make_float2(0.f, 0.f);
+        } else if (prm.out_f32) {
           float4 *dst = reinterpret_cast<float4 *>(reinterpret_cast<float *>(prm.out) + obase + c * 32);
 #pragma unroll
           for (int e = 0; e < 8; ++e)
@@ -602,9 +632,13 @@ bifocal_prefill_kernel(const __grid_constant__ CUtensorMap tm_kt,
           }
         }
       }
-      if (row_ok && prm.lse)
+      if (row_ok && split_rec) {
+        rec[D] = m_used;
+        rec[D + 1] = l_sum;
+      } else if (row_ok && prm.lse) {
         prm.lse[(static_cast<size_t>(b) * prm.Hq + head) * prm.Lq + qt * BM + rloc] =
             (m_used + log2f(l_sum)) * 0.69314718055994531f;
+      }
     }
   }
 
@@ -674,6 +708,8 @@ cudaError_t launch_d(const PrefillArgs &a, cudaStream_t stream) {
   prm.lse = a.lse;
   prm.out_f32 = a.out_f32;
   prm.dev_error = a.dev_error;
+  prm.n_split = a.n_split > 1 ? a.n_split : 1;
+  prm.partial = a.partial;
   prm.q_raw = a.q;
   prm.remote_interp = a.interp;
   const double log_theta = std::log(static_cast<double>(a.theta));
@@ -688,9 +724,12 @@ cudaError_t launch_d(const PrefillArgs &a, cudaStream_t stream) {
   const int smem = Layout<D>::ALLOC;
   cudaError_t e = ensure_smem_limit<bifocal_prefill_kernel<D>>(smem);
   if (e != cudaSuccess) return e;
-  const dim3 grid(prm.n_qt, a.Hkv * prm.npair, a.B);
+  const dim3 grid(prm.n_qt, a.Hkv * prm.npair, a.B * prm.n_split);
   bifocal_prefill_kernel<D><<<grid, kThreads, smem, stream>>>(tkt, tkr, tv, prm);
-  return cudaGetLastError();
+  e = cudaGetLastError();
+  if (e != cudaSuccess || prm.n_split == 1) return e;
+  return launch_split_merge(a.partial, prm.n_split, a.out, a.out_f32, a.lse, a.B, a.Lq, a.Hq, D,
+                            stream);
 }
 
 }  // namespace

@@ -31,6 +31,7 @@ JL_ERR_NO_DEVICE = -8
 JL_ERR_RANGE = -9
 JL_BF16 = 0
 JL_F32 = 1
+CHUNK_TENSOR_MIN = 6  # JL_CHUNK_TENSOR_MIN: chunks this long take the tensor-core path
 
 # Every symbol the header declares, with its ctypes signature.
 _VP, _I, _F, _SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
