@@ -54,8 +54,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # whose code lines' SHA-256 is recorded here; the capture and its command are summarised
 # in the profile named below.  The line reports it only while those sources
 # are unchanged, and null otherwise.
-TRAFFIC_RECORD = {"bytes": 6.12e9, "read_bytes": 4.98e9, "write_bytes": 1.14e9,
-                  "sources_sha256": "f79d1e483ed80ccdc36ef9456c9571bc1f72921f63c5943ae50a9ef765d06e52",
+TRAFFIC_RECORD = {"bytes": 6.11e9, "read_bytes": 4.99e9, "write_bytes": 1.12e9,
+                  "sources_sha256": "ad470d19dfb6e6b21fdd6440826cb275c2c345c2a67b7cf2b5f6b511ceda76e3",
                   "profile": "profiles/prefill_attention_qwen3_8b_L131072_dram.md"}
 TRAFFIC_SOURCES = ("zero_shot_rope_bifocal_b200/csrc/prefill_sm100.cu",
                    "zero_shot_rope_bifocal_b200/csrc/sm100_ptx.cuh")
@@ -145,7 +145,8 @@ def reduce_sum(x: float, world: int, device=None) -> float:
 
 # ---------------------------------------------------------------- clocks
 class ClockSampler:
-    """Samples SM clocks and throttle reasons with nvidia-smi (every 100 ms).
+    """Samples SM clocks and throttle reasons with nvidia-smi (every 25 ms, so
+    that the ~0.7 s prefill region gets about 25 samples).
 
     The sampler starts on entry and waits for its first sample, so that the
     timed region that follows is covered; ``window(t0, t1)`` (times from
@@ -155,7 +156,7 @@ class ClockSampler:
     QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
-    PERIOD_S = 0.1
+    PERIOD_S = 0.025
 
     def __init__(self, gpu_index: int):
         self.gpu = gpu_index
