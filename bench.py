@@ -334,10 +334,12 @@ def run_reference(args):
 L2_BYTES = 126 * 2 ** 20
 
 
-def sweep_prefill(jl, torch, dev, stream, name: str, w0: int | None = None, reps: int = 3) -> dict:
+def sweep_prefill(jl, torch, dev, stream, name: str, w0: int | None = None, reps: int = 5) -> dict:
     """One named prefill workload (the RoPE operand pass plus the attention
     kernel): median per-step and per-kernel times over ``reps`` steps, each
-    preceded by an L2 flush outside the timed events."""
+    preceded by an L2 flush outside the timed events.  Warm-up steps run back
+    to back first, so that the clocks have left their idle state (the first
+    millisecond after an idle gap runs measurably slower)."""
     from zero_shot_rope_bifocal_b200.synth import WORKLOADS, prefill_inputs
     w = WORKLOADS[name] if w0 is None else WORKLOADS[name].with_(w0=w0)
     x = prefill_inputs(w, device=dev)
@@ -355,7 +357,8 @@ def sweep_prefill(jl, torch, dev, stream, name: str, w0: int | None = None, reps
         jl.jetlong_prefill_attend(x.q, out, lse, Hkv, w.w_pretrained, w.w0, w.theta, ws,
                                   stream=stream)
 
-    for _ in range(2):
+    n_warm = max(3, int(20.0 / max(prefill_flops(B, Hq, L, D) / 1e12, 1.0)))  # ~20 ms of work
+    for _ in range(min(n_warm, 50)):
         rotate()
         attend()
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
@@ -928,7 +931,7 @@ def run_native(args):
                 "vs_alias_decode_host_launched": interp_us_tok / host_loop_us},
             "configs": {
                 "what": "each workload of the benchmark plan on this rank: prefill = RoPE operand "
-                        "pass + attention kernel, median of 3 steps after an L2 flush; decode = "
+                        "pass + attention kernel, median of 5 steps after an L2 flush; decode = "
                         "graph replays of 256-step loops",
                 "prefill": [dict(c, attend_frac=c["attend_tflops"] / peak) for c in sweep["prefill"]],
                 "decode": [dict(c, frac=c["achieved_gbs"] / peaks["hbm_gbs"])
