@@ -2,6 +2,7 @@
 
     python -m zero_shot_rope_bifocal_b200.profile_case --case prefill --workload qwen3_8b_64k --L 16384
     python -m zero_shot_rope_bifocal_b200.profile_case --case decode --workload decode_8b_32k
+    python -m zero_shot_rope_bifocal_b200.profile_case --case decode --two-form ...
 
 Inputs are the seeded synthetic ones of ``synth``; sizes default to the named
 workload, ``--L`` overrides the sequence length (keep captures small: a
@@ -27,6 +28,8 @@ def main(argv=None) -> int:
     ap.add_argument("--w0", type=int, default=None)
     ap.add_argument("--w-pretrained", type=int, default=None)
     ap.add_argument("--reps", type=int, default=3)
+    ap.add_argument("--two-form", action="store_true",
+                    help="decode: read remote keys from the FP16 remote form of the cache")
     args = ap.parse_args(argv)
     name = args.workload or ("qwen3_8b_64k" if args.case == "prefill" else "decode_8b_32k")
     w = WORKLOADS[name]
@@ -57,9 +60,17 @@ def main(argv=None) -> int:
         ws = torch.empty(jl.jetlong_decode_workspace_size(w.B, w.Hq, w.Hkv, w.L, w.D),
                          dtype=torch.uint8, device=dev)
 
-        def call():
-            jl.jetlong_decode(d.q, kc, d.v, w.L, w.w_pretrained, w.w0, w.theta, out=out, lse=lse,
-                              workspace=ws)
+        if args.two_form:
+            kr = torch.empty(kc.shape, dtype=torch.float16, device=dev)
+            jl.jetlong_remote_cache(kc, kr, 0, w.L, w.L, w.w_pretrained, w.theta)
+
+            def call():
+                jl.jetlong_decode_two_form(d.q, kc, kr, d.v, w.L, w.w_pretrained, w.w0, w.theta,
+                                           out=out, lse=lse, workspace=ws)
+        else:
+            def call():
+                jl.jetlong_decode(d.q, kc, d.v, w.L, w.w_pretrained, w.w0, w.theta, out=out,
+                                  lse=lse, workspace=ws)
     call()
     torch.cuda.synchronize()
     ev0.record()
