@@ -47,6 +47,10 @@
 // files then allow 168 registers per thread: enough for a whole row.
 // TMEM (512 columns): S0 | S1 | O0 | O1; a row's P (packed FP16) is written
 // over the first 64 columns of its S once the scores are in registers.
+// A chunk with few query tiles splits each tile's visit list into contiguous
+// ranges, one CTA each (grid z): such a CTA writes its rows' unnormalised O
+// with the running max and sum, and a log-sum-exp merge kernel forms the
+// output (launch_split_merge).
 // Each wait is bounded in time (jl::kWaitLimitNs) and also gives up when
 // another role has given up; the CTA then records a device error, drains its
 // MMAs and in-flight copies, frees TMEM and exits.
