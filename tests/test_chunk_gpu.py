@@ -72,6 +72,17 @@ def test_chunk_key_split_every_row(Hq, Hkv, D, wp, w0, P0, n):
     assert_lse(f64(lse), lse_ref, "key split")
 
 
+def test_chunk_key_split_at_the_largest_split_count():
+    # one query tile and one head pair: 148 splits of about one key tile each
+    # (the merge's widest case), G = 5, every row against the oracle
+    w = Workload("chunk_split148", 1, 2, 1, 64, 0, 4096, 1000, 1e4, 71, True, kind="decode")
+    P0, n = 19000, 8
+    assert jl.jetlong_prefill_chunk_workspace_size(1, 2, 1, P0, n, 64) > 3 * (P0 + n) * 64 * 2
+    out, lse, o_ref, lse_ref = run_chunk(w, P0, n)
+    assert_o(f64(out), o_ref, "148 splits")
+    assert_lse(f64(lse), lse_ref, "148 splits")
+
+
 def test_chunk_across_the_appendix_e_boundary_uses_one_group_size():
     # P0 + n = 98,308: G = 4 for every query of the chunk, although a
     # token-by-token decode would use G = 3 for the first four of them.
