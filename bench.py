@@ -55,7 +55,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # in the profile named below.  The line reports it only while those sources
 # are unchanged, and null otherwise.
 TRAFFIC_RECORD = {"bytes": 6.11e9, "read_bytes": 4.99e9, "write_bytes": 1.12e9,
-                  "sources_sha256": "ad470d19dfb6e6b21fdd6440826cb275c2c345c2a67b7cf2b5f6b511ceda76e3",
+                  "sources_sha256": "8bb8601af8afb6a4232bb0c1244219ccfe2f131a13d6cda644cdb4ffa1ba45f9",
                   "profile": "profiles/prefill_attention_qwen3_8b_L131072_dram.md"}
 TRAFFIC_SOURCES = ("zero_shot_rope_bifocal_b200/csrc/prefill_sm100.cu",
                    "zero_shot_rope_bifocal_b200/csrc/sm100_ptx.cuh")
