@@ -73,7 +73,7 @@ constexpr int kMmaWarp = 9;
 // Column pairs per 8 whose exponential runs on the FMA pipe (the rest on the
 // special-function unit, which would otherwise be the softmax's limit).
 #ifndef JL_PREFILL_FMA_PAIRS
-#define JL_PREFILL_FMA_PAIRS 2
+#define JL_PREFILL_FMA_PAIRS 1
 #endif
 constexpr int kFmaPairsPer8 = JL_PREFILL_FMA_PAIRS;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
